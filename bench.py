@@ -1,0 +1,493 @@
+#!/usr/bin/env python
+"""Benchmark: rotated + quantized GB/s and tokens/s on B200, fraction of HBM peak.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c4]
+                    [--impl kq|reference] [--no-extras]
+
+A step is one pass of the hot path over one batch of the workload: load +
+sign, Hadamard butterflies, normalisation folded into the scales, extrema,
+exact scales, 4-bit rounding, nibble packing and stores.  The default
+workload is the 16384 x 4096 bf16 batch with a full-row Hadamard and NVFP4
+output (static fp32 tensor scale, computed once by the dynamic path during
+warm-up; the dynamic two-pass time is reported alongside).
+
+Inputs are resident in HBM before the timed region; consecutive steps cycle
+through enough independent buffer sets that every step reads its input from
+DRAM (the sets together exceed three times the 126 MB L2), so no L2 flush is
+needed between steps.  Times come from CUDA events on the launching stream;
+for N > 1 every rank times its own batch (weak scaling, no data-path
+collective) and the maximum over ranks is reported.
+
+`--impl reference` times the CPU oracle (fp64 dense D.H product + scalar
+quantizer) on the host cores over a bounded sample of rows per step.
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--workload", default="c4")
+    p.add_argument("--impl", default="kq", choices=["kq", "reference"])
+    p.add_argument("--no-extras", action="store_true",
+                   help="skip the per-workload table, dynamic and round-trip timings")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0,
+                   help="target CPU time of the oracle baseline sample")
+    return p.parse_args()
+
+
+# ------------------------------------------------------------------ peaks
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_digest():
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "hadamard_rotated_activation_b200", "csrc", "*"))):
+        with open(f, "rb") as fh:
+            h.update(os.path.basename(f).encode())
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_key):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        e = d[kernel_key]
+        if e.get("source_digest") != source_digest():
+            return None
+        return float(e["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, torch_device):
+        self.ok = False
+        self.samples = []
+        self.reasons = 0
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            h = None
+            try:
+                import torch
+                props = torch.cuda.get_device_properties(torch_device)
+                bus = "%08x:%02x:%02x.0" % (props.pci_domain_id, props.pci_bus_id,
+                                            props.pci_device_id)
+                h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                h = pynvml.nvmlDeviceGetHandleByIndex(0)
+            self.h = h
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def sample(self):
+        if not self.ok:
+            return
+        try:
+            self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+            self.reasons |= int(self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+        except Exception:
+            pass
+
+    def summary(self):
+        names = [n for b, n in self.REASONS.items() if self.reasons & b and b != 0x1]
+        return {
+            "sm_mhz": statistics.median(self.samples) if self.samples else None,
+            "sm_max_mhz": self.max_mhz,
+            "reasons": names,
+            "samples": len(self.samples),
+            "source": "nvml",
+        }
+
+
+# ------------------------------------------------------------- workloads
+def make_step(torch, kq, w, dev_inputs, signs, tensor_scale=None, mode="static"):
+    """Returns (make_set, step(set), kernel launches per step)."""
+    t, n, b = w.tokens, w.dim, w.block
+
+    if w.fmt == "nvfp4":
+        def make_set(x):
+            c, bs, ts, ws = kq.empty_nvfp4(t, n, b)
+            if tensor_scale is not None:
+                ts.fill_(float(tensor_scale))
+            return (x, c, bs, ts, ws)
+
+        if mode == "static":
+            def step(s):
+                kq.kq_rht_quant_nvfp4(s[0], b, signs, s[1], s[2], s[3], None, dynamic=False)
+            launches = 1
+        else:
+            def step(s):
+                kq.kq_rht_quant_nvfp4(s[0], b, signs, s[1], s[2], s[3], s[4], dynamic=True)
+            launches = 3
+    elif w.fmt == "int4_sym":
+        def make_set(x):
+            return (x,) + kq.empty_int4_sym(t, n)
+
+        def step(s):
+            kq.kq_rht_quant_int4(s[0], b, signs, 0, False, s[1], s[2])
+        launches = 1
+    else:
+        def make_set(x):
+            return (x,) + kq.empty_int4_asym(t, n, w.group)
+
+        def step(s):
+            kq.kq_rht_quant_int4(s[0], b, signs, w.group, True, s[1], s[2], s[3])
+        launches = 1
+    return make_set, step, launches
+
+
+def device_input(torch, inp, wl, dev):
+    import numpy as np
+    if inp.workload.dtype == wl.BF16:
+        return torch.from_numpy(inp.stored.view(np.int16)).to(dev).view(torch.bfloat16)
+    return torch.from_numpy(inp.stored).to(dev)
+
+
+def n_sets(bytes_per_set):
+    return max(2, -(-3 * L2_BYTES // max(bytes_per_set, 1)))
+
+
+def time_steps(torch, step, sets, k, warmup, sampler=None, stream=None):
+    for i in range(warmup):
+        step(sets[i % len(sets)])
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(k):
+        step(sets[i % len(sets)])
+    end.record(stream)
+    if sampler is not None:
+        while not end.query():
+            sampler.sample()
+            time.sleep(0.0002)
+    torch.cuda.synchronize()
+    return start.elapsed_time(end)
+
+
+# -------------------------------------------------------------- CPU oracle
+def oracle_step(oracle_mod, wl, inp_rows, w):
+    y = oracle_mod.rht(inp_rows.values, inp_rows.signs, w.block)
+    if w.fmt == wl.NVFP4:
+        oracle_mod.nvfp4(y)
+    elif w.fmt == wl.INT4_SYM:
+        oracle_mod.int4_sym_per_token(y)
+    else:
+        oracle_mod.int4_asym_group(y, w.group)
+
+
+def cpu_sample_rows(oracle_mod, wl, w, seconds):
+    """Rows of the workload the oracle handles in about `seconds`."""
+    probe = wl.make_inputs(w, tokens=4)
+    oracle_step(oracle_mod, wl, probe, w)          # builds and caches H
+    t0 = time.perf_counter()
+    oracle_step(oracle_mod, wl, probe, w)
+    per_row = max((time.perf_counter() - t0) / 4, 1e-6)
+    return int(max(4, min(w.tokens, seconds / per_row)))
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max(int(i.get("num_threads", 1)) for i in threadpool_info()) or 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_cpu_baseline(w, seconds):
+    import oracle as oracle_mod
+    from hadamard_rotated_activation_b200 import workloads as wl
+    rows = cpu_sample_rows(oracle_mod, wl, w, seconds)
+    inp = wl.make_inputs(w, tokens=rows)
+    t0 = time.perf_counter()
+    oracle_step(oracle_mod, wl, inp, w)
+    dt = time.perf_counter() - t0
+    wb = w.with_tokens(rows)
+    return {
+        "value": round(wb.algorithmic_bytes() / dt / 1e9, 6),
+        "unit": "GB/s",
+        "tokens_per_s": round(rows / dt, 3),
+        "cores": cpu_threads(),
+        "kind": "oracle",
+        "sample": f"{rows} of {w.tokens} rows of workload {w.key} "
+                  f"(fp64 dense D.H + scalar quantizer), {dt:.2f} s wall",
+    }
+
+
+def run_reference(args, rank, world):
+    """--impl reference: the CPU oracle, timed on the host cores."""
+    if rank != 0:
+        return
+    import oracle as oracle_mod
+    from hadamard_rotated_activation_b200 import workloads as wl
+    w = wl.WORKLOADS[args.workload]
+    per_step_s = max(2.0, min(20.0, 150.0 / max(args.steps + args.warmup, 1)))
+    rows = cpu_sample_rows(oracle_mod, wl, w, per_step_s)
+    inp = wl.make_inputs(w, tokens=rows)
+    for _ in range(args.warmup):
+        oracle_step(oracle_mod, wl, inp, w)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(oracle_mod, wl, inp, w)
+    dt = (time.perf_counter() - t0) / max(args.steps, 1)
+    wb = w.with_tokens(rows)
+    gbs = wb.algorithmic_bytes() / dt / 1e9
+    line = {
+        "impl": "reference",
+        "metric": "rotated+quantized GB/s (algorithmic bytes)",
+        "value": round(gbs, 6), "unit": "GB/s", "n_gpus": 0, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, sample_rows=rows),
+        "tokens_per_s": round(rows / dt, 3),
+        "cpu_baseline": {"value": round(gbs, 6), "unit": "GB/s", "cores": cpu_threads(),
+                         "kind": "oracle",
+                         "sample": f"{rows} of {w.tokens} rows per step"},
+        "e2e": {"value": round(gbs, 6), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w, **extra):
+    d = {
+        "workload": f"{w.key}: {w.description}",
+        "tokens": w.tokens, "dim": w.dim, "block": w.block,
+        "input_dtype": w.dtype, "format": w.fmt, "seed": w.seed,
+        "global_batch": w.tokens, "seq_len": None, "parallelism": "dp (independent batches)",
+    }
+    d.update(extra)
+    return d
+
+
+# ------------------------------------------------------------------ main
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import numpy as np
+    import torch
+    import hadamard_rotated_activation_b200 as kq
+    from hadamard_rotated_activation_b200 import workloads as wl
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    kq.lib()
+
+    w = wl.WORKLOADS[args.workload]
+    peak, peak_kind = measured_peaks()
+    # every rank draws its own batch (weak scaling)
+    inp = wl.make_inputs(w, seed=w.seed + 1000 * rank)
+    x0 = device_input(torch, inp, wl, dev)
+    signs = None if inp.signs is None else torch.from_numpy(inp.signs).to(dev)
+
+    # tensor scale for the static NVFP4 step: the dynamic path's own result
+    tscale = None
+    if w.fmt == wl.NVFP4:
+        c, bs, ts, ws = kq.empty_nvfp4(w.tokens, w.dim, w.block)
+        kq.kq_rht_quant_nvfp4(x0, w.block, signs, c, bs, ts, ws, dynamic=True)
+        torch.cuda.synchronize()
+        tscale = float(ts.item())
+        del c, bs, ts, ws
+
+    make_set, step, launches = make_step(torch, kq, w, None, signs, tscale, "static")
+    set_bytes = w.algorithmic_bytes()
+    sets = [make_set(x0 if i == 0 else x0.clone()) for i in range(n_sets(set_bytes))]
+
+    sampler = ClockSampler(dev)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    ms = time_steps(torch, step, sets, args.steps, args.warmup, sampler, stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+        tt = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    ms_step = ms / max(args.steps, 1)
+    alg = w.algorithmic_bytes()
+    gbs_rank = alg / (ms_step * 1e-3) / 1e9
+    value = gbs_rank * world
+    tokens_s = w.tokens * world / (ms_step * 1e-3)
+
+    # ---- end to end through the public API: pinned host in, host out
+    x_host = torch.from_numpy(inp.stored.view(np.int16) if w.dtype == wl.BF16
+                              else inp.stored).pin_memory()
+    e2e_set = make_set(torch.empty_like(x0))
+    outs_host = [torch.empty(o.shape, dtype=o.dtype).pin_memory()
+                 for o in e2e_set[1:3]]
+    in_bytes = x_host.numel() * x_host.element_size()
+    out_bytes = sum(o.numel() * o.element_size() for o in outs_host)
+
+    def e2e_step(_s):
+        dst = e2e_set[0].view(torch.int16) if w.dtype == wl.BF16 else e2e_set[0]
+        dst.copy_(x_host, non_blocking=True)
+        step(e2e_set)
+        for h, d in zip(outs_host, e2e_set[1:3]):
+            h.copy_(d, non_blocking=True)
+
+    k_e2e = max(3, min(args.steps, 50))
+    ms_e2e = time_steps(torch, e2e_step, [None], k_e2e, max(3, min(args.warmup, 5)))
+    if dist is not None:
+        tt = torch.tensor([ms_e2e], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_e2e = float(tt.item())
+    e2e_gbs = alg * world / (ms_e2e / k_e2e * 1e-3) / 1e9
+
+    kernel_key = f"{w.key}_{w.fmt}_static" if w.fmt == wl.NVFP4 else f"{w.key}_{w.fmt}"
+    traffic = ncu_traffic(kernel_key)
+    line = {
+        "metric": "rotated+quantized GB/s (algorithmic bytes: input read + codes/scales written)",
+        "value": round(value, 3), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 6),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic",
+        "config": workload_config(w, l2="inputs larger than L2: %d rotating buffer sets"
+                                  % len(sets),
+                                  tensor_scale="static (computed once by the dynamic path)"
+                                  if w.fmt == wl.NVFP4 else None),
+        "tokens_per_s": round(tokens_s, 1),
+        "frac_of_hbm_peak": round(gbs_rank / peak, 4),
+        "gpu_launches": launches * args.steps,
+        "clocks": sampler.summary(),
+        "roofline": {
+            "bound": "hbm", "achieved": round(gbs_rank, 3), "peak": peak, "unit": "GB/s",
+            "frac": round(gbs_rank / peak, 4), "peak_kind": peak_kind,
+            "traffic": None if traffic is None else round(traffic),
+            "kernel": kernel_key,
+            "bytes_per_launch": alg,
+        },
+        "e2e": {"value": round(e2e_gbs, 3), "unit": "GB/s",
+                "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": out_bytes,
+                "ms_per_step": round(ms_e2e / k_e2e, 4)},
+    }
+
+    if not args.no_extras and rank == 0:
+        line["per_workload"] = extras(torch, kq, wl, dev, peak, args)
+    if not args.no_cpu_baseline and rank == 0 and world == 1:
+        line["cpu_baseline"] = run_cpu_baseline(w, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def extras(torch, kq, wl, dev, peak, args):
+    """Per-workload forward timings (all five), NVFP4 dynamic, and the c4
+    dequant + inverse round trip.  Not part of the headline value."""
+    import numpy as np
+    out = {}
+    k = max(20, min(args.steps, 200))
+    for key, w in wl.WORKLOADS.items():
+        inp = wl.make_inputs(w)
+        x0 = device_input(torch, inp, wl, dev)
+        signs = None if inp.signs is None else torch.from_numpy(inp.signs).to(dev)
+        modes = ["static", "dynamic"] if w.fmt == wl.NVFP4 else ["-"]
+        tscale = None
+        if w.fmt == wl.NVFP4:
+            c, bs, ts, ws = kq.empty_nvfp4(w.tokens, w.dim, w.block)
+            kq.kq_rht_quant_nvfp4(x0, w.block, signs, c, bs, ts, ws, dynamic=True)
+            torch.cuda.synchronize()
+            tscale = float(ts.item())
+        for mode in modes:
+            make_set, step, launches = make_step(torch, kq, w, None, signs, tscale,
+                                                 mode if mode != "-" else "static")
+            nset = n_sets(w.algorithmic_bytes())
+            sets = [make_set(x0 if i == 0 else x0.clone()) for i in range(nset)]
+            ms = time_steps(torch, step, sets, k, 5) / k
+            alg = w.algorithmic_bytes()
+            gbs = alg / (ms * 1e-3) / 1e9
+            name = key if mode == "-" else f"{key}_{mode}"
+            out[name] = {"ms": round(ms, 5), "GB/s": round(gbs, 2),
+                         "frac": round(gbs / peak, 4),
+                         "tokens_per_s": round(w.tokens / (ms * 1e-3), 1),
+                         "launches_per_step": launches,
+                         "bytes": alg}
+            del sets
+        if key == "c4":
+            # round trip: dequant + inverse rotation
+            c, bs, ts, ws = kq.empty_nvfp4(w.tokens, w.dim, w.block)
+            kq.kq_rht_quant_nvfp4(x0, w.block, signs, c, bs, ts, ws, dynamic=True)
+            deq = torch.empty((w.tokens, w.dim), dtype=torch.float32, device=dev)
+            back = torch.empty_like(deq)
+
+            def rt(_s):
+                kq.kq_dequant(kq.KQ_FMT_NVFP4, c, bs, None, ts, w.tokens, w.dim, 0, deq)
+                kq.kq_rht(deq, w.block, signs, back, inverse=True)
+            ms = time_steps(torch, rt, [None], 20, 3) / 20
+            rbytes = (w.tokens * w.dim // 2 + w.tokens * w.dim // 16) + 2 * 4 * w.tokens * w.dim \
+                + 4 * w.tokens * w.dim
+            out["c4_roundtrip"] = {"ms": round(ms, 5),
+                                   "GB/s": round(rbytes / (ms * 1e-3) / 1e9, 2),
+                                   "bytes": rbytes,
+                                   "launches_per_step": 2}
+        del x0
+        torch.cuda.empty_cache()
+    return out
+
+
+if __name__ == "__main__":
+    main()

@@ -1,1 +1,196 @@
-"""Fused randomized Hadamard rotation + 4-bit quantization of activations (B200)."""
+"""Fused randomized Hadamard rotation + 4-bit quantization of activations (B200).
+
+Thin ctypes binding over the C ABI in include/kq.h (libkq.so, built in-tree by
+`python -m hadamard_rotated_activation_b200.build`).  Functions carry the C
+names and only marshal arguments: torch CUDA tensors become device pointers and
+the current torch stream becomes the kq stream.  Every step of the path runs in
+the library's CUDA kernels; there is no other implementation here, and a
+missing library is an error.
+
+PyTorch is used for device memory and streams only.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libkq.so")
+
+KQ_OK = 0
+KQ_ERR_INVALID_ARG = -1
+KQ_ERR_UNSUPPORTED = -2
+KQ_ERR_MISALIGNED = -3
+KQ_ERR_CUDA = -4
+
+KQ_F32 = 0
+KQ_BF16 = 1
+
+KQ_INVERSE = 1
+KQ_SCALE_STATIC = 2
+KQ_SCALE_DYNAMIC = 4
+
+KQ_FMT_INT4_SYM = 0
+KQ_FMT_INT4_ASYM = 1
+KQ_FMT_NVFP4 = 2
+
+C_SYMBOLS = (
+    "kq_rht", "kq_rht_quant_int4", "kq_rht_quant_nvfp4", "kq_dequant",
+    "kq_workspace_size", "kq_status_str", "kq_last_cuda_error", "kq_version",
+)
+
+_lib = None
+
+
+class KQError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        msg = f"{where}: {status_str(status)} ({status})"
+        if status == KQ_ERR_CUDA:
+            msg += f", cuda error {lib().kq_last_cuda_error()}"
+        super().__init__(msg)
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """Load libkq.so (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"{LIB_PATH} is missing: build it with "
+            "`python -m hadamard_rotated_activation_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+    L.kq_rht.argtypes = [vp, i32, i64, i32, i32, vp, vp, i32, vp]
+    L.kq_rht.restype = i32
+    L.kq_rht_quant_int4.argtypes = [vp, i32, i64, i32, i32, vp, i32, i32, vp, vp, vp, vp]
+    L.kq_rht_quant_int4.restype = i32
+    L.kq_rht_quant_nvfp4.argtypes = [vp, i32, i64, i32, i32, vp, vp, vp, vp, vp, sz, i32, vp]
+    L.kq_rht_quant_nvfp4.restype = i32
+    L.kq_dequant.argtypes = [i32, vp, vp, vp, vp, i64, i32, i32, vp, vp]
+    L.kq_dequant.restype = i32
+    L.kq_workspace_size.argtypes = [i64, i32, i32]
+    L.kq_workspace_size.restype = sz
+    L.kq_status_str.argtypes = [i32]
+    L.kq_status_str.restype = ctypes.c_char_p
+    L.kq_last_cuda_error.argtypes = []
+    L.kq_last_cuda_error.restype = i32
+    L.kq_version.argtypes = []
+    L.kq_version.restype = i32
+    _lib = L
+    return L
+
+
+def status_str(status: int) -> str:
+    return lib().kq_status_str(int(status)).decode()
+
+
+# ------------------------------------------------------------ marshalling
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_cuda:
+        raise ValueError("kq functions take CUDA tensors (device pointers)")
+    if not t.is_contiguous():
+        raise ValueError("kq functions take contiguous tensors")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _dtype_code(x) -> int:
+    import torch
+    if x.dtype == torch.bfloat16:
+        return KQ_BF16
+    if x.dtype == torch.float32:
+        return KQ_F32
+    raise ValueError(f"unsupported input dtype {x.dtype}")
+
+
+def _check(status: int, where: str) -> None:
+    if status != KQ_OK:
+        raise KQError(status, where)
+
+
+# -------------------------------------------------------------- C names
+def kq_rht(x, block: int, signs, out, inverse: bool = False, stream=None) -> None:
+    """Rotation only (fp32 out): forward y = x D H^T / sqrt(b), or the inverse."""
+    t, n = x.shape
+    _check(lib().kq_rht(_ptr(x), _dtype_code(x), t, n, block, _ptr(signs), _ptr(out),
+                        KQ_INVERSE if inverse else 0, _stream(stream)), "kq_rht")
+
+
+def kq_rht_quant_int4(x, block: int, signs, group: int, asym: bool, codes, scales,
+                      zeros=None, stream=None) -> None:
+    """Rotation + INT4: symmetric per token (group 0, fp32 scales) or
+    asymmetric per group of 128 (fp16 scales and zero-points)."""
+    t, n = x.shape
+    _check(lib().kq_rht_quant_int4(_ptr(x), _dtype_code(x), t, n, block, _ptr(signs),
+                                   group, 1 if asym else 0, _ptr(codes), _ptr(scales),
+                                   _ptr(zeros), _stream(stream)), "kq_rht_quant_int4")
+
+
+def kq_rht_quant_nvfp4(x, block: int, signs, codes, block_scales, tensor_scale,
+                       workspace=None, dynamic: bool = True, stream=None) -> None:
+    """Rotation + NVFP4 (E2M1 codes, E4M3 scale per 16, fp32 tensor scale).
+    dynamic=True computes and writes the tensor scale (needs `workspace` of
+    kq_workspace_size bytes); dynamic=False reads it."""
+    t, n = x.shape
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    flags = KQ_SCALE_DYNAMIC if dynamic else KQ_SCALE_STATIC
+    _check(lib().kq_rht_quant_nvfp4(_ptr(x), _dtype_code(x), t, n, block, _ptr(signs),
+                                    _ptr(codes), _ptr(block_scales), _ptr(tensor_scale),
+                                    _ptr(workspace), ws_bytes, flags, _stream(stream)),
+           "kq_rht_quant_nvfp4")
+
+
+def kq_dequant(fmt: int, codes, scales, zeros, tensor_scale, tokens: int, dim: int,
+               group: int, out, stream=None) -> None:
+    """Codes and scales back to fp32 (exact product, one rounding)."""
+    _check(lib().kq_dequant(fmt, _ptr(codes), _ptr(scales), _ptr(zeros),
+                            _ptr(tensor_scale), tokens, dim, group, _ptr(out),
+                            _stream(stream)), "kq_dequant")
+
+
+def kq_workspace_size(tokens: int, dim: int, block: int) -> int:
+    return int(lib().kq_workspace_size(tokens, dim, block))
+
+
+def kq_version() -> int:
+    return int(lib().kq_version())
+
+
+# ------------------------------------------------- output allocation helpers
+def empty_int4_sym(tokens: int, dim: int, device="cuda"):
+    import torch
+    return (torch.empty((tokens, dim // 2), dtype=torch.uint8, device=device),
+            torch.empty((tokens,), dtype=torch.float32, device=device))
+
+
+def empty_int4_asym(tokens: int, dim: int, group: int = 128, device="cuda"):
+    import torch
+    g = dim // group
+    return (torch.empty((tokens, dim // 2), dtype=torch.uint8, device=device),
+            torch.empty((tokens, g), dtype=torch.float16, device=device),
+            torch.empty((tokens, g), dtype=torch.float16, device=device))
+
+
+def empty_nvfp4(tokens: int, dim: int, block: int = 0, device="cuda"):
+    """(codes, block_scales, tensor_scale, workspace) for kq_rht_quant_nvfp4."""
+    import torch
+    ws = kq_workspace_size(tokens, dim, block)
+    return (torch.empty((tokens, dim // 2), dtype=torch.uint8, device=device),
+            torch.empty((tokens, dim // 16), dtype=torch.uint8, device=device),
+            torch.empty((1,), dtype=torch.float32, device=device),
+            torch.empty((max(ws, 16),), dtype=torch.uint8, device=device))

@@ -1,0 +1,188 @@
+// C ABI of the kq library: host-side validation and dispatch (see include/kq.h).
+//
+// Every argument is checked here, before anything is enqueued; a rejected call
+// leaves the stream untouched.  The library allocates nothing.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "kq.h"
+#include "kq_internal.h"
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+bool is_pow2(int64_t v) { return v > 0 && (v & (v - 1)) == 0; }
+
+int ilog2(int64_t v) {
+  int r = 0;
+  while ((int64_t(1) << (r + 1)) <= v) ++r;
+  return r;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// Validates (dim, block) and fills the transform geometry.
+kq_status make_geometry(int dim, int block, kq::Geometry* g) {
+  const bool pow2 = is_pow2(dim) && dim >= 32 && dim <= 16384;
+  const bool paley = (dim % 12 == 0) && is_pow2(dim / 12) && dim >= 384 && dim <= 12288;
+  if (!pow2 && !paley) return KQ_ERR_UNSUPPORTED;
+  int b = dim;
+  if (block != 0) {
+    if (block < 16 || !is_pow2(block) || block > dim || dim % block != 0)
+      return KQ_ERR_UNSUPPORTED;
+    b = block;
+  }
+  g->n = dim;
+  g->b = b;
+  g->paley = (b % 12 == 0 && !is_pow2(b)) ? 1 : 0;
+  g->m = g->paley ? b / 12 : b;
+  g->depth = ilog2(g->m) + (g->paley ? 11 : 0);
+  g->sqrt_b = std::sqrt((double)b);
+  g->inv_sqrt_b = (float)(1.0 / g->sqrt_b);
+  return KQ_OK;
+}
+
+kq_status check_common(const void* x, int dtype, int64_t tokens, int dim, int block,
+                       const int8_t* signs, kq::Geometry* g) {
+  if (!x || tokens < 0) return KQ_ERR_INVALID_ARG;
+  if (dtype != KQ_F32 && dtype != KQ_BF16) return KQ_ERR_UNSUPPORTED;
+  const kq_status st = make_geometry(dim, block, g);
+  if (st != KQ_OK) return st;
+  if (!aligned(x, 16)) return KQ_ERR_MISALIGNED;
+  if (signs && !aligned(signs, 8)) return KQ_ERR_MISALIGNED;
+  return KQ_OK;
+}
+
+kq_status finish(cudaError_t e) {
+  if (e != cudaSuccess) {
+    g_last_cuda_error = (int)e;
+    return KQ_ERR_CUDA;
+  }
+  return KQ_OK;
+}
+
+size_t nv_workspace_bytes(int64_t tokens) {
+  return kq::kNvWorkspaceHeader + (size_t)tokens * sizeof(float2);
+}
+
+}  // namespace
+
+extern "C" {
+
+KQ_API kq_status kq_rht(const void* x, int dtype, int64_t tokens, int dim, int block,
+                        const int8_t* signs, float* out, int flags, kq_stream_t stream) {
+  kq::Geometry g;
+  kq_status st = check_common(x, dtype, tokens, dim, block, signs, &g);
+  if (st != KQ_OK) return st;
+  if (!out) return KQ_ERR_INVALID_ARG;
+  if (flags & ~KQ_INVERSE) return KQ_ERR_INVALID_ARG;
+  if (!aligned(out, 16)) return KQ_ERR_MISALIGNED;
+  if (tokens == 0) return KQ_OK;
+  return finish(kq::launch_rht(x, dtype, tokens, g, signs, out, (flags & KQ_INVERSE) ? 1 : 0,
+                               reinterpret_cast<cudaStream_t>(stream)));
+}
+
+KQ_API kq_status kq_rht_quant_int4(const void* x, int dtype, int64_t tokens, int dim,
+                                   int block, const int8_t* signs, int group, int asym,
+                                   uint8_t* codes, void* scales, void* zeros,
+                                   kq_stream_t stream) {
+  kq::Geometry g;
+  kq_status st = check_common(x, dtype, tokens, dim, block, signs, &g);
+  if (st != KQ_OK) return st;
+  if (!codes || !scales) return KQ_ERR_INVALID_ARG;
+  if (asym != 0 && asym != 1) return KQ_ERR_INVALID_ARG;
+  if (asym == 0) {
+    if (group != 0) return KQ_ERR_UNSUPPORTED;
+    if (zeros) return KQ_ERR_INVALID_ARG;
+    if (!aligned(scales, 4)) return KQ_ERR_MISALIGNED;
+  } else {
+    if (group != 128 || dim % group != 0) return KQ_ERR_UNSUPPORTED;
+    if (!zeros) return KQ_ERR_INVALID_ARG;
+    if (!aligned(scales, 2) || !aligned(zeros, 2)) return KQ_ERR_MISALIGNED;
+  }
+  if (!aligned(codes, 16)) return KQ_ERR_MISALIGNED;
+  if (tokens == 0) return KQ_OK;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (asym == 0)
+    return finish(kq::launch_int4_sym(x, dtype, tokens, g, signs, codes,
+                                      static_cast<float*>(scales), s));
+  return finish(kq::launch_int4_asym(x, dtype, tokens, g, signs, group, codes,
+                                     static_cast<uint16_t*>(scales),
+                                     static_cast<uint16_t*>(zeros), s));
+}
+
+KQ_API kq_status kq_rht_quant_nvfp4(const void* x, int dtype, int64_t tokens, int dim,
+                                    int block, const int8_t* signs, uint8_t* codes,
+                                    uint8_t* block_scales, float* tensor_scale,
+                                    void* workspace, size_t ws_bytes, int flags,
+                                    kq_stream_t stream) {
+  kq::Geometry g;
+  kq_status st = check_common(x, dtype, tokens, dim, block, signs, &g);
+  if (st != KQ_OK) return st;
+  if (!codes || !block_scales || !tensor_scale) return KQ_ERR_INVALID_ARG;
+  const int mode = flags & (KQ_SCALE_STATIC | KQ_SCALE_DYNAMIC);
+  if ((flags & ~(KQ_SCALE_STATIC | KQ_SCALE_DYNAMIC)) != 0) return KQ_ERR_INVALID_ARG;
+  if (mode != KQ_SCALE_STATIC && mode != KQ_SCALE_DYNAMIC) return KQ_ERR_INVALID_ARG;
+  if (!aligned(codes, 16) || !aligned(tensor_scale, 4)) return KQ_ERR_MISALIGNED;
+  kq::NvWorkspace* ws = nullptr;
+  if (mode == KQ_SCALE_DYNAMIC) {
+    if (!workspace || ws_bytes < nv_workspace_bytes(tokens)) return KQ_ERR_INVALID_ARG;
+    if (!aligned(workspace, 16)) return KQ_ERR_MISALIGNED;
+    ws = static_cast<kq::NvWorkspace*>(workspace);
+  }
+  if (tokens == 0) return KQ_OK;
+  return finish(kq::launch_nvfp4(x, dtype, tokens, g, signs, codes, block_scales,
+                                 tensor_scale, ws, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+KQ_API kq_status kq_dequant(int fmt, const uint8_t* codes, const void* scales,
+                            const void* zeros, const float* tensor_scale, int64_t tokens,
+                            int dim, int group, float* out, kq_stream_t stream) {
+  if (!codes || !scales || !out || tokens < 0) return KQ_ERR_INVALID_ARG;
+  if (dim <= 0 || dim % 32 != 0) return KQ_ERR_UNSUPPORTED;
+  if (!aligned(codes, 16) || !aligned(out, 16)) return KQ_ERR_MISALIGNED;
+  switch (fmt) {
+    case KQ_FMT_INT4_SYM:
+      if (!aligned(scales, 4)) return KQ_ERR_MISALIGNED;
+      break;
+    case KQ_FMT_INT4_ASYM:
+      if (group != 128 || dim % group != 0) return KQ_ERR_UNSUPPORTED;
+      if (!zeros) return KQ_ERR_INVALID_ARG;
+      if (!aligned(scales, 2) || !aligned(zeros, 2)) return KQ_ERR_MISALIGNED;
+      break;
+    case KQ_FMT_NVFP4:
+      if (!tensor_scale) return KQ_ERR_INVALID_ARG;
+      if (!aligned(tensor_scale, 4)) return KQ_ERR_MISALIGNED;
+      break;
+    default:
+      return KQ_ERR_INVALID_ARG;
+  }
+  if (tokens == 0) return KQ_OK;
+  return finish(kq::launch_dequant(fmt, codes, scales, zeros, tensor_scale, tokens, dim,
+                                   group, out, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+KQ_API size_t kq_workspace_size(int64_t tokens, int dim, int block) {
+  kq::Geometry g;
+  if (tokens < 0 || make_geometry(dim, block, &g) != KQ_OK) return 0;
+  return nv_workspace_bytes(tokens);
+}
+
+KQ_API const char* kq_status_str(int status) {
+  switch (status) {
+    case KQ_OK: return "KQ_OK";
+    case KQ_ERR_INVALID_ARG: return "KQ_ERR_INVALID_ARG";
+    case KQ_ERR_UNSUPPORTED: return "KQ_ERR_UNSUPPORTED";
+    case KQ_ERR_MISALIGNED: return "KQ_ERR_MISALIGNED";
+    case KQ_ERR_CUDA: return "KQ_ERR_CUDA";
+    default: return "KQ_ERR_UNKNOWN";
+  }
+}
+
+KQ_API int kq_last_cuda_error(void) { return g_last_cuda_error; }
+
+KQ_API int kq_version(void) { return (1 << 16) | 0; }
+
+}  // extern "C"

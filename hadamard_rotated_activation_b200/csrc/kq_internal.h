@@ -1,0 +1,38 @@
+// Internal interface between the C ABI (kq_api.cu) and the kernel files.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "kq_device.cuh"
+
+namespace kq {
+
+// Workspace of the dynamic NVFP4 tensor scale.
+//   lower_bits: fp32 bits of a lower bound on max|S| over the tensor
+//   gmax_bits:  fp64 bits of the exact max|S| (unnormalised)
+//   rows[t]:    (computed row max |S_hat|, error bound) per row
+struct NvWorkspace {
+  unsigned int lower_bits;
+  unsigned int pad_;
+  unsigned long long gmax_bits;
+  float2 rows[1];
+};
+constexpr size_t kNvWorkspaceHeader = 16;
+
+cudaError_t launch_rht(const void* x, int dtype, int64_t tokens, const Geometry& g,
+                       const int8_t* signs, float* out, int inverse, cudaStream_t s);
+cudaError_t launch_int4_sym(const void* x, int dtype, int64_t tokens, const Geometry& g,
+                            const int8_t* signs, uint8_t* codes, float* scales,
+                            cudaStream_t s);
+cudaError_t launch_int4_asym(const void* x, int dtype, int64_t tokens, const Geometry& g,
+                             const int8_t* signs, int group, uint8_t* codes,
+                             uint16_t* scales, uint16_t* zeros, cudaStream_t s);
+cudaError_t launch_nvfp4(const void* x, int dtype, int64_t tokens, const Geometry& g,
+                         const int8_t* signs, uint8_t* codes, uint8_t* bscales,
+                         float* tensor_scale, NvWorkspace* ws, cudaStream_t s);
+cudaError_t launch_dequant(int fmt, const uint8_t* codes, const void* scales,
+                           const void* zeros, const float* tensor_scale, int64_t tokens,
+                           int n, int group, float* out, cudaStream_t s);
+
+}  // namespace kq

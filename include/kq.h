@@ -1,0 +1,198 @@
+/*
+ * kq.h -- C ABI of the fused randomized Hadamard rotation + 4-bit
+ * quantization library for NVIDIA B200 (sm_100a).
+ *
+ * What the library computes
+ * -------------------------
+ * The randomized Hadamard transform (RHT) of activation rows followed by a
+ * 4-bit quantizer, as discussed on these pages:
+ *   - "QuaRot: Outlier-Free 4-Bit Inference in Rotated LLMs" (OpenReview
+ *     reviews): review 1 Summary (online Hadamard run with the fast
+ *     Walsh-Hadamard algorithm), review 2 Summary (the RHT is invertible up to
+ *     machine epsilon; activations are then rounded to nearest INT4),
+ *     review 3 Questions (the Hadamard block computes Y = X H^T), final
+ *     comments (RHT per batch of tokens = data parallel; RHT for the KV cache).
+ *   - "Bug: Qwen3-8B integration issue" (KronQ issue #2), Model Details table:
+ *     12288 = 12 x 1024 is Hadamard-compatible.
+ *   - "Methodology checks for NVFP4 W4A4 on Qwen3-8B" (forum thread):
+ *     block-Hadamard-128 (discrete_descent's note) and NVFP4 at 4.50 bits per
+ *     element (krylov_schur section 3 table).
+ *
+ * Rotation.  For a row x of `dim` values, a +-1 sign vector s (the diagonal D)
+ * and Hadamard blocks of width b (b = dim when block == 0):
+ *     y_i = (1/sqrt(b)) * sum_j H_b[i][j] * s_j * x_j      (inside each block)
+ * H_b is the Sylvester-Hadamard matrix in natural order,
+ * H[i][j] = (-1)^popcount(i & j), when b is a power of two, and
+ * Paley-12 (construction I, q = 11) kron Sylvester(b/12) when b = 12 * 2^k
+ * (full-row mode only).  The inverse is x_j = s_j * sum_i H_b[i][j] y_i / sqrt(b).
+ *
+ * Quantizers (readings of points the pages leave open are noted):
+ *   INT4 symmetric per token: scale = fp32(amax_row / 7), q = clamp(rint(y /
+ *     scale), -8, 7), ties to even.  A zero row has scale 0 and codes 0.
+ *   INT4 asymmetric per group of `group` elements: scale = fp16((max - min) /
+ *     15), z = rint(-min / scale) stored as fp16, u = clamp(rint(y / scale) + z,
+ *     0, 15).
+ *   NVFP4: tensor scale t = fp32(amax_tensor / 2688) (2688 = 6 * 448) when
+ *     dynamic, else supplied; per 16 elements r = fp32(amax_16 / (6 t)),
+ *     block scale s_b = E4M3(r) (nearest even, saturating at 448), codes =
+ *     E2M1(y / (value(s_b) * t)) (nearest even, saturating at 6), sign bit set
+ *     when y < 0.
+ *   Scales are computed from the exact rotated values (the library recomputes
+ *   the deciding elements in fp64 when its fp32 transform cannot decide the
+ *   rounding), so they equal an fp64 evaluation of the formulas bit for bit.
+ *
+ * Layouts (all row-major, no padding between rows):
+ *   x            [tokens, dim] of fp32 or bf16 (kq_dtype).
+ *   out          [tokens, dim] fp32.
+ *   codes        [tokens, dim/2] bytes; element 2k in bits 0-3, 2k+1 in
+ *                bits 4-7.  INT4 symmetric: two's complement nibble.
+ *                INT4 asymmetric: 0..15.  NVFP4: E2M1 (bit 3 = sign).
+ *   INT4 sym scales   fp32 [tokens].
+ *   INT4 asym scales  fp16 [tokens, dim/group], zeros fp16 [tokens, dim/group].
+ *   NVFP4 block_scales E4M3 bytes [tokens, dim/16]; tensor_scale one fp32.
+ *   signs        int8 [dim] of +1/-1, or NULL (no D).
+ *
+ * Ownership and execution: every pointer is a device pointer owned by the
+ * caller.  The library never allocates, frees, synchronizes, or keeps a pointer
+ * after a call returns.  Work is enqueued on `stream` (NULL = the legacy
+ * default stream) and runs asynchronously.  Calls are safe from several host
+ * threads on different streams; outputs of calls that overlap on the GPU must
+ * not alias.
+ *
+ * Errors: arguments are validated on the host before anything is launched.  A
+ * bad argument returns KQ_ERR_INVALID_ARG / KQ_ERR_UNSUPPORTED /
+ * KQ_ERR_MISALIGNED and enqueues nothing.  KQ_ERR_CUDA means a launch failed
+ * (the CUDA error is reported by kq_last_cuda_error()).  No call traps on the
+ * device.  Inputs must be finite; NaN or Inf inputs give unspecified outputs.
+ * tokens == 0 is a valid no-op.
+ *
+ * Supported shapes:
+ *   dim = 2^k with 32 <= dim <= 16384, or dim = 12 * 2^k with
+ *   384 <= dim <= 12288 (the 12 * 2^k form only with block == 0).
+ *   block = 0 (Hadamard over the whole row) or a power of two with
+ *   16 <= block <= dim that divides dim.
+ * Alignment: x, out and codes 16-byte aligned; scales/zeros/block_scales at
+ * their element size.
+ */
+#ifndef KQ_H
+#define KQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define KQ_API __attribute__((visibility("default")))
+#else
+#define KQ_API
+#endif
+
+struct CUstream_st;
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* kq_stream_t;
+
+typedef enum {
+  KQ_OK = 0,
+  KQ_ERR_INVALID_ARG = -1,  /* null pointer, negative size, bad flag combination */
+  KQ_ERR_UNSUPPORTED = -2,  /* shape, block, group or dtype outside the list above */
+  KQ_ERR_MISALIGNED = -3,   /* a pointer breaks the alignment rule */
+  KQ_ERR_CUDA = -4          /* a kernel launch or memset failed */
+} kq_status;
+
+typedef enum { KQ_F32 = 0, KQ_BF16 = 1 } kq_dtype;
+
+/* flags */
+enum {
+  KQ_INVERSE = 1,        /* kq_rht: inverse transform x = D H^T y / sqrt(b) */
+  KQ_SCALE_STATIC = 2,   /* kq_rht_quant_nvfp4: *tensor_scale is an input */
+  KQ_SCALE_DYNAMIC = 4   /* kq_rht_quant_nvfp4: *tensor_scale is computed and written */
+};
+
+/* formats for kq_dequant */
+enum { KQ_FMT_INT4_SYM = 0, KQ_FMT_INT4_ASYM = 1, KQ_FMT_NVFP4 = 2 };
+
+/*
+ * kq_rht -- rotation only, fp32 output.
+ * Forward (flags = 0): out = y as defined above (QuaRot reviews, review 2
+ * Summary and review 3 Questions: Y = X H^T).  Inverse (flags = KQ_INVERSE):
+ * out = x_j = s_j sum_i H[i][j] y_i / sqrt(b), the exact inverse of the forward
+ * map ("fully invertible up to machine epsilon", review 2 Summary).
+ * x: [tokens, dim] fp32 or bf16; signs: int8[dim] or NULL; out: fp32
+ * [tokens, dim] (may not alias x).
+ */
+KQ_API kq_status kq_rht(const void* x, int dtype, int64_t tokens, int dim,
+                        int block, const int8_t* signs, float* out, int flags,
+                        kq_stream_t stream);
+
+/*
+ * kq_rht_quant_int4 -- rotation fused with INT4 quantization into packed
+ * nibbles (QuaRot reviews, review 2 Summary/Weaknesses: RTN INT4 on rotated
+ * activations; final comments: KV cache at 4 bits; NVFP4 thread,
+ * discrete_descent's INT4-g128 note).
+ * asym == 0: symmetric per token; group must be 0; scales = fp32 [tokens];
+ *            zeros must be NULL.
+ * asym == 1: asymmetric per group; group must be 128 and divide dim;
+ *            scales and zeros = fp16 [tokens, dim/group].
+ * codes: [tokens, dim/2] bytes.
+ */
+KQ_API kq_status kq_rht_quant_int4(const void* x, int dtype, int64_t tokens,
+                                   int dim, int block, const int8_t* signs,
+                                   int group, int asym, uint8_t* codes,
+                                   void* scales, void* zeros,
+                                   kq_stream_t stream);
+
+/*
+ * kq_rht_quant_nvfp4 -- rotation fused with NVFP4 quantization (NVFP4 thread,
+ * krylov_schur section 3 table: E2M1 codes + one E4M3 scale per 16 elements,
+ * 4.50 bits per element; per-tensor fp32 scale).
+ * flags must hold exactly one of KQ_SCALE_STATIC (tensor_scale is read) or
+ * KQ_SCALE_DYNAMIC (tensor_scale = fp32(amax/2688) of this call's rotated
+ * tensor is computed and written).  For the same tensor scale both modes give
+ * identical codes and block scales.
+ * Dynamic mode needs `workspace`, a device buffer of at least
+ * kq_workspace_size(tokens, dim, block) bytes, 16-byte aligned; its contents on
+ * entry do not matter and are clobbered.  Static mode ignores it.
+ * codes: [tokens, dim/2]; block_scales: E4M3 [tokens, dim/16]; tensor_scale:
+ * one fp32 in device memory.
+ */
+KQ_API kq_status kq_rht_quant_nvfp4(const void* x, int dtype, int64_t tokens,
+                                    int dim, int block, const int8_t* signs,
+                                    uint8_t* codes, uint8_t* block_scales,
+                                    float* tensor_scale, void* workspace,
+                                    size_t ws_bytes, int flags,
+                                    kq_stream_t stream);
+
+/*
+ * kq_dequant -- codes and scales back to fp32: each output is the exact
+ * product of the code value and its scale(s), rounded once to fp32.
+ * fmt = KQ_FMT_INT4_SYM: scales fp32 [tokens]; zeros and tensor_scale unused.
+ * fmt = KQ_FMT_INT4_ASYM: scales, zeros fp16 [tokens, dim/group]; group = 128.
+ * fmt = KQ_FMT_NVFP4: scales = E4M3 bytes [tokens, dim/16]; tensor_scale =
+ *   device fp32.
+ * out: fp32 [tokens, dim].
+ */
+KQ_API kq_status kq_dequant(int fmt, const uint8_t* codes, const void* scales,
+                            const void* zeros, const float* tensor_scale,
+                            int64_t tokens, int dim, int group, float* out,
+                            kq_stream_t stream);
+
+/* Bytes of workspace the dynamic NVFP4 path needs (0 on bad arguments). */
+KQ_API size_t kq_workspace_size(int64_t tokens, int dim, int block);
+
+/* Human-readable name of a status code (static string). */
+KQ_API const char* kq_status_str(int status);
+
+/* The CUDA error code behind the calling thread's last KQ_ERR_CUDA (0 if none). */
+KQ_API int kq_last_cuda_error(void);
+
+/* ABI version: (major << 16) | minor. */
+KQ_API int kq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KQ_H */

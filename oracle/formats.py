@@ -46,21 +46,26 @@ def e2m1_encode(v: np.ndarray) -> np.ndarray:
     """Round float64 values to E2M1 codes: nearest, ties to even index, satfinite.
 
     Sign bit = (v < 0), so a negative value that rounds to zero gives 0x8.
+    Elementwise; processed in chunks only to bound memory.
     """
     v = np.asarray(v, dtype=np.float64)
-    a = np.abs(v)
-    d = np.abs(a[..., None] - E2M1_GRID)                 # distance to each code
-    best = np.min(d, axis=-1, keepdims=True)
-    tie = d == best
-    # among equally near codes take the even index; at most two can tie
-    even = tie & ((np.arange(8) & 1) == 0)
-    idx = np.where(np.any(even, axis=-1), np.argmax(even, axis=-1),
-                   np.argmax(tie, axis=-1))
-    idx = np.where(a >= E2M1_GRID[7], 7, idx)            # saturate
-    # 5 is the midpoint of 4 (index 6) and 6 (index 7): even index 6 wins,
-    # which the search above already does; values above 6 saturate to 6.
-    sign = (v < 0).astype(np.int64) << 3
-    return (idx.astype(np.int64) | sign).astype(np.uint8)
+    flat = v.reshape(-1)
+    out = np.empty(flat.shape, dtype=np.uint8)
+    chunk = 1 << 20
+    for s in range(0, flat.size, chunk):
+        x = flat[s:s + chunk]
+        a = np.abs(x)
+        d = np.abs(a[:, None] - E2M1_GRID[None, :])          # distance to each code
+        best = np.min(d, axis=1, keepdims=True)
+        tie = d == best
+        # among equally near codes take the even index; at most two can tie
+        even = tie & ((np.arange(8) & 1) == 0)[None, :]
+        idx = np.where(np.any(even, axis=1), np.argmax(even, axis=1),
+                       np.argmax(tie, axis=1))
+        idx = np.where(a >= E2M1_GRID[7], 7, idx)             # saturate
+        sign = (x < 0).astype(np.int64) << 3
+        out[s:s + chunk] = idx.astype(np.int64) | sign
+    return out.reshape(v.shape)
 
 
 def _e4m3_value(code: int) -> float:

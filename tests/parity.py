@@ -1,0 +1,197 @@
+"""Comparison helpers: CUDA path (through the C ABI) vs the CPU oracle.
+
+Criteria (from the parity contract of the method):
+  * rotated fp32 values: relative L2 error per row <= 2e-6; an all-zero row
+    must come out exactly zero;
+  * scales (fp32 per token, fp16 scale/zero, E4M3 block scale, fp32 tensor
+    scale): bit-exact;
+  * packed 4-bit codes: bit-exact, except where the oracle's value before
+    rounding lies within 1e-5 (relative) of a rounding boundary; those cases
+    are counted and returned, not hidden.  For NVFP4 the sign bit of a code
+    whose magnitude rounds to zero is decided at 0, which is treated as a
+    boundary with an absolute window of 1e-5 in code units.
+  * dequantized values: bit-exact (the GPU's codes and scales fed to the
+    oracle's dequantizer).
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from oracle.quant import int4_from_nibble
+from hadamard_rotated_activation_b200 import workloads as wl
+import hadamard_rotated_activation_b200 as kq
+
+REL_L2 = 2e-6
+NEAR = 1e-5
+E2M1_MIDPOINTS = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+
+
+# ------------------------------------------------------------ device I/O
+def to_device(inp: wl.Inputs, device="cuda"):
+    w = inp.workload
+    if w.dtype == wl.BF16:
+        x = torch.from_numpy(inp.stored.view(np.int16)).to(device).view(torch.bfloat16)
+    else:
+        x = torch.from_numpy(inp.stored).to(device)
+    s = None if inp.signs is None else torch.from_numpy(inp.signs).to(device)
+    return x, s
+
+
+def stored_from_values(values: np.ndarray, dtype: str) -> np.ndarray:
+    if dtype == wl.BF16:
+        return wl.bf16_bits(values)
+    return values.astype(np.float32)
+
+
+def inputs_from_values(w: wl.Workload, values: np.ndarray, signs) -> wl.Inputs:
+    return wl.Inputs(w.with_tokens(values.shape[0]), values,
+                     stored_from_values(values, w.dtype), signs)
+
+
+# ---------------------------------------------------------- GPU runners
+def gpu_rht(inp: wl.Inputs, inverse=False, x_override=None):
+    w = inp.workload
+    x, s = to_device(inp)
+    if x_override is not None:
+        x = x_override
+    out = torch.empty((x.shape[0], w.dim), dtype=torch.float32, device=x.device)
+    kq.kq_rht(x, w.block, s, out, inverse=inverse)
+    torch.cuda.synchronize()
+    return out.cpu().numpy()
+
+
+def gpu_int4_sym(inp: wl.Inputs):
+    w = inp.workload
+    x, s = to_device(inp)
+    codes, scales = kq.empty_int4_sym(w.tokens, w.dim)
+    kq.kq_rht_quant_int4(x, w.block, s, 0, False, codes, scales)
+    torch.cuda.synchronize()
+    return codes.cpu().numpy(), scales.cpu().numpy()
+
+
+def gpu_int4_asym(inp: wl.Inputs, group=128):
+    w = inp.workload
+    x, s = to_device(inp)
+    codes, scales, zeros = kq.empty_int4_asym(w.tokens, w.dim, group)
+    kq.kq_rht_quant_int4(x, w.block, s, group, True, codes, scales, zeros)
+    torch.cuda.synchronize()
+    return codes.cpu().numpy(), scales.cpu().numpy(), zeros.cpu().numpy()
+
+
+def gpu_nvfp4(inp: wl.Inputs, tensor_scale=None):
+    """Dynamic tensor scale when tensor_scale is None, else static."""
+    w = inp.workload
+    x, s = to_device(inp)
+    codes, bs, ts, ws = kq.empty_nvfp4(w.tokens, w.dim, w.block)
+    if tensor_scale is None:
+        kq.kq_rht_quant_nvfp4(x, w.block, s, codes, bs, ts, ws, dynamic=True)
+    else:
+        ts.fill_(float(np.float32(tensor_scale)))
+        kq.kq_rht_quant_nvfp4(x, w.block, s, codes, bs, ts, None, dynamic=False)
+    torch.cuda.synchronize()
+    return codes.cpu().numpy(), bs.cpu().numpy(), np.float32(ts.cpu().numpy()[0])
+
+
+def gpu_dequant(fmt, codes, scales, zeros, tensor_scale, tokens, dim, group=0):
+    dev = "cuda"
+    c = torch.from_numpy(np.ascontiguousarray(codes)).to(dev)
+    if fmt == kq.KQ_FMT_INT4_SYM:
+        s = torch.from_numpy(np.ascontiguousarray(scales)).to(dev)
+        z = None
+        t = None
+    elif fmt == kq.KQ_FMT_INT4_ASYM:
+        s = torch.from_numpy(np.ascontiguousarray(scales)).to(dev)
+        z = torch.from_numpy(np.ascontiguousarray(zeros)).to(dev)
+        t = None
+    else:
+        s = torch.from_numpy(np.ascontiguousarray(scales)).to(dev)
+        z = None
+        t = torch.tensor([float(tensor_scale)], dtype=torch.float32, device=dev)
+    out = torch.empty((tokens, dim), dtype=torch.float32, device=dev)
+    kq.kq_dequant(fmt, c, s, z, t, tokens, dim, group, out)
+    torch.cuda.synchronize()
+    return out.cpu().numpy()
+
+
+# ------------------------------------------------------------ comparisons
+def check_rotation(got: np.ndarray, want: np.ndarray) -> float:
+    """Max relative L2 error per row; asserts the contract."""
+    err = np.linalg.norm(got.astype(np.float64) - want, axis=1)
+    ref = np.linalg.norm(want, axis=1)
+    zero = ref == 0
+    assert np.all(err[zero] == 0), "zero rows must rotate to exact zeros"
+    rel = np.where(zero, 0.0, err / np.where(zero, 1.0, ref))
+    assert rel.max() <= REL_L2, f"rel L2 {rel.max():.3e} > {REL_L2}"
+    return float(rel.max())
+
+
+def _near_half_integer(v: np.ndarray) -> np.ndarray:
+    b = np.floor(v) + 0.5
+    return np.abs(v - b) <= NEAR * np.abs(b)
+
+
+def check_int4_sym(codes, scales, y64):
+    """Returns the number of near-boundary code differences."""
+    q_ref, s_ref = oracle.int4_sym_per_token(y64)
+    assert np.array_equal(scales.view(np.uint32), s_ref.view(np.uint32)), \
+        _first_diff(scales.view(np.uint32), s_ref.view(np.uint32), "scale")
+    q = int4_from_nibble(oracle.unpack_nibbles(codes))
+    diff = q != q_ref
+    s64 = s_ref.astype(np.float64)[:, None]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        v = np.where(s64 > 0, y64 / s64, 0.0)
+    near = _near_half_integer(v)
+    bad = diff & ~near
+    assert not bad.any(), _first_diff(q, q_ref, "int4 code", bad)
+    return int(diff.sum())
+
+
+def check_int4_asym(codes, scales, zeros, y64, group=128):
+    u_ref, s_ref, z_ref = oracle.int4_asym_group(y64, group)
+    assert np.array_equal(scales.view(np.uint16), s_ref.view(np.uint16)), \
+        _first_diff(scales.view(np.uint16), s_ref.view(np.uint16), "fp16 scale")
+    assert np.array_equal(zeros.view(np.uint16), z_ref.view(np.uint16)), \
+        _first_diff(zeros.view(np.uint16), z_ref.view(np.uint16), "fp16 zero")
+    u = oracle.unpack_nibbles(codes)
+    diff = u != u_ref
+    t, n = y64.shape
+    s = np.repeat(s_ref.astype(np.float64), group, axis=1)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        v = np.where(s > 0, y64 / s, 0.0)
+    near = _near_half_integer(v)
+    bad = diff & ~near
+    assert not bad.any(), _first_diff(u, u_ref, "asym code", bad)
+    return int(diff.sum())
+
+
+def check_nvfp4(codes, bscales, tscale, y64, tensor_scale=None):
+    c_ref, sb_ref, t_ref = oracle.nvfp4(y64, tensor_scale)
+    assert np.float32(tscale).view(np.uint32) == np.float32(t_ref).view(np.uint32), \
+        f"tensor scale {tscale!r} != {t_ref!r}"
+    assert np.array_equal(bscales, sb_ref), _first_diff(bscales, sb_ref, "E4M3 scale")
+    c = oracle.unpack_nibbles(codes)
+    diff = c != c_ref
+    t, n = y64.shape
+    den = np.repeat(oracle.e4m3_decode(sb_ref), 16, axis=1) * np.float64(t_ref)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        v = np.abs(np.where(den > 0, y64 / den, 0.0))
+    near = np.any(np.abs(v[..., None] - E2M1_MIDPOINTS) <= NEAR * E2M1_MIDPOINTS, axis=-1)
+    # sign of a zero-magnitude code: boundary at 0
+    zero_mag = (c_ref & 7) == 0
+    sign_only = diff & zero_mag & ((c & 7) == 0)
+    near |= sign_only & (v <= NEAR)
+    bad = diff & ~near
+    assert not bad.any(), _first_diff(c, c_ref, "e2m1 code", bad)
+    return int(diff.sum())
+
+
+def _first_diff(a, b, what, mask=None):
+    if mask is None:
+        mask = a != b
+    idx = np.argwhere(mask)
+    if len(idx) == 0:
+        return f"{what}: no difference"
+    i = tuple(idx[0])
+    return f"{what}: {int(mask.sum())} differences, first at {i}: got {a[i]!r} want {b[i]!r}"

@@ -1,0 +1,107 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol that
+include/kq.h declares, and rejects bad arguments on the host before any CUDA
+call (validation never dereferences the pointers, so fake aligned addresses
+are enough)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import hadamard_rotated_activation_b200 as kq
+from hadamard_rotated_activation_b200 import build as kqbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    kqbuild.build()
+    return kq.lib()
+
+
+def _declared_symbols():
+    with open(os.path.join(ROOT, "include", "kq.h")) as f:
+        src = f.read()
+    return sorted(set(re.findall(r"KQ_API\s+[\w\s\*]+?\b(kq_\w+)\s*\(", src)))
+
+
+def test_header_symbols_exported(L):
+    names = _declared_symbols()
+    assert set(names) == set(kq.C_SYMBOLS)
+    for n in names:
+        assert hasattr(L, n), n
+        assert ctypes.cast(getattr(L, n), ctypes.c_void_p).value
+
+
+def test_version_and_status_strings(L):
+    assert kq.kq_version() >> 16 == 1
+    for code, name in [(0, "KQ_OK"), (-1, "KQ_ERR_INVALID_ARG"), (-2, "KQ_ERR_UNSUPPORTED"),
+                       (-3, "KQ_ERR_MISALIGNED"), (-4, "KQ_ERR_CUDA")]:
+        assert kq.status_str(code) == name
+
+
+P = 1 << 20          # a fake, 16-byte-aligned device address (never dereferenced)
+Q = 2 << 20
+
+
+@pytest.mark.parametrize("dim,block,want", [
+    (4096, 0, 0), (4096, 128, 0), (12288, 0, 0), (12288, 128, 0), (32, 16, 0),
+    (16384, 0, 0), (384, 0, 0),
+    (16, 0, -2), (4095, 0, -2), (32768, 0, -2), (24576, 0, -2), (96, 0, -2),
+    (4096, 8, -2), (4096, 100, -2), (4096, 8192, -2), (12288, 3072, -2),
+])
+def test_shape_validation(L, dim, block, want):
+    # tokens = 0: a valid call is a no-op and returns KQ_OK without CUDA
+    st = L.kq_rht(P, kq.KQ_BF16, 0, dim, block, None, Q, 0, None)
+    assert st == want
+
+
+def test_argument_errors(L):
+    assert L.kq_rht(None, 1, 4, 4096, 0, None, Q, 0, None) == kq.KQ_ERR_INVALID_ARG
+    assert L.kq_rht(P, 1, -1, 4096, 0, None, Q, 0, None) == kq.KQ_ERR_INVALID_ARG
+    assert L.kq_rht(P, 7, 4, 4096, 0, None, Q, 0, None) == kq.KQ_ERR_UNSUPPORTED
+    assert L.kq_rht(P, 1, 4, 4096, 0, None, None, 0, None) == kq.KQ_ERR_INVALID_ARG
+    assert L.kq_rht(P, 1, 4, 4096, 0, None, Q, 8, None) == kq.KQ_ERR_INVALID_ARG
+    assert L.kq_rht(P + 2, 1, 4, 4096, 0, None, Q, 0, None) == kq.KQ_ERR_MISALIGNED
+    assert L.kq_rht(P, 1, 4, 4096, 0, P + 3, Q, 0, None) == kq.KQ_ERR_MISALIGNED
+    # int4: sym needs group 0 and no zeros; asym needs group 128 and zeros
+    f = L.kq_rht_quant_int4
+    assert f(P, 1, 0, 4096, 0, None, 0, 0, Q, Q, None, None) == kq.KQ_OK
+    assert f(P, 1, 4, 4096, 0, None, 128, 0, Q, Q, None, None) == kq.KQ_ERR_UNSUPPORTED
+    assert f(P, 1, 4, 4096, 0, None, 0, 0, Q, Q, Q, None) == kq.KQ_ERR_INVALID_ARG
+    assert f(P, 1, 4, 4096, 0, None, 64, 1, Q, Q, Q, None) == kq.KQ_ERR_UNSUPPORTED
+    assert f(P, 1, 4, 4096, 0, None, 128, 1, Q, Q, None, None) == kq.KQ_ERR_INVALID_ARG
+    assert f(P, 1, 4, 4096, 0, None, 128, 2, Q, Q, Q, None) == kq.KQ_ERR_INVALID_ARG
+    assert f(P, 1, 4, 4096, 0, None, 0, 0, Q + 4, Q, None, None) == kq.KQ_ERR_MISALIGNED
+    assert f(P, 1, 4, 4096, 0, None, 0, 0, Q, Q + 2, None, None) == kq.KQ_ERR_MISALIGNED
+    # nvfp4: exactly one scale mode; dynamic needs a large enough workspace
+    g = L.kq_rht_quant_nvfp4
+    ws = L.kq_workspace_size(4, 4096, 0)
+    assert ws >= 16 + 4 * 8
+    assert g(P, 1, 0, 4096, 0, None, Q, Q, Q, None, 0, kq.KQ_SCALE_STATIC, None) == kq.KQ_OK
+    assert g(P, 1, 4, 4096, 0, None, Q, Q, Q, None, 0, 0, None) == kq.KQ_ERR_INVALID_ARG
+    assert g(P, 1, 4, 4096, 0, None, Q, Q, Q, None, 0, 6, None) == kq.KQ_ERR_INVALID_ARG
+    assert g(P, 1, 4, 4096, 0, None, Q, Q, Q, None, 0, kq.KQ_SCALE_DYNAMIC, None) \
+        == kq.KQ_ERR_INVALID_ARG
+    assert g(P, 1, 4, 4096, 0, None, Q, Q, Q, P, ws - 1, kq.KQ_SCALE_DYNAMIC, None) \
+        == kq.KQ_ERR_INVALID_ARG
+    assert g(P, 1, 4, 4096, 0, None, Q, Q, Q, P + 8, ws, kq.KQ_SCALE_DYNAMIC, None) \
+        == kq.KQ_ERR_MISALIGNED
+    assert g(P, 1, 0, 4096, 0, None, Q, Q, Q, P, ws, kq.KQ_SCALE_DYNAMIC, None) == kq.KQ_OK
+    # dequant
+    d = L.kq_dequant
+    assert d(3, Q, Q, None, None, 4, 4096, 0, P, None) == kq.KQ_ERR_INVALID_ARG
+    assert d(2, Q, Q, None, None, 4, 4096, 0, P, None) == kq.KQ_ERR_INVALID_ARG
+    assert d(1, Q, Q, None, None, 4, 4096, 128, P, None) == kq.KQ_ERR_INVALID_ARG
+    assert d(1, Q, Q, Q, None, 4, 4096, 64, P, None) == kq.KQ_ERR_UNSUPPORTED
+    assert d(0, Q, Q, None, None, 4, 4100, 0, P, None) == kq.KQ_ERR_UNSUPPORTED
+    assert d(0, Q, Q, None, None, 0, 4096, 0, P, None) == kq.KQ_OK
+    assert L.kq_workspace_size(4, 4095, 0) == 0
+
+
+def test_python_binding_rejects_host_tensors(L):
+    import torch
+    x = torch.zeros(2, 64)
+    with pytest.raises(ValueError):
+        kq.kq_rht(x, 0, None, torch.zeros(2, 64))

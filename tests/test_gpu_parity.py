@@ -1,0 +1,216 @@
+"""GPU parity: the CUDA path through the C ABI vs the CPU oracle.
+
+Small cases span several CTAs and a ragged row count, plus degenerate rows
+(zeros, a single spike, constant, alternating, tiny, huge).  Full-size cases
+run each workload at its published size in the launch configuration the
+benchmark times and compare sampled rows (or every row where a global
+quantity such as the NVFP4 tensor scale needs them).
+"""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import oracle
+from hadamard_rotated_activation_b200 import workloads as wl
+import hadamard_rotated_activation_b200 as kq
+import parity as P
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    kq.lib()
+
+
+def small_inputs(key, tokens, with_edges=True):
+    w = wl.WORKLOADS[key]
+    inp = wl.make_inputs(w, tokens=tokens)
+    if not with_edges:
+        return inp
+    edges = wl.edge_rows(w.dim, w.dtype)
+    vals = np.concatenate([inp.values, edges])
+    return P.inputs_from_values(w, vals, inp.signs)
+
+
+# ------------------------------------------------------------- rotation
+@pytest.mark.parametrize("key,tokens", [("c1", 37), ("c2", 37), ("c3", 13), ("c4", 37),
+                                        ("c5", 37)])
+def test_rotation_forward_and_inverse(key, tokens):
+    inp = small_inputs(key, tokens)
+    w = inp.workload
+    y_ref = oracle.rht(inp.values, inp.signs, w.block)
+    y = P.gpu_rht(inp)
+    P.check_rotation(y, y_ref)
+    # inverse of the oracle's rotated values (fed as fp32)
+    y32 = y_ref.astype(np.float32)
+    winv = wl.Workload(w.key, w.tokens, w.dim, wl.F32, w.block, w.use_signs, w.fmt, w.seed)
+    inv_inp = wl.Inputs(winv, y32.astype(np.float64), y32, inp.signs)
+    x_back = P.gpu_rht(inv_inp, inverse=True)
+    P.check_rotation(x_back, oracle.rht_inverse(y32.astype(np.float64), inp.signs, w.block))
+
+
+@pytest.mark.parametrize("dim,block,dtype", [
+    (32, 16, wl.BF16), (256, 32, wl.F32), (256, 0, wl.BF16), (384, 0, wl.BF16),
+    (768, 0, wl.F32), (1024, 64, wl.BF16), (16384, 0, wl.BF16), (8192, 256, wl.F32),
+    (12288, 1024, wl.BF16),
+])
+def test_rotation_other_shapes(dim, block, dtype):
+    rng = np.random.default_rng(dim + block)
+    x = rng.standard_normal((9, dim)) * rng.lognormal(0, 1, dim)
+    x = wl.round_to_bf16(x) if dtype == wl.BF16 else x.astype(np.float32).astype(np.float64)
+    s = (1 - 2 * rng.integers(0, 2, dim)).astype(np.int8)
+    w = wl.Workload("x", 9, dim, dtype, block, True, wl.INT4_SYM, 0)
+    inp = P.inputs_from_values(w, x, s)
+    P.check_rotation(P.gpu_rht(inp), oracle.rht(x, s, block))
+    q, sc = P.gpu_int4_sym(inp)
+    P.check_int4_sym(q, sc, oracle.rht(x, s, block))
+
+
+# ---------------------------------------------------------------- INT4
+@pytest.mark.parametrize("key,tokens", [("c1", 37), ("c3", 13)])
+def test_int4_sym_small(key, tokens):
+    inp = small_inputs(key, tokens)
+    w = inp.workload
+    y = oracle.rht(inp.values, inp.signs, w.block)
+    codes, scales = P.gpu_int4_sym(inp)
+    P.check_int4_sym(codes, scales, y)
+    deq = P.gpu_dequant(kq.KQ_FMT_INT4_SYM, codes, scales, None, None, w.tokens, w.dim)
+    want = oracle.dequant_int4_sym(oracle.quant.int4_from_nibble(oracle.unpack_nibbles(codes)),
+                                   scales)
+    assert np.array_equal(deq.view(np.uint32), want.view(np.uint32))
+
+
+def test_int4_asym_small():
+    inp = small_inputs("c5", 37)
+    w = inp.workload
+    y = oracle.rht(inp.values, inp.signs, w.block)
+    codes, scales, zeros = P.gpu_int4_asym(inp)
+    P.check_int4_asym(codes, scales, zeros, y)
+    deq = P.gpu_dequant(kq.KQ_FMT_INT4_ASYM, codes, scales, zeros, None, w.tokens, w.dim, 128)
+    want = oracle.dequant_int4_asym(oracle.unpack_nibbles(codes), scales, zeros, 128)
+    assert np.array_equal(deq.view(np.uint32), want.view(np.uint32))
+
+
+def test_int4_asym_other_rotations():
+    """Asymmetric g128 after a full-row rotation and with signs."""
+    rng = np.random.default_rng(11)
+    x = wl.round_to_bf16(rng.standard_normal((7, 4096)) * 3)
+    s = (1 - 2 * rng.integers(0, 2, 4096)).astype(np.int8)
+    for block in (0, 256):
+        w = wl.Workload("x", 7, 4096, wl.BF16, block, True, wl.INT4_ASYM, 0, group=128)
+        inp = P.inputs_from_values(w, x, s)
+        c, sc, z = P.gpu_int4_asym(inp)
+        P.check_int4_asym(c, sc, z, oracle.rht(x, s, block))
+
+
+# --------------------------------------------------------------- NVFP4
+@pytest.mark.parametrize("key,tokens", [("c2", 37), ("c4", 37)])
+def test_nvfp4_small_dynamic_and_static(key, tokens):
+    inp = small_inputs(key, tokens)
+    w = inp.workload
+    y = oracle.rht(inp.values, inp.signs, w.block)
+    codes, bs, ts = P.gpu_nvfp4(inp)
+    P.check_nvfp4(codes, bs, ts, y)
+    # static mode with the same tensor scale gives identical output
+    codes2, bs2, ts2 = P.gpu_nvfp4(inp, tensor_scale=ts)
+    assert np.array_equal(codes2, codes) and np.array_equal(bs2, bs) and ts2 == ts
+    # static mode with another tensor scale (saturating and subnormal scales)
+    for f in (0.37, 4.0, 1e-3):
+        t = np.float32(ts * f)
+        c3, b3, _ = P.gpu_nvfp4(inp, tensor_scale=t)
+        P.check_nvfp4(c3, b3, t, y, tensor_scale=t)
+    deq = P.gpu_dequant(kq.KQ_FMT_NVFP4, codes, bs, None, ts, w.tokens, w.dim)
+    want = oracle.dequant_nvfp4(oracle.unpack_nibbles(codes), bs, ts)
+    assert np.array_equal(deq.view(np.uint32), want.view(np.uint32))
+
+
+def test_nvfp4_round_trip_c4_small():
+    inp = small_inputs("c4", 37)
+    w = inp.workload
+    codes, bs, ts = P.gpu_nvfp4(inp)
+    deq = P.gpu_dequant(kq.KQ_FMT_NVFP4, codes, bs, None, ts, w.tokens, w.dim)
+    winv = wl.Workload("inv", w.tokens, w.dim, wl.F32, w.block, True, w.fmt, 0)
+    back = P.gpu_rht(wl.Inputs(winv, deq.astype(np.float64), deq, inp.signs), inverse=True)
+    want = oracle.rht_inverse(deq.astype(np.float64), inp.signs, w.block)
+    P.check_rotation(back, want)
+    # ||x - x'|| = ||y - y_hat||: per element at most one scale unit (half a
+    # grid gap, or the saturation error), and a block whose E4M3 scale flushes
+    # to zero (r <= 2^-10) holds only values below 6 t 2^-10
+    err = np.linalg.norm(back - inp.values, axis=1)
+    unit = np.repeat(oracle.e4m3_decode(bs), 16, axis=1) * np.float64(ts)
+    unit = np.where(unit > 0, unit, 6.0 * np.float64(ts) * 2.0 ** -10)
+    assert np.all(err <= np.sqrt(np.sum(unit ** 2, axis=1)) * 1.0001 + 1e-30)
+
+
+def test_nvfp4_all_zero_tensor():
+    w = wl.WORKLOADS["c4"].with_tokens(5)
+    vals = np.zeros((5, 4096))
+    inp = P.inputs_from_values(w, vals, wl.make_inputs(w).signs)
+    codes, bs, ts = P.gpu_nvfp4(inp)
+    assert ts == 0 and not bs.any() and not codes.any()
+
+
+def test_zero_tokens_is_noop():
+    x = torch.empty((0, 4096), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty((0, 4096), dtype=torch.float32, device="cuda")
+    kq.kq_rht(x, 0, None, out)
+
+
+def test_deterministic_bitwise():
+    inp = small_inputs("c3", 9)
+    a = P.gpu_int4_sym(inp)
+    b = P.gpu_int4_sym(inp)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+    inp2 = small_inputs("c4", 9)
+    assert np.array_equal(P.gpu_rht(inp2), P.gpu_rht(inp2))
+
+
+# ------------------------------------------------------------ full size
+def _sample_rows(t, k, seed):
+    rng = np.random.default_rng(seed)
+    rows = set(rng.choice(t, size=min(k, t), replace=False).tolist())
+    rows |= {0, t - 1}
+    return np.array(sorted(rows))
+
+
+@pytest.mark.parametrize("key", ["c1", "c3", "c5"])
+def test_full_size_per_token_formats(key):
+    w = wl.WORKLOADS[key]
+    inp = wl.make_inputs(w)
+    rows = _sample_rows(w.tokens, 48, 1)
+    if key == "c3":
+        # include the sink rows
+        big = np.argsort(-np.abs(inp.values).max(axis=1))[:10]
+        rows = np.unique(np.concatenate([rows, big]))
+    y = oracle.rht(inp.values[rows], inp.signs, w.block)
+    if w.fmt == wl.INT4_SYM:
+        codes, scales = P.gpu_int4_sym(inp)
+        P.check_int4_sym(codes[rows], scales[rows], y)
+    else:
+        codes, scales, zeros = P.gpu_int4_asym(inp, w.group)
+        P.check_int4_asym(codes[rows], scales[rows], zeros[rows], y, w.group)
+
+
+@pytest.mark.parametrize("key", ["c2", "c4"])
+def test_full_size_nvfp4(key):
+    w = wl.WORKLOADS[key]
+    inp = wl.make_inputs(w)
+    y = oracle.rht(inp.values, inp.signs, w.block)       # every row: global amax
+    codes, bs, ts = P.gpu_nvfp4(inp)
+    t_ref = oracle.nvfp4_tensor_scale(y)
+    assert np.float32(ts).view(np.uint32) == t_ref.view(np.uint32)
+    rows = _sample_rows(w.tokens, 96, 2)
+    gmax_row = int(np.argmax(np.abs(y).max(axis=1)))
+    rows = np.unique(np.append(rows, gmax_row))
+    P.check_nvfp4(codes[rows], bs[rows], ts, y[rows], tensor_scale=t_ref)
+    if key == "c4":
+        deq = P.gpu_dequant(kq.KQ_FMT_NVFP4, codes, bs, None, ts, w.tokens, w.dim)
+        winv = wl.Workload("inv", w.tokens, w.dim, wl.F32, w.block, True, w.fmt, 0)
+        back = P.gpu_rht(wl.Inputs(winv, deq.astype(np.float64), deq, inp.signs),
+                         inverse=True)
+        want = oracle.rht_inverse(deq[rows].astype(np.float64), inp.signs, w.block)
+        P.check_rotation(back[rows], want)
