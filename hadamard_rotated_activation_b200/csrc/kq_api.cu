@@ -46,7 +46,7 @@ kq_status make_geometry(int dim, int block, kq::Geometry* g) {
 
 kq_status check_common(const void* x, int dtype, int64_t tokens, int dim, int block,
                        const int8_t* signs, kq::Geometry* g) {
-  if (!x || tokens < 0) return KQ_ERR_INVALID_ARG;
+  if (tokens < 0 || (tokens > 0 && !x)) return KQ_ERR_INVALID_ARG;
   if (dtype != KQ_F32 && dtype != KQ_BF16) return KQ_ERR_UNSUPPORTED;
   const kq_status st = make_geometry(dim, block, g);
   if (st != KQ_OK) return st;
@@ -76,7 +76,7 @@ KQ_API kq_status kq_rht(const void* x, int dtype, int64_t tokens, int dim, int b
   kq::Geometry g;
   kq_status st = check_common(x, dtype, tokens, dim, block, signs, &g);
   if (st != KQ_OK) return st;
-  if (!out) return KQ_ERR_INVALID_ARG;
+  if (tokens > 0 && !out) return KQ_ERR_INVALID_ARG;
   if (flags & ~KQ_INVERSE) return KQ_ERR_INVALID_ARG;
   if (!aligned(out, 16)) return KQ_ERR_MISALIGNED;
   if (tokens == 0) return KQ_OK;
@@ -91,7 +91,7 @@ KQ_API kq_status kq_rht_quant_int4(const void* x, int dtype, int64_t tokens, int
   kq::Geometry g;
   kq_status st = check_common(x, dtype, tokens, dim, block, signs, &g);
   if (st != KQ_OK) return st;
-  if (!codes || !scales) return KQ_ERR_INVALID_ARG;
+  if (tokens > 0 && (!codes || !scales)) return KQ_ERR_INVALID_ARG;
   if (asym != 0 && asym != 1) return KQ_ERR_INVALID_ARG;
   if (asym == 0) {
     if (group != 0) return KQ_ERR_UNSUPPORTED;
@@ -99,7 +99,7 @@ KQ_API kq_status kq_rht_quant_int4(const void* x, int dtype, int64_t tokens, int
     if (!aligned(scales, 4)) return KQ_ERR_MISALIGNED;
   } else {
     if (group != 128 || dim % group != 0) return KQ_ERR_UNSUPPORTED;
-    if (!zeros) return KQ_ERR_INVALID_ARG;
+    if (tokens > 0 && !zeros) return KQ_ERR_INVALID_ARG;
     if (!aligned(scales, 2) || !aligned(zeros, 2)) return KQ_ERR_MISALIGNED;
   }
   if (!aligned(codes, 16)) return KQ_ERR_MISALIGNED;
@@ -121,14 +121,15 @@ KQ_API kq_status kq_rht_quant_nvfp4(const void* x, int dtype, int64_t tokens, in
   kq::Geometry g;
   kq_status st = check_common(x, dtype, tokens, dim, block, signs, &g);
   if (st != KQ_OK) return st;
-  if (!codes || !block_scales || !tensor_scale) return KQ_ERR_INVALID_ARG;
+  if (tokens > 0 && (!codes || !block_scales || !tensor_scale)) return KQ_ERR_INVALID_ARG;
   const int mode = flags & (KQ_SCALE_STATIC | KQ_SCALE_DYNAMIC);
   if ((flags & ~(KQ_SCALE_STATIC | KQ_SCALE_DYNAMIC)) != 0) return KQ_ERR_INVALID_ARG;
   if (mode != KQ_SCALE_STATIC && mode != KQ_SCALE_DYNAMIC) return KQ_ERR_INVALID_ARG;
   if (!aligned(codes, 16) || !aligned(tensor_scale, 4)) return KQ_ERR_MISALIGNED;
   kq::NvWorkspace* ws = nullptr;
   if (mode == KQ_SCALE_DYNAMIC) {
-    if (!workspace || ws_bytes < nv_workspace_bytes(tokens)) return KQ_ERR_INVALID_ARG;
+    if ((tokens > 0 && !workspace) || ws_bytes < nv_workspace_bytes(tokens))
+      return KQ_ERR_INVALID_ARG;
     if (!aligned(workspace, 16)) return KQ_ERR_MISALIGNED;
     ws = static_cast<kq::NvWorkspace*>(workspace);
   }
@@ -140,7 +141,7 @@ KQ_API kq_status kq_rht_quant_nvfp4(const void* x, int dtype, int64_t tokens, in
 KQ_API kq_status kq_dequant(int fmt, const uint8_t* codes, const void* scales,
                             const void* zeros, const float* tensor_scale, int64_t tokens,
                             int dim, int group, float* out, kq_stream_t stream) {
-  if (!codes || !scales || !out || tokens < 0) return KQ_ERR_INVALID_ARG;
+  if (tokens < 0 || (tokens > 0 && (!codes || !scales || !out))) return KQ_ERR_INVALID_ARG;
   if (dim <= 0 || dim % 32 != 0) return KQ_ERR_UNSUPPORTED;
   if (!aligned(codes, 16) || !aligned(out, 16)) return KQ_ERR_MISALIGNED;
   switch (fmt) {
@@ -149,11 +150,11 @@ KQ_API kq_status kq_dequant(int fmt, const uint8_t* codes, const void* scales,
       break;
     case KQ_FMT_INT4_ASYM:
       if (group != 128 || dim % group != 0) return KQ_ERR_UNSUPPORTED;
-      if (!zeros) return KQ_ERR_INVALID_ARG;
+      if (tokens > 0 && !zeros) return KQ_ERR_INVALID_ARG;
       if (!aligned(scales, 2) || !aligned(zeros, 2)) return KQ_ERR_MISALIGNED;
       break;
     case KQ_FMT_NVFP4:
-      if (!tensor_scale) return KQ_ERR_INVALID_ARG;
+      if (tokens > 0 && !tensor_scale) return KQ_ERR_INVALID_ARG;
       if (!aligned(tensor_scale, 4)) return KQ_ERR_MISALIGNED;
       break;
     default:

@@ -64,7 +64,8 @@
  * KQ_ERR_MISALIGNED and enqueues nothing.  KQ_ERR_CUDA means a launch failed
  * (the CUDA error is reported by kq_last_cuda_error()).  No call traps on the
  * device.  Inputs must be finite; NaN or Inf inputs give unspecified outputs.
- * tokens == 0 is a valid no-op.
+ * tokens == 0 is a valid no-op: shapes and flags are still checked, but
+ * data pointers may then be NULL.
  *
  * Supported shapes:
  *   dim = 2^k with 32 <= dim <= 16384, or dim = 12 * 2^k with

@@ -97,6 +97,9 @@ def test_argument_errors(L):
     assert d(1, Q, Q, Q, None, 4, 4096, 64, P, None) == kq.KQ_ERR_UNSUPPORTED
     assert d(0, Q, Q, None, None, 4, 4100, 0, P, None) == kq.KQ_ERR_UNSUPPORTED
     assert d(0, Q, Q, None, None, 0, 4096, 0, P, None) == kq.KQ_OK
+    # tokens == 0: data pointers may be NULL
+    assert L.kq_rht(None, 1, 0, 4096, 0, None, None, 0, None) == kq.KQ_OK
+    assert d(2, None, None, None, None, 0, 4096, 0, None, None) == kq.KQ_OK
     assert L.kq_workspace_size(4, 4095, 0) == 0
 
 
