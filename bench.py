@@ -46,6 +46,8 @@ def parse_args():
     p.add_argument("--steps", type=int, default=200)
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--workload", default="c4")
+    p.add_argument("--tokens", type=int, default=0,
+                   help="override the workload's row count (small cases for profiling)")
     p.add_argument("--impl", default="kq", choices=["kq", "reference"])
     p.add_argument("--no-extras", action="store_true",
                    help="skip the per-workload table, dynamic and round-trip timings")
@@ -266,6 +268,8 @@ def run_reference(args, rank, world):
     import oracle as oracle_mod
     from hadamard_rotated_activation_b200 import workloads as wl
     w = wl.WORKLOADS[args.workload]
+    if args.tokens:
+        w = w.with_tokens(args.tokens)
     per_step_s = max(2.0, min(20.0, 150.0 / max(args.steps + args.warmup, 1)))
     rows = cpu_sample_rows(oracle_mod, wl, w, per_step_s)
     inp = wl.make_inputs(w, tokens=rows)
@@ -335,6 +339,8 @@ def main():
     kq.lib()
 
     w = wl.WORKLOADS[args.workload]
+    if args.tokens:
+        w = w.with_tokens(args.tokens)
     peak, peak_kind = measured_peaks()
     # every rank draws its own batch (weak scaling)
     inp = wl.make_inputs(w, seed=w.seed + 1000 * rank)
