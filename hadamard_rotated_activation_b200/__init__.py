@@ -38,7 +38,12 @@ KQ_FMT_NVFP4 = 2
 C_SYMBOLS = (
     "kq_rht", "kq_rht_quant_int4", "kq_rht_quant_nvfp4", "kq_dequant",
     "kq_workspace_size", "kq_status_str", "kq_last_cuda_error", "kq_version",
+    "kq_rht_quant_nvfp4_dynamic_noalloc",
 )
+
+# Fixed device scratch of kq_rht_quant_nvfp4_dynamic_noalloc (see include/kq.h).
+KQ_NOALLOC_SCRATCH_BYTES = 1 << 20
+KQ_NOALLOC_MAX_TOKENS = (KQ_NOALLOC_SCRATCH_BYTES - 16) // 8
 
 _lib = None
 
@@ -71,6 +76,9 @@ def lib() -> ctypes.CDLL:
     L.kq_rht_quant_nvfp4.restype = i32
     L.kq_dequant.argtypes = [i32, vp, vp, vp, vp, i64, i32, i32, vp, vp]
     L.kq_dequant.restype = i32
+    L.kq_rht_quant_nvfp4_dynamic_noalloc.argtypes = [vp, i32, i64, i32, i32, vp, vp, vp,
+                                                     vp, vp]
+    L.kq_rht_quant_nvfp4_dynamic_noalloc.restype = i32
     L.kq_workspace_size.argtypes = [i64, i32, i32]
     L.kq_workspace_size.restype = sz
     L.kq_status_str.argtypes = [i32]
@@ -153,6 +161,17 @@ def kq_rht_quant_nvfp4(x, block: int, signs, codes, block_scales, tensor_scale,
                                     _ptr(codes), _ptr(block_scales), _ptr(tensor_scale),
                                     _ptr(workspace), ws_bytes, flags, _stream(stream)),
            "kq_rht_quant_nvfp4")
+
+
+def kq_rht_quant_nvfp4_dynamic_noalloc(x, block: int, signs, codes, block_scales,
+                                       tensor_scale, stream=None) -> None:
+    """Dynamic-scale NVFP4 for callers that cannot allocate device memory: the
+    workspace is the library's own fixed device array (at most
+    KQ_NOALLOC_MAX_TOKENS rows).  Calls that overlap on the GPU race."""
+    t, n = x.shape
+    _check(lib().kq_rht_quant_nvfp4_dynamic_noalloc(
+        _ptr(x), _dtype_code(x), t, n, block, _ptr(signs), _ptr(codes), _ptr(block_scales),
+        _ptr(tensor_scale), _stream(stream)), "kq_rht_quant_nvfp4_dynamic_noalloc")
 
 
 def kq_dequant(fmt: int, codes, scales, zeros, tensor_scale, tokens: int, dim: int,

@@ -69,6 +69,10 @@ size_t nv_workspace_bytes(int64_t tokens) {
 
 }  // namespace
 
+namespace kq {
+void set_last_cuda_error(int err) { g_last_cuda_error = err; }
+}  // namespace kq
+
 extern "C" {
 
 KQ_API kq_status kq_rht(const void* x, int dtype, int64_t tokens, int dim, int block,

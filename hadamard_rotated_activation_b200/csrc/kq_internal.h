@@ -20,6 +20,9 @@ struct NvWorkspace {
 };
 constexpr size_t kNvWorkspaceHeader = 16;
 
+// Records a CUDA error for kq_last_cuda_error() on the calling thread.
+void set_last_cuda_error(int err);
+
 cudaError_t launch_rht(const void* x, int dtype, int64_t tokens, const Geometry& g,
                        const int8_t* signs, float* out, int inverse, cudaStream_t s);
 cudaError_t launch_int4_sym(const void* x, int dtype, int64_t tokens, const Geometry& g,

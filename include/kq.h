@@ -180,6 +180,36 @@ KQ_API kq_status kq_dequant(int fmt, const uint8_t* codes, const void* scales,
                             int64_t tokens, int dim, int group, float* out,
                             kq_stream_t stream);
 
+/*
+ * kq_rht_quant_nvfp4_dynamic_noalloc -- kq_rht_quant_nvfp4 with
+ * KQ_SCALE_DYNAMIC, for callers that cannot allocate device memory.  The
+ * pages have no counterpart to this entry point; it exists for integration.
+ *
+ * Who needs it: code that may not call cudaMalloc or any allocator -- a plugin
+ * whose host framework owns all device memory and passes it no workspace, or a
+ * serving loop that reserves HBM up front and cannot afford cudaMalloc (which
+ * may synchronize the device) on its hot path.  The caller still passes the
+ * input and all outputs, exactly as for kq_rht_quant_nvfp4.
+ *
+ * The dynamic tensor scale's workspace lives instead in a fixed array of
+ * KQ_NOALLOC_SCRATCH_BYTES (1 MiB) of the library's own device memory, which
+ * every GPU that loads the library holds until the process exits.  tokens
+ * above KQ_NOALLOC_MAX_TOKENS returns KQ_ERR_UNSUPPORTED and launches nothing.
+ * The call allocates nothing and calls no allocating routine.
+ *
+ * The first call on each device looks up the array's device address (with
+ * that device current) and caches it; make that first call before any stream
+ * capture.  All calls share the one array and it keeps the last call's
+ * contents (each call clears what must start at zero), so calls that overlap
+ * on the GPU -- on different streams or from different threads -- race and
+ * must be serialized by the caller.
+ */
+#define KQ_NOALLOC_SCRATCH_BYTES (1u << 20)
+#define KQ_NOALLOC_MAX_TOKENS ((KQ_NOALLOC_SCRATCH_BYTES - 16u) / 8u)
+KQ_API kq_status kq_rht_quant_nvfp4_dynamic_noalloc(
+    const void* x, int dtype, int64_t tokens, int dim, int block, const int8_t* signs,
+    uint8_t* codes, uint8_t* block_scales, float* tensor_scale, kq_stream_t stream);
+
 /* Bytes of workspace the dynamic NVFP4 path needs (0 on bad arguments). */
 KQ_API size_t kq_workspace_size(int64_t tokens, int dim, int block);
 
