@@ -3,6 +3,7 @@
 // Every argument is checked here, before anything is enqueued; a rejected call
 // leaves the stream untouched.  The library allocates nothing.
 #include <cmath>
+#include <cstdlib>
 #include <cstdint>
 #include <cstring>
 
@@ -84,6 +85,9 @@ KQ_API kq_status kq_rht(const void* x, int dtype, int64_t tokens, int dim, int b
   if (flags & ~KQ_INVERSE) return KQ_ERR_INVALID_ARG;
   if (!aligned(out, 16)) return KQ_ERR_MISALIGNED;
   if (tokens == 0) return KQ_OK;
+  if (!(flags & KQ_INVERSE) && kq::tc_row_supported(g, dtype))
+    return finish(kq::launch_tc_rot(x, tokens, g, signs, out,
+                                    reinterpret_cast<cudaStream_t>(stream)));
   return finish(kq::launch_rht(x, dtype, tokens, g, signs, out, (flags & KQ_INVERSE) ? 1 : 0,
                                reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -109,6 +113,13 @@ KQ_API kq_status kq_rht_quant_int4(const void* x, int dtype, int64_t tokens, int
   if (!aligned(codes, 16)) return KQ_ERR_MISALIGNED;
   if (tokens == 0) return KQ_OK;
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (asym == 1 && kq::blk128_supported(g, dtype) && aligned(signs, 16))
+    return finish(kq::launch_blk128_asym(x, tokens, g, signs, codes,
+                                         static_cast<uint16_t*>(scales),
+                                         static_cast<uint16_t*>(zeros), s));
+  if (asym == 0 && kq::rowwarp_supported(g, dtype))
+    return finish(kq::launch_rowwarp_int4(x, dtype, tokens, g, signs, codes,
+                                          static_cast<float*>(scales), s));
   if (asym == 0)
     return finish(kq::launch_int4_sym(x, dtype, tokens, g, signs, codes,
                                       static_cast<float*>(scales), s));
@@ -138,6 +149,17 @@ KQ_API kq_status kq_rht_quant_nvfp4(const void* x, int dtype, int64_t tokens, in
     ws = static_cast<kq::NvWorkspace*>(workspace);
   }
   if (tokens == 0) return KQ_OK;
+  if (kq::blk128_supported(g, dtype) && aligned(signs, 16) && aligned(block_scales, 8))
+    return finish(kq::launch_blk128_nvfp4(x, tokens, g, signs, codes, block_scales,
+                                          tensor_scale, ws,
+                                          reinterpret_cast<cudaStream_t>(stream)));
+  if (kq::tc_row_supported(g, dtype) && aligned(block_scales, 8))
+    return finish(kq::launch_tc_nvfp4(x, tokens, g, signs, codes, block_scales, tensor_scale,
+                                      ws, reinterpret_cast<cudaStream_t>(stream)));
+  if (kq::rowwarp_supported(g, dtype) && aligned(block_scales, 8))
+    return finish(kq::launch_rowwarp_nvfp4(x, dtype, tokens, g, signs, codes, block_scales,
+                                           tensor_scale, ws,
+                                           reinterpret_cast<cudaStream_t>(stream)));
   return finish(kq::launch_nvfp4(x, dtype, tokens, g, signs, codes, block_scales,
                                  tensor_scale, ws, reinterpret_cast<cudaStream_t>(stream)));
 }

@@ -1,0 +1,605 @@
+// Thread-per-block kernels for 128-wide Hadamard blocks (block = 128).
+//
+// "Block-Hadamard-128" (NVFP4 thread, discrete_descent's note) and the
+// per-head 128-point Hadamard of the KV cache (QuaRot reviews, final comments)
+// apply an independent H_128 to every 128 consecutive columns.  Here one
+// thread owns one (row, block) unit: its 128 inputs arrive by sixteen 16-byte
+// loads straight into registers, the sign flips are XORs on the bf16 sign
+// bits, and the seven butterfly stages run in registers (stage 0 in scalar
+// fp32, stages 1..6 on packed f32x2 pairs).  The 16-element NVFP4 blocks and
+// the 128-element INT4 groups lie inside the thread, so extrema, scales,
+// rounding and nibble packing need no communication.  There is no shared
+// memory and no barrier.
+//
+// Exact scales.  The fp32 transform of one 128-block is within
+// E = gamma_7 sqrt(128) max|S_hat| of the exact sums (see error_bound in
+// kq_device.cuh).  A scale is decided from the fp32 values when both ends of
+// its interval round to the same stored value; the rare undecided ones are
+// recomputed by the whole warp as exact fp64 dot products with the input.
+#include <cfloat>
+#include <climits>
+#include <cstdint>
+
+#include "kq_device.cuh"
+#include "kq_internal.h"
+
+namespace kq {
+namespace blk {
+
+constexpr int B = 128;          // Hadamard block width
+constexpr int kThreads = 128;
+
+struct Params {
+  const uint16_t* x;            // bf16 bits [T, n]
+  const int8_t* signs;          // [n] or null
+  uint8_t* codes;               // [T, n/2]
+  uint8_t* scales8;             // NVFP4 E4M3 [T, n/16]
+  uint16_t* scales16;           // asym fp16 [T, n/128]
+  uint16_t* zeros16;            // asym fp16 [T, n/128]
+  float* tensor_scale;          // NVFP4 t (device): read if static, written if dynamic
+  NvWorkspace* ws;              // NVFP4 dynamic: gmax (read) / row stats (written)
+  int64_t units;                // T * n / 128
+  int n;
+  float e_coef;                 // E = e_coef * max|S_hat| (rounded up)
+};
+
+__device__ __forceinline__ int stage_chunk(int unit, int c);
+
+// packed f32x2 butterfly: (a, b) <- (a + b, a - b) on two lanes at once
+__device__ __forceinline__ void bfly2(float2& a, float2& b) {
+  uint64_t ua = *reinterpret_cast<uint64_t*>(&a), ub = *reinterpret_cast<uint64_t*>(&b), s, d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(s) : "l"(ua), "l"(ub));
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(ua), "l"(ub));
+  a = *reinterpret_cast<float2*>(&s);
+  b = *reinterpret_cast<float2*>(&d);
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+  float d;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  uint64_t ua = *reinterpret_cast<uint64_t*>(&a), ub = *reinterpret_cast<uint64_t*>(&b),
+           uc = *reinterpret_cast<uint64_t*>(&c), r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(ua), "l"(ub), "l"(uc));
+  return *reinterpret_cast<float2*>(&r);
+}
+
+// Shared-memory stage of one warp: 32 units x 256 bytes, 16-byte chunk c of
+// unit t stored at chunk position c ^ (t & 15) of its row.  Warp-wide
+// coalesced writes (lane l -> chunk l + 32 j) and per-thread row reads are
+// both bank-conflict-free.
+__device__ __forceinline__ int stage_chunk(int unit, int c) { return unit * 16 + (c ^ (unit & 15)); }
+
+
+// Starts copying the warp's 32 consecutive units (8 KB, contiguous in memory)
+// into the stage with coalesced 16-byte asynchronous copies, as one commit
+// group.  Units at or beyond `units` are skipped.
+__device__ __forceinline__ void prefetch_units(const uint16_t* __restrict__ x, int64_t ub,
+                                               int64_t units, uint4* stage) {
+  const int lane = threadIdx.x & 31;
+  const uint4* src = reinterpret_cast<const uint4*>(x + ub * B);
+  const uint32_t base = (uint32_t)__cvta_generic_to_shared(stage);
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const int idx = lane + 32 * j;
+    if (ub + (idx >> 4) < units) {
+      const uint32_t dst = base + 16u * (uint32_t)stage_chunk(idx >> 4, idx & 15);
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"(dst), "l"(src + idx)
+                   : "memory");
+    }
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+__device__ __forceinline__ void wait_prefetch(bool newer_pending) {
+  if (newer_pending)
+    asm volatile("cp.async.wait_group 1;" ::: "memory");
+  else
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+  __syncwarp();
+}
+
+// Sign masks of every 128-column block, staged per CTA: 16-byte chunk c of
+// column block k (four bf16-pair masks: bit 15 even, bit 31 odd element) at
+// chunk position c ^ (k & 15).
+__device__ __forceinline__ void stage_signs(const int8_t* __restrict__ signs, int n,
+                                            uint4* smask) {
+  for (int i = threadIdx.x; i < n / 8; i += blockDim.x) {
+    const uint2 sv = __ldg(reinterpret_cast<const uint2*>(signs) + i);
+    const int k = i >> 4, c = i & 15;
+    smask[k * 16 + (c ^ (k & 15))] =
+        make_uint4(__byte_perm(sv.x, 0, 0x1404) & 0x80008000u,
+                   __byte_perm(sv.x, 0, 0x3424) & 0x80008000u,
+                   __byte_perm(sv.y, 0, 0x1404) & 0x80008000u,
+                   __byte_perm(sv.y, 0, 0x3424) & 0x80008000u);
+  }
+}
+
+// Transforms this thread's unit from the stage: applies the signs of column
+// block k (if smask) and runs the unnormalised H_128; v[p] = {S[2p], S[2p+1]}.
+__device__ __forceinline__ void load_transform(const uint4* stage, int t, const uint4* smask,
+                                               int k, float2 (&v)[64]) {
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    const uint4 w = stage[stage_chunk(t, c)];
+    uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+    if (smask) {
+      const uint4 m = smask[k * 16 + (c ^ (k & 15))];
+      ww[0] ^= m.x;
+      ww[1] ^= m.y;
+      ww[2] ^= m.z;
+      ww[3] ^= m.w;
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float lo = __uint_as_float(ww[q] << 16);
+      const float hi = __uint_as_float(ww[q] & 0xffff0000u);
+      v[4 * c + q] = make_float2(lo + hi, lo - hi);   // stage on bit 0
+    }
+  }
+#pragma unroll
+  for (int h = 1; h < 64; h <<= 1)
+#pragma unroll
+    for (int p = 0; p < 64; ++p)
+      if (!(p & h)) bfly2(v[p], v[p | h]);
+}
+
+// Writes each thread's 64 code bytes (4 chunks) through the stage so that the
+// warp stores 2 KB with coalesced 16-byte stores.
+__device__ __forceinline__ void store_codes(uint4* stage, const uint4 (&cw)[4], uint8_t* codes,
+                                            int64_t ub, int64_t units) {
+  const int lane = threadIdx.x & 31;
+  __syncwarp();
+#pragma unroll
+  for (int k = 0; k < 4; ++k) stage[lane * 4 + (k ^ (lane & 3))] = cw[k];
+  __syncwarp();
+  uint4* dst = reinterpret_cast<uint4*>(codes + ub * (B / 2));
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int idx = lane + 32 * j;       // chunk idx = unit * 4 + k
+    const int t = idx >> 2, k = idx & 3;
+    if (ub + t < units) dst[idx] = stage[t * 4 + (k ^ (t & 3))];
+  }
+}
+
+// Exact S of element `e` (0..127) of the warp's unit `t`, computed by the
+// whole warp in fp64 from the staged input (lane l sums inputs 4l..4l+3) and
+// the staged sign masks of column block k; every lane gets the result.
+__device__ __noinline__ double warp_exact_S(const uint4* stage, const uint4* smask, int t,
+                                            int k, int e) {
+  const int lane = threadIdx.x & 31;
+  const uint4 w = stage[stage_chunk(t, lane >> 1)];
+  const uint32_t a = (lane & 1) ? w.z : w.x, b = (lane & 1) ? w.w : w.y;
+  uint32_t ma = 0, mb = 0;
+  if (smask) {
+    const uint4 m = smask[k * 16 + ((lane >> 1) ^ (k & 15))];
+    ma = (lane & 1) ? m.z : m.x;
+    mb = (lane & 1) ? m.w : m.y;
+  }
+  const uint32_t pr[2] = {a ^ ma, b ^ mb};
+  double acc = 0.0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int j = 4 * lane + q;
+    const uint32_t bits = (q & 1) ? (pr[q >> 1] & 0xffff0000u) : (pr[q >> 1] << 16);
+    const double xv = (double)__uint_as_float(bits);
+    acc += (__popc(e & j) & 1) ? -xv : xv;
+  }
+  return warp_sum_d(acc);
+}
+
+// E4M3 code of r (>= 0) with the conversion instruction, nearest-even, satfinite.
+__device__ __forceinline__ uint32_t e4m3_pair(float r_lo, float r_hi) {
+  uint32_t out;
+  asm("{.reg .b16 t; cvt.rn.satfinite.e4m3x2.f32 t, %1, %2; cvt.u32.u16 %0, t;}"
+      : "=r"(out) : "f"(r_hi), "f"(r_lo));
+  return out;   // bits 0-7: code(r_lo), bits 8-15: code(r_hi)
+}
+
+// 1 / value(E4M3 code) for a non-zero code (exact power-of-two scaling of a
+// rounded reciprocal of the significand).
+__device__ __forceinline__ float e4m3_recip(uint32_t c) {
+  const uint32_t e = (c >> 3) & 15u, m = c & 7u;
+  if (e == 0) return 512.0f / (float)m;                  // m * 2^-9
+  const float r = 1.0f / (1.0f + 0.125f * (float)m);     // (1 + m/8)^-1
+  return ldexpf(r, 7 - (int)e);
+}
+
+// ---------------------------------------------------------------- NVFP4
+// kMode 0: quantize with the static/dynamic tensor scale.
+// kMode 1: dynamic-scale statistics (row max and bound), no outputs.
+template <int kMode>
+__global__ void __launch_bounds__(kThreads)
+k_blk128_nvfp4(Params P) {
+  const int lane = threadIdx.x & 31;
+  float t = 0.0f, c6 = 0.0f, inv_bt = 0.0f;
+  const float sqrt_b = 11.313708498984761f;  // sqrt(128), only in fp32 factors
+  if (kMode == 0) {
+    if (P.ws) {
+      const double g = __longlong_as_double((long long)P.ws->gmax_bits);
+      t = __double2float_rn((g / 11.313708498984761) / 2688.0);
+      if (blockIdx.x == 0 && threadIdx.x == 0) *P.tensor_scale = t;
+    } else {
+      t = *P.tensor_scale;
+    }
+    // r = max|S| / (sqrt(b) 6 t); c6 rounded down/up bracket handled by margins
+    c6 = (t > 0.0f) ? (float)(1.0 / (11.313708498984761 * 6.0 * (double)t)) : 0.0f;
+    inv_bt = (t > 0.0f) ? (float)(1.0 / (11.313708498984761 * (double)t)) : 0.0f;
+  }
+  (void)sqrt_b;
+  extern __shared__ __align__(16) uint4 smem4[];
+  uint4* stages = smem4 + (threadIdx.x >> 5) * 1024;      // two 8 KB stages per warp
+  uint4* smask = P.signs ? smem4 + (blockDim.x >> 5) * 1024 : nullptr;
+  if (smask) stage_signs(P.signs, P.n, smask);
+  __syncthreads();
+  const int kpr = P.n / B;                  // column blocks per row (power of two)
+  const int kpr_log2 = __ffs(kpr) - 1;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  // uniform trip count across the warp so warp-cooperative steps are safe
+  const int64_t base0 = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31);
+  if (base0 < P.units) prefetch_units(P.x, base0, P.units, stages);
+  int it = 0;
+  for (int64_t ub = base0; ub < P.units; ub += stride, ++it) {
+    const int64_t u = ub + lane;
+    const bool active = u < P.units;
+    float2 v[64];
+    const int64_t row = active ? (u >> kpr_log2) : 0;
+    uint4* stage = stages + (it & 1) * 512;
+    __syncwarp();
+    const bool more = ub + stride < P.units;
+    if (more) prefetch_units(P.x, ub + stride, P.units, stages + ((it + 1) & 1) * 512);
+    wait_prefetch(more);
+    load_transform(stage, lane, smask, (int)(u & (kpr - 1)), v);
+    if (!active) {
+#pragma unroll
+      for (int p = 0; p < 64; ++p) v[p] = make_float2(0.f, 0.f);
+    }
+    // per 16-block maxima
+    float bm[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      float m = 0.0f;
+#pragma unroll
+      for (int p = 8 * j; p < 8 * j + 8; ++p) m = fmax3(m, fabsf(v[p].x), fabsf(v[p].y));
+      bm[j] = m;
+    }
+    float mh = bm[0];
+#pragma unroll
+    for (int j = 1; j < 8; ++j) mh = fmaxf(mh, bm[j]);
+    const float E = __fmul_ru(P.e_coef, mh);
+
+    if (kMode == 1) {
+      if (active) {
+        const float lower = fmaxf(__fsub_rd(mh, E), 0.0f);
+        atomicMax(reinterpret_cast<unsigned int*>(&P.ws->rows[row].x), __float_as_uint(mh));
+        atomicMax(reinterpret_cast<unsigned int*>(&P.ws->rows[row].y), __float_as_uint(E));
+        atomicMax(&P.ws->lower_bits, __float_as_uint(lower));
+      }
+      continue;
+    }
+
+    // E4M3 block scales from the interval [m - E, m + E] (scaled by c6 with a
+    // relative margin covering every fp32 rounding on the way); sc holds the
+    // eight codes as bytes
+    uint32_t sc[2] = {0, 0};
+    uint32_t undecided = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float lo = fmaxf(bm[j] - E, 0.0f) * c6 * (1.0f - 0x1p-20f);
+      const float hi = (bm[j] + E) * c6 * (1.0f + 0x1p-20f);
+      const uint32_t cc = e4m3_pair(lo, hi);
+      sc[j >> 2] |= (cc & 0xffu) << (8 * (j & 3));
+      if ((cc & 0xffu) != (cc >> 8)) undecided |= 1u << j;
+    }
+    if (t <= 0.0f) undecided = 0;
+    // warp-cooperative exact fix-up of undecided block scales
+    unsigned todo = __ballot_sync(0xffffffffu, active && undecided != 0);
+    while (todo) {
+      const int src = __ffs(todo) - 1;
+      todo &= todo - 1;
+      const uint32_t und = __shfl_sync(0xffffffffu, undecided, src);
+      const int kk = (int)((ub + src) & (kpr - 1));
+      for (int j = 0; j < 8; ++j) {
+        if (!((und >> j) & 1u)) continue;
+        // candidates: |S_hat| >= bm[j] - 2E inside block j of thread src
+        uint32_t cand = 0;
+        if (lane == src) {
+          float thr = 0.0f, bmj = 0.0f;
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            if (q == j) bmj = bm[q];
+          thr = bmj - 2.0f * E;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            if (q != j) continue;
+#pragma unroll
+            for (int p = 0; p < 8; ++p) {
+              const float2 a = v[8 * q + p];
+              if (fabsf(a.x) >= thr) cand |= 1u << (2 * p);
+              if (fabsf(a.y) >= thr) cand |= 1u << (2 * p + 1);
+            }
+          }
+        }
+        cand = __shfl_sync(0xffffffffu, cand, src);
+        double best = 0.0;
+        while (cand) {
+          const int e = __ffs(cand) - 1;
+          cand &= cand - 1;
+          best = fmax(best, fabs(warp_exact_S(stage, smask, src, kk, 16 * j + e)));
+        }
+        const double y = best / 11.313708498984761;
+        const float r = __double2float_rn(y / (6.0 * (double)t));
+        const uint32_t code = e4m3_pair(r, r) & 0xffu;
+        if (lane == src) {
+          const int w = j >> 2, sh = 8 * (j & 3);
+          sc[w] = (sc[w] & ~(0xffu << sh)) | (code << sh);
+        }
+      }
+    }
+    // codes, two 16-blocks (one 16-byte chunk) at a time
+    uint4 cw[4];
+    const float2 zero2 = make_float2(0.0f, 0.0f);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      uint32_t words[4];
+#pragma unroll
+      for (int jj = 0; jj < 2; ++jj) {
+        const int j = 2 * k + jj;
+        const uint32_t code = (sc[j >> 2] >> (8 * (j & 3))) & 0xffu;
+        if (code != 0 && t > 0.0f) {
+          const float c = inv_bt * e4m3_recip(code);
+          const float2 c2 = make_float2(c, c);
+          float q[16];
+#pragma unroll
+          for (int p = 0; p < 8; ++p) {
+            const float2 a = fma2(v[8 * j + p], c2, zero2);   // + 0 turns -0 into +0
+            q[2 * p] = a.x;
+            q[2 * p + 1] = a.y;
+          }
+          words[2 * jj] = e2m1x8_hw(q);
+          words[2 * jj + 1] = e2m1x8_hw(q + 8);
+        } else {
+          uint32_t w0 = 0, w1 = 0;
+#pragma unroll
+          for (int p = 0; p < 4; ++p) {
+            w0 |= (v[8 * j + p].x < 0.0f ? 8u : 0u) << (8 * p);
+            w0 |= (v[8 * j + p].y < 0.0f ? 8u : 0u) << (8 * p + 4);
+            w1 |= (v[8 * j + 4 + p].x < 0.0f ? 8u : 0u) << (8 * p);
+            w1 |= (v[8 * j + 4 + p].y < 0.0f ? 8u : 0u) << (8 * p + 4);
+          }
+          words[2 * jj] = w0;
+          words[2 * jj + 1] = w1;
+        }
+      }
+      cw[k] = make_uint4(words[0], words[1], words[2], words[3]);
+    }
+    store_codes(stage, cw, P.codes, ub, P.units);
+    if (active) *reinterpret_cast<uint2*>(P.scales8 + u * (B / 16)) = make_uint2(sc[0], sc[1]);
+  }
+}
+
+// ------------------------------------------------------- INT4 asym, g128
+__device__ __forceinline__ uint32_t f16x2_pair(float lo, float hi) {
+  uint32_t out;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(out) : "f"(hi), "f"(lo));
+  return out;   // bits 0-15: fp16(lo), bits 16-31: fp16(hi)
+}
+
+__global__ void __launch_bounds__(kThreads)
+k_blk128_asym(Params P) {
+  const int lane = threadIdx.x & 31;
+  const float k15 = (float)(1.0 / (15.0 * 11.313708498984761));
+  extern __shared__ __align__(16) uint4 smem4[];
+  uint4* stages = smem4 + (threadIdx.x >> 5) * 1024;
+  uint4* smask = P.signs ? smem4 + (blockDim.x >> 5) * 1024 : nullptr;
+  if (smask) stage_signs(P.signs, P.n, smask);
+  __syncthreads();
+  const int kpr = P.n / B;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const int64_t base0 = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31);
+  if (base0 < P.units) prefetch_units(P.x, base0, P.units, stages);
+  int it = 0;
+  for (int64_t ub = base0; ub < P.units; ub += stride, ++it) {
+    const int64_t u = ub + lane;
+    const bool active = u < P.units;
+    float2 v[64];
+    uint4* stage = stages + (it & 1) * 512;
+    __syncwarp();
+    const bool more = ub + stride < P.units;
+    if (more) prefetch_units(P.x, ub + stride, P.units, stages + ((it + 1) & 1) * 512);
+    wait_prefetch(more);
+    load_transform(stage, lane, smask, (int)(u & (kpr - 1)), v);
+    if (!active) {
+#pragma unroll
+      for (int p = 0; p < 64; ++p) v[p] = make_float2(0.f, 0.f);
+    }
+    float mx = -FLT_MAX, mn = FLT_MAX;
+#pragma unroll
+    for (int p = 0; p < 64; ++p) {
+      mx = fmax3(mx, v[p].x, v[p].y);
+      mn = fmin3(mn, v[p].x, v[p].y);
+    }
+    const float E = __fmul_ru(P.e_coef, fmaxf(fabsf(mx), fabsf(mn)));
+    // scale16 = fp16((mx - mn) / (15 sqrt(b))) over the interval of (mx, mn)
+    const float r_lo = fmaxf(mx - mn - 2.0f * E, 0.0f) * k15 * (1.0f - 0x1p-20f);
+    const float r_hi = (mx - mn + 2.0f * E) * k15 * (1.0f + 0x1p-20f);
+    const uint32_t hh = f16x2_pair(r_lo, r_hi);
+    uint32_t s16 = hh & 0xffffu;
+    bool decided = s16 == (hh >> 16);
+    float zf = 0.0f;
+    if (decided && s16 != 0) {
+      // z = rint(-mn / (sqrt(b) s16)) over the interval of mn
+      const float inv = 1.0f / (11.313708498984761f * f16_bits_to_f32((uint16_t)s16));
+      const float z_hi = rintf(-(mn - E) * inv * (1.0f + 0x1p-20f * (mn - E < 0 ? 1.f : -1.f)));
+      const float z_lo = rintf(-(mn + E) * inv * (1.0f - 0x1p-20f * (mn + E < 0 ? 1.f : -1.f)));
+      decided = z_hi == z_lo;
+      zf = z_lo;
+    }
+    // warp-cooperative exact extremes for undecided groups
+    unsigned todo = __ballot_sync(0xffffffffu, active && !decided);
+    while (todo) {
+      const int src = __ffs(todo) - 1;
+      todo &= todo - 1;
+      const int kk = (int)((ub + src) & (kpr - 1));
+      uint32_t cmax[4] = {0, 0, 0, 0}, cmin[4] = {0, 0, 0, 0};
+      if (lane == src) {
+        const float th = mx - 2.0f * E, tl = mn + 2.0f * E;
+#pragma unroll
+        for (int p = 0; p < 64; ++p) {
+          if (v[p].x >= th) cmax[p >> 4] |= 1u << (2 * (p & 15));
+          if (v[p].y >= th) cmax[p >> 4] |= 1u << (2 * (p & 15) + 1);
+          if (v[p].x <= tl) cmin[p >> 4] |= 1u << (2 * (p & 15));
+          if (v[p].y <= tl) cmin[p >> 4] |= 1u << (2 * (p & 15) + 1);
+        }
+      }
+      double smax = -DBL_MAX, smin = DBL_MAX;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        uint32_t a = __shfl_sync(0xffffffffu, cmax[w], src);
+        uint32_t b = __shfl_sync(0xffffffffu, cmin[w], src);
+        uint32_t any = a | b;
+        while (any) {
+          const int e = __ffs(any) - 1;
+          any &= any - 1;
+          const double s = warp_exact_S(stage, smask, src, kk, 32 * w + e);
+          if ((a >> e) & 1u) smax = fmax(smax, s);
+          if ((b >> e) & 1u) smin = fmin(smin, s);
+        }
+      }
+      if (lane == src) {
+        const double ymx = smax / 11.313708498984761, ymn = smin / 11.313708498984761;
+        s16 = f64_to_f16_bits((ymx - ymn) / 15.0);
+        const double sd = f16_bits_to_f64((uint16_t)s16);
+        zf = sd > 0.0 ? (float)rint(-ymn / sd) : 0.0f;
+        decided = true;
+      }
+    }
+    uint32_t words[16];
+    if (s16 != 0) {
+      const float c = 1.0f / (11.313708498984761f * f16_bits_to_f32((uint16_t)s16));
+      const float2 c2 = make_float2(c, c);
+      // (S c) + (1.5 2^23 + z) rounds S c + z to an integer in the low bits
+      const float magic = 12582912.0f + zf;
+      const float2 m2 = make_float2(magic, magic);
+#pragma unroll
+      for (int w = 0; w < 16; ++w) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          const float2 a = fma2(v[4 * w + p], c2, m2);
+          int qx = __float_as_int(a.x) - 0x4B400000;
+          int qy = __float_as_int(a.y) - 0x4B400000;
+          qx = min(max(qx, 0), 15);
+          qy = min(max(qy, 0), 15);
+          word |= ((uint32_t)qx << (8 * p)) | ((uint32_t)qy << (8 * p + 4));
+        }
+        words[w] = word;
+      }
+    } else {
+#pragma unroll
+      for (int w = 0; w < 16; ++w) words[w] = 0;
+      zf = 0.0f;
+    }
+    uint4 cw[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      cw[k] = make_uint4(words[4 * k], words[4 * k + 1], words[4 * k + 2], words[4 * k + 3]);
+    store_codes(stage, cw, P.codes, ub, P.units);
+    if (active) {
+      uint16_t zh;
+      asm("cvt.rn.f16.f32 %0, %1;" : "=h"(zh) : "f"(zf));
+      P.scales16[u] = (uint16_t)s16;
+      P.zeros16[u] = zh;
+    }
+  }
+}
+
+}  // namespace blk
+
+// ------------------------------------------------------------- launchers
+namespace {
+size_t blk_smem(int n, bool signs) {
+  return (size_t)(blk::kThreads / 32) * 1024 * 16 + (signs ? (size_t)n / 8 * 16 : 0);
+}
+
+int blk_grid(const void* kernel, int64_t units, size_t smem) {
+  int dev = 0, sms = 0, per_sm = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (smem > 48 * 1024)
+    cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, blk::kThreads, smem);
+  if (per_sm < 1) per_sm = 1;
+  const int64_t need = (units + blk::kThreads - 1) / blk::kThreads;
+  const int64_t cap = (int64_t)sms * per_sm;
+  return (int)(need < cap ? need : cap);
+}
+
+float e_coef_128() {
+  const double u = 0x1p-24, L = 7.0;
+  const double gam = L * u / (1.0 - L * u);
+  const double c = gam * std::sqrt(128.0);
+  return (float)((c / (1.0 - c)) * 1.001);
+}
+}  // namespace
+
+bool blk128_supported(const Geometry& g, int dtype) {
+  const int kpr = g.n / 128;
+  return dtype == 1 && g.b == 128 && !g.paley && g.n % 128 == 0 && (kpr & (kpr - 1)) == 0;
+}
+
+cudaError_t launch_blk128_nvfp4(const void* x, int64_t tokens, const Geometry& g,
+                                const int8_t* signs, uint8_t* codes, uint8_t* bscales,
+                                float* tensor_scale, NvWorkspace* ws, cudaStream_t s) {
+  blk::Params P{};
+  P.x = static_cast<const uint16_t*>(x);
+  P.signs = signs;
+  P.codes = codes;
+  P.scales8 = bscales;
+  P.tensor_scale = tensor_scale;
+  P.ws = ws;
+  P.units = tokens * (g.n / blk::B);
+  P.n = g.n;
+  P.e_coef = e_coef_128();
+  if (ws) {
+    cudaError_t e = cudaMemsetAsync(ws, 0, kNvWorkspaceHeader + (size_t)tokens * sizeof(float2), s);
+    if (e != cudaSuccess) return e;
+    auto k1 = blk::k_blk128_nvfp4<1>;
+    const size_t sm1 = blk_smem(g.n, signs != nullptr);
+    k1<<<blk_grid((const void*)k1, P.units, sm1), blk::kThreads, sm1, s>>>(P);
+    e = launch_nvfp4_global(x, 1, tokens, g, signs, ws, s);
+    if (e != cudaSuccess) return e;
+  }
+  auto k0 = blk::k_blk128_nvfp4<0>;
+  const size_t sm0 = blk_smem(g.n, signs != nullptr);
+  k0<<<blk_grid((const void*)k0, P.units, sm0), blk::kThreads, sm0, s>>>(P);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_blk128_asym(const void* x, int64_t tokens, const Geometry& g,
+                               const int8_t* signs, uint8_t* codes, uint16_t* scales,
+                               uint16_t* zeros, cudaStream_t s) {
+  blk::Params P{};
+  P.x = static_cast<const uint16_t*>(x);
+  P.signs = signs;
+  P.codes = codes;
+  P.scales16 = scales;
+  P.zeros16 = zeros;
+  P.units = tokens * (g.n / blk::B);
+  P.n = g.n;
+  P.e_coef = e_coef_128();
+  auto k = blk::k_blk128_asym;
+  const size_t sm = blk_smem(g.n, signs != nullptr);
+  k<<<blk_grid((const void*)k, P.units, sm), blk::kThreads, sm, s>>>(P);
+  return cudaGetLastError();
+}
+
+}  // namespace kq

@@ -34,6 +34,36 @@ cudaError_t launch_int4_asym(const void* x, int dtype, int64_t tokens, const Geo
 cudaError_t launch_nvfp4(const void* x, int dtype, int64_t tokens, const Geometry& g,
                          const int8_t* signs, uint8_t* codes, uint8_t* bscales,
                          float* tensor_scale, NvWorkspace* ws, cudaStream_t s);
+cudaError_t launch_nvfp4_global(const void* x, int dtype, int64_t tokens, const Geometry& g,
+                                const int8_t* signs, NvWorkspace* ws, cudaStream_t s);
+
+// Fast kernels for 128-wide Hadamard blocks on bf16 rows (kq_block.cu).
+bool blk128_supported(const Geometry& g, int dtype);
+cudaError_t launch_blk128_nvfp4(const void* x, int64_t tokens, const Geometry& g,
+                                const int8_t* signs, uint8_t* codes, uint8_t* bscales,
+                                float* tensor_scale, NvWorkspace* ws, cudaStream_t s);
+cudaError_t launch_blk128_asym(const void* x, int64_t tokens, const Geometry& g,
+                               const int8_t* signs, uint8_t* codes, uint16_t* scales,
+                               uint16_t* zeros, cudaStream_t s);
+
+// Warp-per-row kernels for full-row transforms of 2048 or 4096 (kq_rowwarp.cu).
+bool rowwarp_supported(const Geometry& g, int dtype);
+cudaError_t launch_rowwarp_int4(const void* x, int dtype, int64_t tokens, const Geometry& g,
+                                const int8_t* signs, uint8_t* codes, float* scales,
+                                cudaStream_t s);
+cudaError_t launch_rowwarp_nvfp4(const void* x, int dtype, int64_t tokens, const Geometry& g,
+                                 const int8_t* signs, uint8_t* codes, uint8_t* bscales,
+                                 float* tensor_scale, NvWorkspace* ws, cudaStream_t s);
+
+// Tensor-core kernels for full-row 4096 transforms of bf16 rows (kq_tc.cu).
+bool tc_row_supported(const Geometry& g, int dtype);
+cudaError_t launch_tc_nvfp4(const void* x, int64_t tokens, const Geometry& g,
+                            const int8_t* signs, uint8_t* codes, uint8_t* bscales,
+                            float* tensor_scale, NvWorkspace* ws, cudaStream_t s);
+cudaError_t launch_tc_rot(const void* x, int64_t tokens, const Geometry& g, const int8_t* signs,
+                          float* out, cudaStream_t s);
+int tc_error_flag();
+
 cudaError_t launch_dequant(int fmt, const uint8_t* codes, const void* scales,
                            const void* zeros, const float* tensor_scale, int64_t tokens,
                            int n, int group, float* out, cudaStream_t s);

@@ -538,8 +538,10 @@ k_nvfp4_global(const T* __restrict__ x, const int8_t* __restrict__ signs,
     if ((double)st.x + (double)st.y < (double)L) continue;   // uniform per CTA
     const T* xr = x + row * g.n;
     transform_row(xr, signs, buf, g, false);
+    // candidates from this kernel's own fp32 values and their own bound
+    const double Eg = error_bound(g, row_absmax(buf, g.n, red));
     const double best = exact_max_abs(xr, signs, g, buf, 0, g.n,
-                                      thr_down((double)L - (double)st.y), red);
+                                      thr_down((double)L - Eg), red);
     if (threadIdx.x == 0)
       atomicMax(&ws->gmax_bits, (unsigned long long)__double_as_longlong(best));
     __syncthreads();
@@ -713,6 +715,21 @@ cudaError_t launch_nvfp4(const void* x, int dtype, int64_t tokens, const Geometr
     auto k = k_nvfp4<float>;
     k<<<grid_for((const void*)k, smem, tokens), kThreads, smem, s>>>(
         static_cast<const float*>(x), signs, codes, bscales, tensor_scale, ws, tokens, g);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_nvfp4_global(const void* x, int dtype, int64_t tokens, const Geometry& g,
+                                const int8_t* signs, NvWorkspace* ws, cudaStream_t s) {
+  const size_t smem_stats = (size_t)g.n * 4 + 64 * 8;
+  if (dtype == 1) {
+    auto k2 = k_nvfp4_global<uint16_t>;
+    k2<<<grid_for((const void*)k2, smem_stats, tokens), kThreads, smem_stats, s>>>(
+        static_cast<const uint16_t*>(x), signs, ws, tokens, g);
+  } else {
+    auto k2 = k_nvfp4_global<float>;
+    k2<<<grid_for((const void*)k2, smem_stats, tokens), kThreads, smem_stats, s>>>(
+        static_cast<const float*>(x), signs, ws, tokens, g);
   }
   return cudaGetLastError();
 }
