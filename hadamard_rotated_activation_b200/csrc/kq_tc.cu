@@ -27,10 +27,11 @@
 // recomputed exactly (fp64) from the staged input, which stays in shared
 // memory until the epilogue releases its stage.
 //
-// Warp roles (16 warps): 0 TMA producer, 1 MMA issuer + TMEM owner, 2-3 sign
-// flip and sum|x| in shared memory (one warp per token), 4-15 epilogue (three groups of four warps, one per
-// TMEM accumulator; warp w reads TMEM lane quarter w % 4).  Every wait on an
-// mbarrier is bounded; on timeout the kernel records an error code and returns.
+// Warp roles (14 warps): 0 TMA producer, 1 MMA issuer + TMEM owner, 2-5 sign
+// flip and sum|x| in shared memory (two warps per token), 6-13 epilogue (two
+// groups of four warps, one per TMEM accumulator; warp w reads TMEM lane
+// quarter w % 4).  Every wait on an mbarrier is bounded; on timeout the kernel
+// records an error code and returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -46,8 +47,10 @@ namespace kq {
 namespace tc {
 
 constexpr int kStages = 8;
-constexpr int kGroups = 3;                     // epilogue groups = TMEM accumulators
-constexpr int kThreads = 512;                  // 16 warps
+constexpr int kGroups = 2;                     // epilogue groups = TMEM accumulators
+constexpr int kSignWarps = 4;                  // two per token
+constexpr int kEpiWarps = 4 * kGroups;
+constexpr int kThreads = 32 * (2 + kSignWarps + kEpiWarps);   // 14 warps
 constexpr int kTileRows = 128;                 // rows of the [T*64, 64] view per tile
 constexpr uint32_t kTileBytes = kTileRows * 64 * 2;    // 16 KB
 constexpr long long kWaitCycles = 4000000000ll;   // about 2 s at 2 GHz
@@ -192,11 +195,17 @@ __device__ __forceinline__ uint32_t e4m3_pair(float r_lo, float r_hi) {
       : "=r"(out) : "f"(r_hi), "f"(r_lo));
   return out;
 }
+// 1 / value of a non-zero E4M3 code: a rounded reciprocal of the significand
+// (table folded at compile time) scaled by an exact power of two.
 __device__ __forceinline__ float e4m3_recip(uint32_t c) {
   const uint32_t e = (c >> 3) & 15u, m = c & 7u;
-  if (e == 0) return 512.0f / (float)m;
-  const float r = 1.0f / (1.0f + 0.125f * (float)m);
-  return ldexpf(r, 7 - (int)e);
+  if (e == 0) return 512.0f / (float)m;                 // subnormal: m * 2^-9
+  constexpr float kR0 = 1.0f / 1.0f, kR1 = 1.0f / 1.125f, kR2 = 1.0f / 1.25f,
+                  kR3 = 1.0f / 1.375f, kR4 = 1.0f / 1.5f, kR5 = 1.0f / 1.625f,
+                  kR6 = 1.0f / 1.75f, kR7 = 1.0f / 1.875f;
+  const float r = m < 4 ? (m < 2 ? (m == 0 ? kR0 : kR1) : (m == 2 ? kR2 : kR3))
+                        : (m < 6 ? (m == 4 ? kR4 : kR5) : (m == 6 ? kR6 : kR7));
+  return __uint_as_float(__float_as_uint(r) + ((7u - e) << 23));   // r * 2^(7-e)
 }
 
 // Byte offset of element (row r, column col) of a 128-byte-swizzled matrix
@@ -240,9 +249,9 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
   uint8_t* sA = smem;                                   // 32 KB: A = I_2 kron H_64
   uint8_t* sB = smem + 32768;                           // kStages x 16 KB
   uint4* smask = reinterpret_cast<uint4*>(sB + kStages * kTileBytes);   // 512 chunks
-  uint4* scode = smask + 512;                           // 12 warps x 1 KB code staging
-  float* sabs = reinterpret_cast<float*>(scode + 12 * 64);   // sum|x| per (stage, token)
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sabs + 2 * kStages);
+  uint4* scode = smask + 512;                           // epilogue warps x 1 KB code staging
+  float* sabs = reinterpret_cast<float*>(scode + kEpiWarps * 64);   // sum|x| per (stage, sign warp)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sabs + kSignWarps * kStages);
   uint64_t* full = bars;                                // TMA landed
   uint64_t* ready = bars + kStages;                     // signs applied
   uint64_t* empty = bars + 2 * kStages;                 // epilogue done with the stage
@@ -275,7 +284,7 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&ready[s], 64);
+      mbar_init(&ready[s], 32 * kSignWarps);
       mbar_init(&empty[s], 128);
     }
     for (int d = 0; d < kGroups; ++d) {
@@ -342,18 +351,18 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
       for (int64_t k = issued > kGroups ? issued - kGroups : 0; k < issued; ++k)
         mbar_wait(&tfull[k % kGroups], (uint32_t)(k / kGroups) & 1);
     }
-  } else if (warp < 4) {
-    // ================= sign flip + sum|x|: warp 2 token 0, warp 3 token 1
-    const int tk = warp - 2;
+  } else if (warp < 2 + kSignWarps) {
+    // ================= sign flip + sum|x|: warps 2-3 token 0, warps 4-5 token 1
+    const int sw = warp - 2;                 // 0..3: token sw/2, half sw%2
     for (int64_t k = 0; k < my_tiles; ++k) {
       const int s = (int)(k % kStages);
       if (!mbar_wait(&full[s], (uint32_t)(k / kStages) & 1)) break;
       uint8_t* st = sB + s * kTileBytes;
       float2 acc = make_float2(0.0f, 0.0f);
 #pragma unroll 4
-      for (int j = 0; j < 16; ++j) {
-        // physical chunk idx of this token: row r, swizzled chunk pc
-        const int idx = tk * 512 + lane + 32 * j;
+      for (int j = 0; j < 8; ++j) {
+        // physical chunk idx of this token half: row r, swizzled chunk pc
+        const int idx = sw * 256 + lane + 32 * j;
         const int r = idx >> 3, pc = idx & 7;
         const int c = pc ^ (r & 7);
         uint4* p = reinterpret_cast<uint4*>(st + idx * 16);
@@ -369,8 +378,8 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
         const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float2 ab = make_float2(__uint_as_float((ww[e] << 16) & 0x7fffffffu),
-                                        __uint_as_float(ww[e] & 0x7fff0000u));
+          const uint32_t wa = ww[e] & 0x7fff7fffu;      // |x| of both halves
+          const float2 ab = make_float2(__uint_as_float(wa << 16), __uint_as_float(wa & 0xffff0000u));
           uint64_t ua = *reinterpret_cast<const uint64_t*>(&ab),
                    uc = *reinterpret_cast<uint64_t*>(&acc), rr;
           asm("add.rn.f32x2 %0, %1, %2;" : "=l"(rr) : "l"(uc), "l"(ua));
@@ -380,25 +389,25 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
       float sum = acc.x + acc.y;
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-      if (lane == 0) sabs[s * 2 + tk] = sum;
+      if (lane == 0) sabs[s * kSignWarps + sw] = sum;
       if (signs) fence_async_smem();
       __syncwarp();
       mbar_arrive(&ready[s]);
     }
   } else {
-    // ================= epilogue: group g of warps 4+4g .. 7+4g
-    const int g = (warp - 4) >> 2;
+    // ================= epilogue: group g of warps 6+4g .. 9+4g
+    const int g = (warp - 2 - kSignWarps) >> 2;
     const int q = warp & 3;                   // TMEM lane quarter
     const int m = q * 32 + lane;              // accumulator row = (token in tile, block o)
     const int tr = m >> 6, o = m & 63;
-    const int ew = warp - 4;                  // epilogue warp index 0..11
+    const int ew = warp - 2 - kSignWarps;     // epilogue warp index
     uint4* wcode = scode + ew * 64;
     float t = 0.0f, c6 = 0.0f, inv_bt = 0.0f;
     if (kMode == kNvfp4) {
       if (P.ws) {
         const double gm = __longlong_as_double((long long)P.ws->gmax_bits);
         t = __double2float_rn((gm / kSqrtN) / 2688.0);
-        if (blockIdx.x == 0 && threadIdx.x == 128) *P.tensor_scale = t;
+        if (blockIdx.x == 0 && ew == 0 && lane == 0) *P.tensor_scale = t;
       } else {
         t = *P.tensor_scale;
       }
@@ -453,7 +462,9 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
         bm[j] = mm;
       }
       // |S_hat - S| <= E for every output of the token (sum|x| rounded up)
-      const float E = __fmul_ru(P.e_coef, sabs[s * 2 + tr] * 1.001f);
+      const float E =
+          __fmul_ru(P.e_coef, (sabs[s * kSignWarps + 2 * tr] + sabs[s * kSignWarps + 2 * tr + 1]) *
+                                  1.001f);
 
       if (kMode == kRot) {
         if (valid) {
@@ -634,7 +645,7 @@ bool make_tmap(CUtensorMap* map, const void* x, int64_t rows) {
 }
 
 constexpr size_t kSmemBytes = 1024 + 32768 + tc::kStages * tc::kTileBytes + 512 * 16 +
-                              12 * 64 * 16 + 2 * tc::kStages * 4 + 512;
+                              tc::kEpiWarps * 64 * 16 + tc::kSignWarps * tc::kStages * 4 + 512;
 
 template <int kMode>
 cudaError_t launch_tc(const void* x, const int8_t* signs, tc::Params& P, cudaStream_t s) {
