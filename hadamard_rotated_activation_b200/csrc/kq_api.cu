@@ -85,7 +85,7 @@ KQ_API kq_status kq_rht(const void* x, int dtype, int64_t tokens, int dim, int b
   if (flags & ~KQ_INVERSE) return KQ_ERR_INVALID_ARG;
   if (!aligned(out, 16)) return KQ_ERR_MISALIGNED;
   if (tokens == 0) return KQ_OK;
-  if (!(flags & KQ_INVERSE) && kq::tc_row_supported(g, dtype))
+  if (!(flags & KQ_INVERSE) && kq::tc_row_supported(g, dtype, x, tokens))
     return finish(kq::launch_tc_rot(x, tokens, g, signs, out,
                                     reinterpret_cast<cudaStream_t>(stream)));
   return finish(kq::launch_rht(x, dtype, tokens, g, signs, out, (flags & KQ_INVERSE) ? 1 : 0,
@@ -153,7 +153,7 @@ KQ_API kq_status kq_rht_quant_nvfp4(const void* x, int dtype, int64_t tokens, in
     return finish(kq::launch_blk128_nvfp4(x, tokens, g, signs, codes, block_scales,
                                           tensor_scale, ws,
                                           reinterpret_cast<cudaStream_t>(stream)));
-  if (kq::tc_row_supported(g, dtype) && aligned(block_scales, 8))
+  if (kq::tc_row_supported(g, dtype, x, tokens) && aligned(block_scales, 8))
     return finish(kq::launch_tc_nvfp4(x, tokens, g, signs, codes, block_scales, tensor_scale,
                                       ws, reinterpret_cast<cudaStream_t>(stream)));
   if (kq::rowwarp_supported(g, dtype) && aligned(block_scales, 8))

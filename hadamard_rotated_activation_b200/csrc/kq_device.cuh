@@ -180,6 +180,23 @@ __device__ __forceinline__ int warp_min_i(int v) {
   for (int o = 16; o > 0; o >>= 1) v = min(v, __shfl_xor_sync(0xffffffffu, v, o));
   return v;
 }
+// Exact fp64 images of the two bf16 values packed in `w` (low half first),
+// scaled by 2^-896: the bf16 bit pattern is placed in the high word of a
+// double so that its 8-bit exponent field becomes the double's (biased 1023
+// instead of 127).  Zeros and bf16 subnormals land on double zeros and
+// subnormals with the same 2^-896 factor, so the mapping is exact for every
+// finite bf16; infinities and NaNs are NOT preserved (callers route non-finite
+// rows elsewhere).  Three integer operations per value, no conversion unit.
+__device__ __forceinline__ void bf16x2_to_f64_scaled(uint32_t w, double& lo, double& hi) {
+  const uint32_t flo = w << 16, fhi = w & 0xffff0000u;     // the fp32 images
+  const uint32_t hlo = (flo & 0x80000000u) | ((flo >> 3) & 0x0fffffffu);
+  const uint32_t hhi = (fhi & 0x80000000u) | ((fhi >> 3) & 0x0fffffffu);
+  lo = __hiloint2double((int)hlo, 0);
+  hi = __hiloint2double((int)hhi, 0);
+}
+// Undoes the 2^-896 scaling of bf16x2_to_f64_scaled (exact).
+constexpr double kF64Unscale = 0x1p+896;
+
 __device__ __forceinline__ double warp_sum_d(double v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

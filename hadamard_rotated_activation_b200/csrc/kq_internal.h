@@ -56,7 +56,7 @@ cudaError_t launch_rowwarp_nvfp4(const void* x, int dtype, int64_t tokens, const
                                  float* tensor_scale, NvWorkspace* ws, cudaStream_t s);
 
 // Tensor-core kernels for full-row 4096 transforms of bf16 rows (kq_tc.cu).
-bool tc_row_supported(const Geometry& g, int dtype);
+bool tc_row_supported(const Geometry& g, int dtype, const void* x, int64_t tokens);
 cudaError_t launch_tc_nvfp4(const void* x, int64_t tokens, const Geometry& g,
                             const int8_t* signs, uint8_t* codes, uint8_t* bscales,
                             float* tensor_scale, NvWorkspace* ws, cudaStream_t s);

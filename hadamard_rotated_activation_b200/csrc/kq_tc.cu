@@ -1,37 +1,48 @@
 // Tensor-core (tcgen05) kernels for full-row Hadamard transforms of 4096-wide
 // rows (the hidden size of "Bug: Qwen3-8B integration issue", Model Details).
 //
-// A row of n = 4096 values is viewed as 64 blocks of 64 (index i = o*64 + beta).
-// Sylvester H_4096 = H_64 kron H_64 in natural order, so the transform splits
+// A row of n = 4096 values is viewed as 128 rows of 32 (index j = a*32 + beta).
+// Sylvester H_4096 = H_128 kron H_32 in natural order, so the transform splits
 // into
-//   (1) a cross-block mix  D[o][beta] = sum_a H_64[o][a] x'[a*64 + beta]
-//       -- a dense +-1 contraction over the block index, run on the tensor
-//       cores: D (TMEM, fp32) = A * B with A = I_2 kron H_64 (bf16 +-1,
-//       K-major, built in shared memory once) and B = 128 consecutive
-//       64-element blocks of x' (the sign-flipped input, MN-major, one TMA box
-//       per tile), i.e. two tokens per tile;
-//   (2) the in-block H_64 over beta, run by the epilogue thread that owns TMEM
-//       lane (token, o): it reads the 64 columns of its lane and finishes the
-//       transform with six butterfly stages in fp32 (five on f32x2 pairs).
-// The thread then holds the 64 contiguous outputs o*64 .. o*64+63 of its
-// token: four NVFP4 16-blocks, quantized in registers.  (QuaRot reviews,
-// review 1 Summary: Walsh-Hadamard algorithm; NVFP4 thread: NVFP4 format.)
+//   (1) a mix over the row index a: D[o][beta] = sum_a H_128[o][a] x'[a*32+beta]
+//       -- a dense +-1 contraction, run on the tensor cores: D (TMEM, fp32) =
+//       A * B with A = H_128 (bf16 +-1, K-major, built in shared memory once)
+//       and B = the sign-flipped input x' of four tokens side by side
+//       (K = a, N = token*32 + beta; MN-major, 64-byte swizzle, one TMA box
+//       per token);
+//   (2) the H_32 over beta, run by the epilogue thread that owns TMEM lane o:
+//       it reads the 32 columns of a token and finishes the transform with five
+//       butterfly stages in fp32 (four on f32x2 pairs).
+// The thread then holds the 32 contiguous outputs o*32 .. o*32+31 of the
+// token: two NVFP4 16-blocks, quantized in registers and stored as one
+// 16-byte chunk.  (QuaRot reviews, review 1 Summary: Walsh-Hadamard
+// algorithm; NVFP4 thread: NVFP4 format.)
 //
-// Products of bf16 inputs with +-1 are exact; the tensor core accumulates in
-// fp32.  The error of S_hat is bounded by E = 16 u sum|x| per token: four
-// k-steps with non-zero products, each rounding its sum into the fp32
-// accumulator once (at most 2u relative each), then six fp32 butterfly stages
-// (6u).  sum|x| is accumulated by the sign-flip warps while they touch the
-// tile.  (Measured on B200: the largest error seen was 0.94 u sum|x|, on
-// inputs spanning 2^40 in magnitude.)  Scales undecided under the bound are
-// recomputed exactly (fp64) from the staged input, which stays in shared
-// memory until the epilogue releases its stage.
+// Error bound.  On sm_100a one tcgen05.mma kind::f16 step (K = 16, fp32
+// accumulate) with +-1 / bf16 operands behaves, per output, as: take the 16
+// products and the accumulator, truncate each toward zero to a multiple of
+// 2^(emax - 25) (emax = exponent of the largest of them), add exactly, and
+// truncate the sum to fp32.  (Reproduced bit for bit on adversarial operands
+// by the tensor-core rounding test.)  With P_k the sum of |x'| over the rows
+// a < 16(k+1) of a column, step k adds at most 2^-23 P_k (final truncation)
+// + 2^-25 P_k (accumulator truncation, k >= 1), plus, for inputs more than
+// 2^18 below the largest term of their step, their own truncation.  Summed
+// over the eight steps and the 32 columns that is
+//   E = 2.5 u W + 5 u (1 + 5u) sum|x| + R,   u = 2^-24,
+// with W = sum_a (8 - a/16) |x'_a| and R = 16 * 2^-25 * (sum of P_k over the
+// (step, column) pairs that hold an input below 2^-18 P_k: at most 16 inputs
+// there, each losing less than 2^-25 P_k); the 5 u term bounds the five fp32
+// butterfly stages.  The sign-flip warps compute W, sum|x| and R for each
+// token while they touch the tile.  Block scales that E leaves undecided are
+// recomputed exactly (fp64)
+// from the staged input, which stays in shared memory until the epilogue
+// releases its stage.
 //
-// Warp roles (14 warps): 0 TMA producer, 1 MMA issuer + TMEM owner, 2-5 sign
-// flip and sum|x| in shared memory (two warps per token), 6-13 epilogue (two
-// groups of four warps, one per TMEM accumulator; warp w reads TMEM lane
-// quarter w % 4).  Every wait on an mbarrier is bounded; on timeout the kernel
-// records an error code and returns.
+// Warp roles (18 warps): 0 TMA producer, 1 MMA issuer + TMEM owner, 2-9 sign
+// flip and error bound (two per token of a tile), 10-17 epilogue (two groups
+// of four warps; warp w reads TMEM lane quarter w % 4).  Every wait on an
+// mbarrier is bounded; on timeout the kernel records an error code and
+// returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -46,14 +57,21 @@
 namespace kq {
 namespace tc {
 
-constexpr int kStages = 8;
-constexpr int kGroups = 2;                     // epilogue groups = TMEM accumulators
-constexpr int kSignWarps = 4;                  // two per token
+constexpr int kTok = 4;                        // tokens per tile
+constexpr uint32_t kTokBytes = 128 * 32 * 2;   // one token: 128 rows of 32 bf16
+constexpr uint32_t kStageBytes = kTok * kTokBytes;   // 32 KB
+constexpr int kStages = 5;
+constexpr int kGroups = 2;                     // epilogue groups
+constexpr int kAcc = 4;                        // TMEM accumulators, multiple of kGroups
+constexpr int kAccCols = 32 * kTok;            // fp32 columns per accumulator
+constexpr int kTmemCols = kAcc * kAccCols;     // power of two >= 32
+constexpr int kSignWarps = 2 * kTok;           // two per token
 constexpr int kEpiWarps = 4 * kGroups;
-constexpr int kThreads = 32 * (2 + kSignWarps + kEpiWarps);   // 14 warps
-constexpr int kTileRows = 128;                 // rows of the [T*64, 64] view per tile
-constexpr uint32_t kTileBytes = kTileRows * 64 * 2;    // 16 KB
+constexpr int kThreads = 32 * (2 + kSignWarps + kEpiWarps);
 constexpr long long kWaitCycles = 4000000000ll;   // about 2 s at 2 GHz
+static_assert(kAcc % kGroups == 0 && (kTmemCols & (kTmemCols - 1)) == 0 && kTmemCols <= 512,
+              "accumulators: a multiple of the groups, a power-of-two column count <= 512");
+static_assert((3 * kStages + 2 * kAcc) * 8 + 4 <= 512, "barrier area");
 
 __device__ unsigned int g_tc_error = 0;        // nonzero: a wait timed out
 
@@ -65,10 +83,8 @@ struct Params {
   float* tensor_scale;
   NvWorkspace* ws;
   float* out;                   // kRot: fp32 [T, n]
-  const uint16_t* x;            // for exact fix-ups from global (unused) / debug
   int64_t tokens;
   int64_t tiles;
-  float e_coef;                 // E = e_coef * sum|x| of the token (rounded up)
 };
 
 // --------------------------------------------------------------- helpers
@@ -123,30 +139,30 @@ __device__ __forceinline__ void tc_fence_after() {
 }
 
 // Shared-memory matrix descriptor (tcgen05): start >> 4, leading and stride
-// byte offsets >> 4, version 1, layout type 2 (128-byte swizzle).
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+// byte offsets >> 4, version 1, swizzle layout (2 = 128-byte, 4 = 64-byte).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo,
+                                              uint32_t layout) {
   uint64_t d = 0;
   d |= (uint64_t)((addr >> 4) & 0x3FFFu);
   d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
   d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
   d |= (uint64_t)1 << 46;           // version
-  d |= (uint64_t)2 << 61;           // SWIZZLE_128B
+  d |= (uint64_t)layout << 61;
   return d;
 }
 
 // kind::f16 instruction descriptor: D fp32, A and B bf16, A K-major,
-// B MN-major, N = 64, M = 128.
+// B MN-major, N = 128 (four tokens x 32), M = 128.
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) | (1u << 16) |
-                            ((64u >> 3) << 17) | ((128u >> 4) << 24);
+                            ((uint32_t)(kAccCols >> 3) << 17) | ((128u >> 4) << 24);
 
 __device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
                                          uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}"
-      :: "r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate),
-         "r"(0u), "r"(0u), "r"(0u), "r"(0u));
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+      :: "r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate));
 }
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
@@ -178,11 +194,47 @@ __device__ __forceinline__ void bfly2(float2& a, float2& b) {
   a = *reinterpret_cast<float2*>(&s);
   b = *reinterpret_cast<float2*>(&d);
 }
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  uint64_t ua = *reinterpret_cast<uint64_t*>(&a), ub = *reinterpret_cast<uint64_t*>(&b), r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(ua), "l"(ub));
+  return *reinterpret_cast<float2*>(&r);
+}
 __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
   uint64_t ua = *reinterpret_cast<uint64_t*>(&a), ub = *reinterpret_cast<uint64_t*>(&b),
            uc = *reinterpret_cast<uint64_t*>(&c), r;
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(ua), "l"(ub), "l"(uc));
   return *reinterpret_cast<float2*>(&r);
+}
+__device__ __forceinline__ uint32_t min_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("min.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t redux_max(uint32_t v) {
+  uint32_t r;
+  asm volatile("redux.sync.max.u32 %0, %1, 0xffffffff;" : "=r"(r) : "r"(v));
+  return r;
+}
+__device__ __forceinline__ uint32_t redux_add(uint32_t v) {
+  uint32_t r;
+  asm volatile("redux.sync.add.u32 %0, %1, 0xffffffff;" : "=r"(r) : "r"(v));
+  return r;
+}
+__device__ __forceinline__ float pow2f(int j) {   // 2^j, -126 <= j <= 127
+  return __uint_as_float((uint32_t)(127 + j) << 23);
+}
+// Upper bound of the warp sum of v >= 0 (every lane gets it), with integer
+// reductions: each lane's value is rounded up onto the grid 2^-k, where k
+// makes the warp maximum (bit pattern mbits) less than 2^26 units, so the 32
+// terms add exactly in 32 bits.  A non-finite maximum passes through.
+__device__ __forceinline__ float warp_sum_up(float v, uint32_t mbits) {
+  if (mbits >= 0x7f800000u) return __uint_as_float(mbits);
+  if (mbits == 0) return 0.0f;
+  const int e = max((int)(mbits >> 23), 1) - 127;
+  const int k = 25 - e, k1 = k / 2, k2 = k - k1;
+  const uint32_t q = __float2uint_ru(__fmul_ru(__fmul_ru(v, pow2f(k1)), pow2f(k2)));
+  const uint32_t sum = redux_add(q);
+  return __fmul_ru(__fmul_ru(__uint2float_ru(sum), pow2f(-k1)), pow2f(-k2));
 }
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
@@ -208,31 +260,64 @@ __device__ __forceinline__ float e4m3_recip(uint32_t c) {
   return __uint_as_float(__float_as_uint(r) + ((7u - e) << 23));   // r * 2^(7-e)
 }
 
-// Byte offset of element (row r, column col) of a 128-byte-swizzled matrix
-// stored as 16 KB halves of 128 rows x 64 columns (bf16): 16-byte chunk c of
-// row r sits at chunk position c ^ (r & 7).  The input tiles are one half; the
-// 128 x 128 A operand is two.
-__device__ __forceinline__ uint32_t tile_off(int r, int col) {
-  const int h = col >> 6, c = (col >> 3) & 7, e = col & 7;
-  return (uint32_t)(h * 16384 + r * 128 + ((c ^ (r & 7)) << 4) + e * 2);
+// Byte offset of element (row m, column k) of the 128 x 128 A operand: two
+// 16 KB halves of 128 rows x 64 columns (bf16), 128-byte swizzle (16-byte
+// chunk c of row m at chunk position c ^ (m & 7)).
+__device__ __forceinline__ uint32_t a_off(int m, int k) {
+  const int h = k >> 6, c = (k >> 3) & 7, e = k & 7;
+  return (uint32_t)(h * 16384 + m * 128 + ((c ^ (m & 7)) << 4) + e * 2);
+}
+// Byte offset of 16-byte chunk c (0..3) of row a of a staged token (128 rows
+// of 64 bytes, 64-byte swizzle: chunk position c ^ ((a >> 1) & 3)).
+__device__ __forceinline__ uint32_t tok_chunk(int a, int c) {
+  return (uint32_t)(a * 64 + ((c ^ ((a >> 1) & 3)) << 4));
 }
 
-// Exact S_i of token row `tr` of a staged tile (rows tr*64 .. tr*64+63, sign-
-// flipped), warp-cooperative fp64: lane l sums columns l and l + 32 of every
-// block.  Every lane gets the result.
-__device__ __noinline__ double warp_exact_S(const uint8_t* stage, int tr, int i) {
+// Exact S_i of a staged token (sign-flipped, 64-byte swizzled), warp-
+// cooperative fp64.  Lane l reads the 16-byte chunks l, l+32, ...: chunk
+// (a, c) holds x'[a*32 + c*8 .. +7], and H[i][j] for those j is
+// (-1)^(popc(i_hi & a) + popc(i_mid & c) + popc(i_lo & e)) with i = i_hi*32 +
+// i_mid*8 + i_lo, so the Hadamard signs are two bit masks per word selected
+// per chunk.  Values enter fp64 exactly through bf16x2_to_f64_scaled, into
+// four independent accumulators.  Every lane gets the result.  Finite inputs.
+__device__ __noinline__ double warp_exact_S(const uint8_t* tok, int i) {
+  const int lane = threadIdx.x & 31;
+  const int ihi = i >> 5, imid = (i >> 3) & 3, ilo = i & 7;
+  uint32_t em[4];                   // sign bits of elements 2w, 2w+1 of a chunk
+#pragma unroll
+  for (int w = 0; w < 4; ++w)
+    em[w] = ((uint32_t)(__popc(ilo & (2 * w)) & 1) << 15) |
+            ((uint32_t)(__popc(ilo & (2 * w + 1)) & 1) << 31);
+  const uint4* base = reinterpret_cast<const uint4*>(tok);
+  double acc[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll 4
+  for (int k = 0; k < 16; ++k) {
+    const int idx = lane + 32 * k;            // physical chunk: row a, slot pc
+    const int a = idx >> 2, c = (idx & 3) ^ ((a >> 1) & 3);
+    const uint32_t flip = ((__popc(ihi & a) ^ __popc(imid & c)) & 1) ? 0x80008000u : 0u;
+    const uint4 v = base[idx];
+    const uint32_t ww[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      double lo, hi;
+      bf16x2_to_f64_scaled(ww[w] ^ em[w] ^ flip, lo, hi);
+      acc[w] += lo;
+      acc[(w + 2) & 3] += hi;
+    }
+  }
+  return warp_sum_d((acc[0] + acc[1]) + (acc[2] + acc[3])) * kF64Unscale;
+}
+
+// The same for tokens that hold an infinity or NaN (IEEE conversions, slow).
+__device__ __noinline__ double warp_exact_S_ieee(const uint8_t* tok, int i) {
   const int lane = threadIdx.x & 31;
   double acc = 0.0;
-  for (int a = 0; a < 64; ++a) {
-    const int r = tr * 64 + a;
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      const int beta = lane + 32 * q;
-      const uint16_t b = *reinterpret_cast<const uint16_t*>(stage + tile_off(r, beta));
-      const double xv = (double)__uint_as_float((uint32_t)b << 16);
-      const int j = a * 64 + beta;
-      acc += (__popc(i & j) & 1) ? -xv : xv;
-    }
+  for (int a = 0; a < 128; ++a) {
+    const int beta = lane;
+    const uint8_t* p = tok + tok_chunk(a, beta >> 3) + (beta & 7) * 2;
+    const double xv =
+        (double)__uint_as_float((uint32_t)(*reinterpret_cast<const uint16_t*>(p)) << 16);
+    acc += (__popc(i & (a * 32 + beta)) & 1) ? -xv : xv;
   }
   return warp_sum_d(acc);
 }
@@ -246,31 +331,28 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* sA = smem;                                   // 32 KB: A = I_2 kron H_64
-  uint8_t* sB = smem + 32768;                           // kStages x 16 KB
-  uint4* smask = reinterpret_cast<uint4*>(sB + kStages * kTileBytes);   // 512 chunks
-  uint4* scode = smask + 512;                           // epilogue warps x 1 KB code staging
-  float* sabs = reinterpret_cast<float*>(scode + kEpiWarps * 64);   // sum|x| per (stage, sign warp)
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sabs + kSignWarps * kStages);
+  uint8_t* sA = smem;                                   // 32 KB: A = H_128
+  uint8_t* sB = smem + 32768;                           // kStages x 32 KB
+  uint4* smask = reinterpret_cast<uint4*>(sB + kStages * kStageBytes);   // 512 chunks
+  float* sE = reinterpret_cast<float*>(smask + 512);   // error bound halves per (stage, token)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sE + kStages * kTok * 2);
   uint64_t* full = bars;                                // TMA landed
-  uint64_t* ready = bars + kStages;                     // signs applied
+  uint64_t* ready = bars + kStages;                     // signs applied, bounds written
   uint64_t* empty = bars + 2 * kStages;                 // epilogue done with the stage
-  uint64_t* tfull = bars + 3 * kStages;                 // accumulator written (kGroups)
-  uint64_t* tempty = tfull + kGroups;                   // accumulator read (kGroups)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + kGroups);
+  uint64_t* tfull = bars + 3 * kStages;                 // accumulator written (kAcc)
+  uint64_t* tempty = tfull + kAcc;                      // accumulator read (kAcc)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + kAcc);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   // ---- set-up: A operand, sign masks, barriers, TMEM
   for (int idx = threadIdx.x; idx < 128 * 128; idx += blockDim.x) {
     const int m = idx >> 7, k = idx & 127;
-    const int tm = m >> 6, o = m & 63, tk = k >> 6, a = k & 63;
-    uint16_t v = 0;
-    if (tm == tk) v = (__popc(o & a) & 1) ? 0xBF80 : 0x3F80;    // -1 / +1 in bf16
-    *reinterpret_cast<uint16_t*>(sA + tile_off(m, k)) = v;
+    const uint16_t v = (__popc(m & k) & 1) ? 0xBF80 : 0x3F80;    // -1 / +1 in bf16
+    *reinterpret_cast<uint16_t*>(sA + a_off(m, k)) = v;
   }
   for (int i = threadIdx.x; i < 512; i += blockDim.x) {
-    // chunk (a, c): columns c*8 .. c*8+7 of 64-block a = sign bytes 8 i .. 8 i + 7
+    // chunk i = (a, c): elements 8i .. 8i+7 = a*32 + c*8 .. +7
     uint4 m4 = make_uint4(0, 0, 0, 0);
     if (signs) {
       const uint2 sv = __ldg(reinterpret_cast<const uint2*>(signs) + i);
@@ -287,15 +369,15 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
       mbar_init(&ready[s], 32 * kSignWarps);
       mbar_init(&empty[s], 128);
     }
-    for (int d = 0; d < kGroups; ++d) {
+    for (int d = 0; d < kAcc; ++d) {
       mbar_init(&tfull[d], 1);
       mbar_init(&tempty[d], 128);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;"
-                 :: "r"(smem_u32(tmem_slot)));
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 :: "r"(smem_u32(tmem_slot)), "n"(kTmemCols));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   fence_async_smem();
@@ -307,7 +389,7 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
   const int64_t my_tiles = (P.tiles - blockIdx.x + gridDim.x - 1) / gridDim.x;
 
   if (warp == 0) {
-    // ================= TMA producer
+    // ================= TMA producer: one 128-row box per token
     if (lane == 0) {
       int64_t issued = 0;
       for (int64_t k = 0; k < my_tiles; ++k) {
@@ -315,8 +397,11 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
         const uint32_t use = (uint32_t)(k / kStages);
         if (k >= kStages && !mbar_wait(&empty[s], (use - 1) & 1)) break;
         const int64_t tile = blockIdx.x + k * gridDim.x;
-        mbar_expect_tx(&full[s], kTileBytes);
-        tma_load_2d(sB + s * kTileBytes, &tmap, 0, (int)(tile * kTileRows), &full[s]);
+        mbar_expect_tx(&full[s], kStageBytes);
+#pragma unroll
+        for (int t = 0; t < kTok; ++t)
+          tma_load_2d(sB + s * kStageBytes + t * kTokBytes, &tmap, 0,
+                      (int)((tile * kTok + t) * 128), &full[s]);
         issued = k + 1;
       }
       // no copy may still be in flight when the CTA exits (matters only after
@@ -330,235 +415,285 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
       int64_t issued = 0;
       for (int64_t k = 0; k < my_tiles; ++k) {
         const int s = (int)(k % kStages);
-        const int d = (int)(k % kGroups);
+        const int d = (int)(k % kAcc);
         if (!mbar_wait(&ready[s], (uint32_t)(k / kStages) & 1)) break;
-        if (k >= kGroups && !mbar_wait(&tempty[d], (uint32_t)(k / kGroups - 1) & 1)) break;
+        if (k >= kAcc && !mbar_wait(&tempty[d], (uint32_t)(k / kAcc - 1) & 1)) break;
         tc_fence_after();
-        const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB + s * kTileBytes);
-        const uint32_t tmem_d = tmem_base + (uint32_t)(d * 64);
+        const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB + s * kStageBytes);
+        const uint32_t tmem_d = tmem_base + (uint32_t)(d * kAccCols);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
           // A: K-major, K step of 16 = 32 bytes inside a 128-byte swizzle row
-          const uint64_t adesc = smem_desc(a0 + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-          // B: MN-major (one 64-wide atom), K step of 16 rows = two 1 KB atoms
-          const uint64_t bdesc = smem_desc(b0 + ks * 2048, 16384, 1024);
+          const uint64_t adesc = smem_desc(a0 + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, 2);
+          // B: MN-major 64-byte swizzle atoms of 32 columns (one per token,
+          // 8 KB apart), 8-row groups 512 bytes apart; K step of 16 rows = 1 KB
+          const uint64_t bdesc = smem_desc(b0 + ks * 1024, kTokBytes, 512, 4);
           mma_bf16(tmem_d, adesc, bdesc, ks > 0 ? 1u : 0u);
         }
         mma_commit(&tfull[d]);
         issued = k + 1;
       }
       // the accumulators must not be released with MMAs still running
-      for (int64_t k = issued > kGroups ? issued - kGroups : 0; k < issued; ++k)
-        mbar_wait(&tfull[k % kGroups], (uint32_t)(k / kGroups) & 1);
+      for (int64_t k = issued > kAcc ? issued - kAcc : 0; k < issued; ++k)
+        mbar_wait(&tfull[k % kAcc], (uint32_t)(k / kAcc) & 1);
     }
   } else if (warp < 2 + kSignWarps) {
-    // ================= sign flip + sum|x|: warps 2-3 token 0, warps 4-5 token 1
-    const int sw = warp - 2;                 // 0..3: token sw/2, half sw%2
+    // ================= sign flip + error bound, two warps per token (chunk
+    // columns 0-1 and 2-3).  Lane (ks, c', hr) owns rows 16 ks + 8 hr .. +7 of
+    // MMA step ks in chunk column c = 2 hc + c' (8 columns beta); a lane pair
+    // (hr = 0, 1) together knows the step's smallest |x'| and sum |x'| of
+    // each column, and a prefix over the steps gives the partial sums P_ks.
+    const int sw = warp - 2, t = sw >> 1, hc = sw & 1;
+    const int ks = lane >> 2, c = 2 * hc + ((lane >> 1) & 1), hr = lane & 1;
+    const int rot = hr + 4 * (ks & 1);        // conflict-free quarter-warps
+    int rows[8];
+    uint4 msk[8];                             // this lane's sign masks, fixed for all tiles
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      rows[i] = 16 * ks + 8 * hr + ((i + rot) & 7);
+      msk[i] = smask[rows[i] * 4 + c];
+    }
     for (int64_t k = 0; k < my_tiles; ++k) {
       const int s = (int)(k % kStages);
       if (!mbar_wait(&full[s], (uint32_t)(k / kStages) & 1)) break;
-      uint8_t* st = sB + s * kTileBytes;
-      float2 acc = make_float2(0.0f, 0.0f);
-#pragma unroll 4
-      for (int j = 0; j < 8; ++j) {
-        // physical chunk idx of this token half: row r, swizzled chunk pc
-        const int idx = sw * 256 + lane + 32 * j;
-        const int r = idx >> 3, pc = idx & 7;
-        const int c = pc ^ (r & 7);
-        uint4* p = reinterpret_cast<uint4*>(st + idx * 16);
-        uint4 w = *p;
-        if (signs) {
-          const uint4 m = smask[(r & 63) * 8 + c];
-          w.x ^= m.x;
-          w.y ^= m.y;
-          w.z ^= m.z;
-          w.w ^= m.w;
-          *p = w;
-        }
-        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+      uint8_t* tok = sB + s * kStageBytes + t * kTokBytes;
+      float2 acc[4];
+      uint32_t mn[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const uint32_t wa = ww[e] & 0x7fff7fffu;      // |x| of both halves
-          const float2 ab = make_float2(__uint_as_float(wa << 16), __uint_as_float(wa & 0xffff0000u));
-          uint64_t ua = *reinterpret_cast<const uint64_t*>(&ab),
-                   uc = *reinterpret_cast<uint64_t*>(&acc), rr;
-          asm("add.rn.f32x2 %0, %1, %2;" : "=l"(rr) : "l"(uc), "l"(ua));
-          acc = *reinterpret_cast<float2*>(&rr);
+      for (int h = 0; h < 4; ++h) {
+        acc[h] = make_float2(0.0f, 0.0f);
+        mn[h] = 0x7f807f80u;                        // +inf, +inf
+      }
+#pragma unroll
+      for (int i0 = 0; i0 < 8; i0 += 4) {
+        uint4 w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          w[i] = *reinterpret_cast<const uint4*>(tok + tok_chunk(rows[i0 + i], c));
+        if (signs) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            w[i].x ^= msk[i0 + i].x;
+            w[i].y ^= msk[i0 + i].y;
+            w[i].z ^= msk[i0 + i].z;
+            w[i].w ^= msk[i0 + i].w;
+            *reinterpret_cast<uint4*>(tok + tok_chunk(rows[i0 + i], c)) = w[i];
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t ww[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const uint32_t ab = ww[h] & 0x7fff7fffu;   // |x'| of columns 2h, 2h+1
+            mn[h] = min_bf16x2(mn[h], ab);
+            acc[h] = add2(acc[h], make_float2(__uint_as_float(ab << 16),
+                                              __uint_as_float(ab & 0xffff0000u)));
+          }
         }
       }
-      float sum = acc.x + acc.y;
+      float own = 0.0f;                       // this lane's sum |x'|
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-      if (lane == 0) sabs[s * kSignWarps + sw] = sum;
+      for (int h = 0; h < 4; ++h) own += acc[h].x + acc[h].y;
+      // The lane pair (hr = 0, 1) splits the chunk's 8 columns: each keeps
+      // words 2 hr, 2 hr + 1, adds its partner's share of the step's sums and
+      // minima, and then takes the inclusive prefix over the steps: P_ks.
+      float2 pre[2];
+      uint32_t mk[2];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const float2 keep = hr ? acc[2 + j] : acc[j], send = hr ? acc[j] : acc[2 + j];
+        pre[j] = add2(keep, make_float2(__shfl_xor_sync(0xffffffffu, send.x, 1),
+                                        __shfl_xor_sync(0xffffffffu, send.y, 1)));
+        const uint32_t mkeep = hr ? mn[2 + j] : mn[j], msend = hr ? mn[j] : mn[2 + j];
+        mk[j] = min_bf16x2(mkeep, __shfl_xor_sync(0xffffffffu, msend, 1));
+      }
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const float px = __shfl_up_sync(0xffffffffu, pre[j].x, off);
+          const float py = __shfl_up_sync(0xffffffffu, pre[j].y, off);
+          if (lane >= off) pre[j] = add2(pre[j], make_float2(px, py));
+        }
+      }
+      // An input of step ks is truncated only if it is below 2^-18 of the
+      // step's largest term, which is at most P_ks; each of the <= 16 such
+      // inputs of a column then loses less than 2^-25 P_ks.  Columns whose
+      // smallest input clears the threshold lose nothing.
+      float r = 0.0f;
+      constexpr float kTinyRel = 0x1p-18f * (1.0f + 0x1p-16f);
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        if (__uint_as_float(mk[j] << 16) < pre[j].x * kTinyRel) r += pre[j].x;
+        if (__uint_as_float(mk[j] & 0xffff0000u) < pre[j].y * kTinyRel) r += pre[j].y;
+      }
+      // W weights every input by the steps from its own on
+      const float wsum = (float)(8 - ks) * own;
+      const uint32_t mbits = redux_max(max(__float_as_uint(wsum), __float_as_uint(r)));
+      const float S = warp_sum_up(own, mbits);
+      const float W = warp_sum_up(wsum, mbits);
+      const float R = warp_sum_up(r, mbits);
+      if (lane == 0) {
+        // (2.5 W + 5 (1 + 5u) S) u + 16 * 2^-25 (1 + 2^-16) R, all rounded up,
+        // with 2^-10 relative slack for the fp32 sums above
+        const float e1 = __fmul_ru(__fadd_ru(__fmul_ru(2.5f, W), __fmul_ru(5.000002f, S)),
+                                   0x1p-24f);
+        const float e = __fmul_ru(__fadd_ru(e1, __fmul_ru(R, 0x1.0001p-21f)), 1.0f + 0x1p-10f);
+        sE[(s * kTok + t) * 2 + hc] = e;
+      }
       if (signs) fence_async_smem();
       __syncwarp();
       mbar_arrive(&ready[s]);
     }
   } else {
-    // ================= epilogue: group g of warps 6+4g .. 9+4g
+    // ================= epilogue: group g of warps 10+4g .. 13+4g
     const int g = (warp - 2 - kSignWarps) >> 2;
     const int q = warp & 3;                   // TMEM lane quarter
-    const int m = q * 32 + lane;              // accumulator row = (token in tile, block o)
-    const int tr = m >> 6, o = m & 63;
+    const int o = q * 32 + lane;              // accumulator row
     const int ew = warp - 2 - kSignWarps;     // epilogue warp index
-    uint4* wcode = scode + ew * 64;
-    float t = 0.0f, c6 = 0.0f, inv_bt = 0.0f;
+    float ts = 0.0f, c6 = 0.0f, inv_bt = 0.0f;
     if (kMode == kNvfp4) {
       if (P.ws) {
         const double gm = __longlong_as_double((long long)P.ws->gmax_bits);
-        t = __double2float_rn((gm / kSqrtN) / 2688.0);
-        if (blockIdx.x == 0 && ew == 0 && lane == 0) *P.tensor_scale = t;
+        ts = __double2float_rn((gm / kSqrtN) / 2688.0);
+        if (blockIdx.x == 0 && ew == 0 && lane == 0) *P.tensor_scale = ts;
       } else {
-        t = *P.tensor_scale;
+        ts = *P.tensor_scale;
       }
-      c6 = (t > 0.0f) ? (float)(1.0 / (kSqrtN * 6.0 * (double)t)) : 0.0f;
-      inv_bt = (t > 0.0f) ? (float)(1.0 / (kSqrtN * (double)t)) : 0.0f;
+      c6 = (ts > 0.0f) ? (float)(1.0 / (kSqrtN * 6.0 * (double)ts)) : 0.0f;
+      inv_bt = (ts > 0.0f) ? (float)(1.0 / (kSqrtN * (double)ts)) : 0.0f;
     }
     for (int64_t k = g; k < my_tiles; k += kGroups) {
       const int s = (int)(k % kStages);
+      const int d = (int)(k % kAcc);
       const int64_t tile = blockIdx.x + k * gridDim.x;
-      // Both warps of a token pass the same named barriers below, so a timed-out
-      // wait does not leave the loop: the failure is recorded (g_tc_error) and
-      // the tile's outputs are not written.
-      bool ok = mbar_wait(&tfull[g], (uint32_t)(k / kGroups) & 1);
-      // the staged input (read by the fix-ups) is final once its signs are applied
+      // A timed-out wait does not leave the loop: the failure is recorded
+      // (g_tc_error) and the tile's outputs are not written.
+      bool ok = mbar_wait(&tfull[d], (uint32_t)(k / kAcc) & 1);
+      // the staged input (read by the fix-ups) and the bounds are final once
+      // the sign warps have arrived
       ok = mbar_wait(&ready[s], (uint32_t)(k / kStages) & 1) && ok;
       tc_fence_after();
-      float2 v[32];
-      {
-        uint32_t r[32];
-        const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(g * 64);
-#pragma unroll
-        for (int cb = 0; cb < 2; ++cb) {
-          tmem_ld32(taddr + cb * 32, r);
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(d * kAccCols);
+#pragma unroll 1
+      for (int t = 0; t < kTok; ++t) {
+        float2 v[16];
+        {
+          uint32_t r[32];
+          tmem_ld32(taddr + t * 32, r);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 16; ++e)
-            v[cb * 16 + e] = make_float2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
+            v[e] = make_float2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
         }
-      }
-      tc_fence_before();
-      mbar_arrive(&tempty[g]);
-      // in-block H_64 over beta
+        if (t == kTok - 1) {
+          tc_fence_before();
+          mbar_arrive(&tempty[d]);
+        }
+        // in-row H_32 over beta
 #pragma unroll
-      for (int p = 0; p < 32; ++p) {
-        const float a = v[p].x, b = v[p].y;
-        v[p] = make_float2(a + b, a - b);
-      }
+        for (int p = 0; p < 16; ++p) {
+          const float a = v[p].x, b = v[p].y;
+          v[p] = make_float2(a + b, a - b);
+        }
 #pragma unroll
-      for (int hh = 1; hh < 32; hh <<= 1)
-#pragma unroll
-        for (int p = 0; p < 32; ++p)
-          if (!(p & hh)) bfly2(v[p], v[p | hh]);
-
-      const int64_t token = tile * 2 + tr;
-      const bool valid = ok && token < P.tokens;
-      float bm[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        float mm = 0.0f;
-#pragma unroll
-        for (int p = 8 * j; p < 8 * j + 8; ++p) mm = fmax3(mm, fabsf(v[p].x), fabsf(v[p].y));
-        bm[j] = mm;
-      }
-      // |S_hat - S| <= E for every output of the token (sum|x| rounded up)
-      const float E =
-          __fmul_ru(P.e_coef, (sabs[s * kSignWarps + 2 * tr] + sabs[s * kSignWarps + 2 * tr + 1]) *
-                                  1.001f);
-
-      if (kMode == kRot) {
-        if (valid) {
-          const float inv = (float)(1.0 / kSqrtN);
-          float4* dst = reinterpret_cast<float4*>(P.out + token * N + o * 64);
+        for (int hh = 1; hh < 16; hh <<= 1)
 #pragma unroll
           for (int p = 0; p < 16; ++p)
-            dst[p] = make_float4(v[2 * p].x * inv, v[2 * p].y * inv, v[2 * p + 1].x * inv,
-                                 v[2 * p + 1].y * inv);
-        }
-        mbar_arrive(&empty[s]);
-        continue;
-      }
-      if (kMode == kNvStats) {
-        float mh = fmaxf(fmaxf(bm[0], bm[1]), fmaxf(bm[2], bm[3]));
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1)
-          mh = fmaxf(mh, __shfl_xor_sync(0xffffffffu, mh, off));
-        if (valid && lane == 0) {   // two warps per token: max through atomics
-          atomicMax(reinterpret_cast<unsigned int*>(&P.ws->rows[token].x), __float_as_uint(mh));
-          atomicMax(reinterpret_cast<unsigned int*>(&P.ws->rows[token].y), __float_as_uint(E));
-          atomicMax(&P.ws->lower_bits, __float_as_uint(fmaxf(__fsub_rd(mh, E), 0.0f)));
-        }
-        mbar_arrive(&empty[s]);
-        continue;
-      }
+            if (!(p & hh)) bfly2(v[p], v[p | hh]);
 
-      // ---- NVFP4 block scales, exact where undecided
-      uint32_t sc = 0;
-      uint32_t undecided = 0;
+        const int64_t token = tile * kTok + t;
+        const bool valid = ok && token < P.tokens;
+        float bm[2];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float lo = fmaxf(bm[j] - E, 0.0f) * c6 * (1.0f - 0x1p-20f);
-        const float hi = (bm[j] + E) * c6 * (1.0f + 0x1p-20f);
-        const uint32_t cc = e4m3_pair(lo, hi);
-        sc |= (cc & 0xffu) << (8 * j);
-        if ((cc & 0xffu) != (cc >> 8)) undecided |= 1u << j;
-      }
-      if (t <= 0.0f || !valid) undecided = 0;
-      unsigned todo = __ballot_sync(0xffffffffu, undecided != 0);
-      const uint8_t* stage = sB + s * kTileBytes;
-      while (todo) {
-        const int src = __ffs(todo) - 1;
-        todo &= todo - 1;
-        const uint32_t und = __shfl_sync(0xffffffffu, undecided, src);
-        const int src_o = (q * 32 + src) & 63;
-        for (int j = 0; j < 4; ++j) {
-          if (!((und >> j) & 1u)) continue;
-          uint32_t cand = 0;
-          if (lane == src) {
-            float bmj = 0.0f;
+        for (int j = 0; j < 2; ++j) {
+          float mm = 0.0f;
 #pragma unroll
-            for (int qq = 0; qq < 4; ++qq)
-              if (qq == j) bmj = bm[qq];
-            const float thr = bmj - 2.0f * E;
+          for (int p = 8 * j; p < 8 * j + 8; ++p) mm = fmax3(mm, fabsf(v[p].x), fabsf(v[p].y));
+          bm[j] = mm;
+        }
+        // |S_hat - S| <= E for every output of the token
+        const float E = __fadd_ru(sE[(s * kTok + t) * 2], sE[(s * kTok + t) * 2 + 1]);
+
+        if (kMode == kRot) {
+          if (valid) {
+            const float inv = (float)(1.0 / kSqrtN);
+            float4* dst = reinterpret_cast<float4*>(P.out + token * N + o * 32);
 #pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-              if (qq != j) continue;
+            for (int p = 0; p < 8; ++p)
+              dst[p] = make_float4(v[2 * p].x * inv, v[2 * p].y * inv, v[2 * p + 1].x * inv,
+                                   v[2 * p + 1].y * inv);
+          }
+          continue;
+        }
+        if (kMode == kNvStats) {
+          float mh = fmaxf(bm[0], bm[1]);
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1)
+            mh = fmaxf(mh, __shfl_xor_sync(0xffffffffu, mh, off));
+          if (valid && lane == 0) {   // four warps per token: max through atomics
+            atomicMax(reinterpret_cast<unsigned int*>(&P.ws->rows[token].x), __float_as_uint(mh));
+            atomicMax(reinterpret_cast<unsigned int*>(&P.ws->rows[token].y), __float_as_uint(E));
+            atomicMax(&P.ws->lower_bits, __float_as_uint(fmaxf(__fsub_rd(mh, E), 0.0f)));
+          }
+          continue;
+        }
+
+        // ---- NVFP4 block scales, exact where undecided
+        uint32_t sc = 0, undecided = 0;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const float lo = fmaxf(bm[j] - E, 0.0f) * c6 * (1.0f - 0x1p-20f);
+          const float hi = (bm[j] + E) * c6 * (1.0f + 0x1p-20f);
+          const uint32_t cc = e4m3_pair(lo, hi);
+          sc |= (cc & 0xffu) << (8 * j);
+          if ((cc & 0xffu) != (cc >> 8)) undecided |= 1u << j;
+        }
+        if (ts <= 0.0f || !valid) undecided = 0;
+        const bool finite = isfinite(E);   // sum|x| finite: every input finite
+        unsigned todo = __ballot_sync(0xffffffffu, undecided != 0);
+        const uint8_t* tok = sB + s * kStageBytes + t * kTokBytes;
+        while (todo) {
+          const int src = __ffs(todo) - 1;
+          todo &= todo - 1;
+          const uint32_t und = __shfl_sync(0xffffffffu, undecided, src);
+          const int src_o = q * 32 + src;
+          for (int j = 0; j < 2; ++j) {
+            if (!((und >> j) & 1u)) continue;
+            uint32_t cand = 0;
+            if (lane == src) {
+              const float thr = (j ? bm[1] : bm[0]) - 2.0f * E;
 #pragma unroll
               for (int p = 0; p < 8; ++p) {
-                const float2 a = v[8 * qq + p];
+                const float2 a = j ? v[8 + p] : v[p];
                 if (fabsf(a.x) >= thr) cand |= 1u << (2 * p);
                 if (fabsf(a.y) >= thr) cand |= 1u << (2 * p + 1);
               }
             }
+            cand = __shfl_sync(0xffffffffu, cand, src);
+            double best = 0.0;
+            while (cand) {
+              const int e = __ffs(cand) - 1;
+              cand &= cand - 1;
+              const int ii = src_o * 32 + 16 * j + e;
+              best = fmax(best, fabs(finite ? warp_exact_S(tok, ii) : warp_exact_S_ieee(tok, ii)));
+            }
+            const float rr = __double2float_rn((best / kSqrtN) / (6.0 * (double)ts));
+            const uint32_t code = e4m3_pair(rr, rr) & 0xffu;
+            if (lane == src) sc = (sc & ~(0xffu << (8 * j))) | (code << (8 * j));
           }
-          cand = __shfl_sync(0xffffffffu, cand, src);
-          double best = 0.0;
-          while (cand) {
-            const int e = __ffs(cand) - 1;
-            cand &= cand - 1;
-            best = fmax(best, fabs(warp_exact_S(stage, tr, src_o * 64 + 16 * j + e)));
-          }
-          const float r = __double2float_rn((best / kSqrtN) / (6.0 * (double)t));
-          const uint32_t code = e4m3_pair(r, r) & 0xffu;
-          if (lane == src) sc = (sc & ~(0xffu << (8 * j))) | (code << (8 * j));
         }
-      }
-      __syncwarp();
-      mbar_arrive(&empty[s]);        // staged input no longer needed
 
-      // ---- codes: 32 bytes (two 16-byte chunks) per lane
-      const float2 zero2 = make_float2(0.0f, 0.0f);
-      uint4 cw[2];
-#pragma unroll
-      for (int kk = 0; kk < 2; ++kk) {
+        // ---- codes: 16 bytes per lane, contiguous across the warp
+        const float2 zero2 = make_float2(0.0f, 0.0f);
         uint32_t words[4];
 #pragma unroll
-        for (int jj = 0; jj < 2; ++jj) {
-          const int j = 2 * kk + jj;
+        for (int j = 0; j < 2; ++j) {
           const uint32_t code = (sc >> (8 * j)) & 0xffu;
-          if (code != 0 && t > 0.0f) {
-            const float c = inv_bt * e4m3_recip(code);
-            const float2 c2 = make_float2(c, c);
+          if (code != 0 && ts > 0.0f) {
+            const float cs = inv_bt * e4m3_recip(code);
+            const float2 c2 = make_float2(cs, cs);
             float qv[16];
 #pragma unroll
             for (int p = 0; p < 8; ++p) {
@@ -566,8 +701,8 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
               qv[2 * p] = a.x;
               qv[2 * p + 1] = a.y;
             }
-            words[2 * jj] = e2m1x8_hw(qv);
-            words[2 * jj + 1] = e2m1x8_hw(qv + 8);
+            words[2 * j] = e2m1x8_hw(qv);
+            words[2 * j + 1] = e2m1x8_hw(qv + 8);
           } else {
             uint32_t w0 = 0, w1 = 0;
 #pragma unroll
@@ -577,28 +712,18 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
               w1 |= (v[8 * j + 4 + p].x < 0.0f ? 8u : 0u) << (8 * p);
               w1 |= (v[8 * j + 4 + p].y < 0.0f ? 8u : 0u) << (8 * p + 4);
             }
-            words[2 * jj] = w0;
-            words[2 * jj + 1] = w1;
+            words[2 * j] = w0;
+            words[2 * j + 1] = w1;
           }
         }
-        cw[kk] = make_uint4(words[0], words[1], words[2], words[3]);
-      }
-      // the warp's 32 lanes own 1 KB of consecutive code bytes of its token;
-      // stage through shared memory so the warp stores whole 16-byte chunks
-      __syncwarp();
-#pragma unroll
-      for (int kk = 0; kk < 2; ++kk) wcode[lane * 2 + (kk ^ (lane & 1))] = cw[kk];
-      __syncwarp();
-      if (valid) {
-        uint4* dst = reinterpret_cast<uint4*>(P.codes + token * (N / 2) + (o - lane) * 32);
-#pragma unroll
-        for (int jx = 0; jx < 2; ++jx) {
-          const int idx = lane + 32 * jx;
-          const int src = idx >> 1, kk = idx & 1;
-          dst[idx] = wcode[src * 2 + (kk ^ (src & 1))];
+        if (valid) {
+          *reinterpret_cast<uint4*>(P.codes + token * (N / 2) + o * 16) =
+              make_uint4(words[0], words[1], words[2], words[3]);
+          *reinterpret_cast<uint16_t*>(P.scales8 + token * (N / 16) + o * 2) = (uint16_t)sc;
         }
-        *reinterpret_cast<uint32_t*>(P.scales8 + token * (N / 16) + o * 4) = sc;
       }
+      __syncwarp();
+      mbar_arrive(&empty[s]);        // staged input no longer needed
     }
   }
 
@@ -606,7 +731,8 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" :: "r"(tmem_base));
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;"
+                 :: "r"(tmem_base), "n"(kTmemCols));
   }
 }
 
@@ -629,49 +755,46 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   return fn;
 }
 
-// [rows, 64] bf16 view of the input (rows of 128 bytes), 64 x 128 boxes,
-// 128-byte swizzle.
+// [rows, 32] bf16 view of the input (rows of 64 bytes), 32 x 128 boxes (one
+// token), 64-byte swizzle.
 bool make_tmap(CUtensorMap* map, const void* x, int64_t rows) {
   auto enc = get_encode();
   if (!enc) return false;
-  cuuint64_t gdim[2] = {64, (cuuint64_t)rows};
-  cuuint64_t gstride[1] = {128};
-  cuuint32_t box[2] = {64, 128};
+  cuuint64_t gdim[2] = {32, (cuuint64_t)rows};
+  cuuint64_t gstride[1] = {64};
+  cuuint32_t box[2] = {32, 128};
   cuuint32_t estride[2] = {1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), gdim, gstride,
-                   box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
-constexpr size_t kSmemBytes = 1024 + 32768 + tc::kStages * tc::kTileBytes + 512 * 16 +
-                              tc::kEpiWarps * 64 * 16 + tc::kSignWarps * tc::kStages * 4 + 512;
+constexpr size_t kSmemBytes = 1024 + 32768 + tc::kStages * tc::kStageBytes + 512 * 16 +
+                              tc::kStages * tc::kTok * 8 + 512;
 
 template <int kMode>
 cudaError_t launch_tc(const void* x, const int8_t* signs, tc::Params& P, cudaStream_t s) {
   CUtensorMap map;
-  if (!make_tmap(&map, x, P.tokens * 64)) return cudaErrorNotSupported;
+  if (!make_tmap(&map, x, P.tokens * 128)) return cudaErrorNotSupported;
   auto k = tc::k_tc4096<kMode>;
   cudaFuncSetAttribute((const void*)k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        (int)kSmemBytes);
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  P.tiles = (P.tokens * 64 + tc::kTileRows - 1) / tc::kTileRows;
+  P.tiles = (P.tokens + tc::kTok - 1) / tc::kTok;
   const int64_t grid = P.tiles < sms ? P.tiles : sms;
   k<<<(int)grid, tc::kThreads, kSmemBytes, s>>>(map, signs, P);
   return cudaGetLastError();
 }
 
-float e_coef_tc() {
-  // 4 accumulation steps x 2u + 6 fp32 stages = 14u, rounded up to 16u
-  return (float)(16.0 * 0x1p-24);
-}
-
 }  // namespace
 
-bool tc_row_supported(const Geometry& g, int dtype) {
-  return dtype == 1 && !g.paley && g.b == g.n && g.n == 4096;
+bool tc_row_supported(const Geometry& g, int dtype, const void* x, int64_t tokens) {
+  // TMA: 16-byte aligned base, int32 row coordinates
+  return dtype == 1 && !g.paley && g.b == g.n && g.n == 4096 &&
+         (reinterpret_cast<uintptr_t>(x) & 15) == 0 && tokens < (int64_t(1) << 24);
 }
 
 cudaError_t launch_tc_nvfp4(const void* x, int64_t tokens, const Geometry& g,
@@ -683,8 +806,6 @@ cudaError_t launch_tc_nvfp4(const void* x, int64_t tokens, const Geometry& g,
   P.tensor_scale = tensor_scale;
   P.ws = ws;
   P.tokens = tokens;
-  P.x = static_cast<const uint16_t*>(x);
-  P.e_coef = e_coef_tc();
   cudaError_t e;
   if (ws) {
     e = cudaMemsetAsync(ws, 0, kNvWorkspaceHeader + (size_t)tokens * sizeof(float2), s);
@@ -702,8 +823,6 @@ cudaError_t launch_tc_rot(const void* x, int64_t tokens, const Geometry& g, cons
   tc::Params P{};
   P.out = out;
   P.tokens = tokens;
-  P.x = static_cast<const uint16_t*>(x);
-  P.e_coef = e_coef_tc();
   (void)g;
   return launch_tc<tc::kRot>(x, signs, P, s);
 }
