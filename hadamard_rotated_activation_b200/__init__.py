@@ -38,7 +38,7 @@ KQ_FMT_NVFP4 = 2
 C_SYMBOLS = (
     "kq_rht", "kq_rht_quant_int4", "kq_rht_quant_nvfp4", "kq_dequant",
     "kq_workspace_size", "kq_status_str", "kq_last_cuda_error", "kq_version",
-    "kq_rht_quant_nvfp4_dynamic_noalloc",
+    "kq_rht_quant_nvfp4_dynamic_noalloc", "kq_diag_tc_steps",
 )
 
 # Fixed device scratch of kq_rht_quant_nvfp4_dynamic_noalloc (see include/kq.h).
@@ -87,6 +87,8 @@ def lib() -> ctypes.CDLL:
     L.kq_last_cuda_error.restype = i32
     L.kq_version.argtypes = []
     L.kq_version.restype = i32
+    L.kq_diag_tc_steps.argtypes = [vp, vp, vp, vp, vp, vp]
+    L.kq_diag_tc_steps.restype = i32
     _lib = L
     return L
 
@@ -180,6 +182,14 @@ def kq_dequant(fmt: int, codes, scales, zeros, tensor_scale, tokens: int, dim: i
     _check(lib().kq_dequant(fmt, _ptr(codes), _ptr(scales), _ptr(zeros),
                             _ptr(tensor_scale), tokens, dim, group, _ptr(out),
                             _stream(stream)), "kq_dequant")
+
+
+def kq_diag_tc_steps(a, b, d1, d2, status, stream=None) -> None:
+    """Two tensor-core accumulation steps on caller data (diagnostic; see
+    include/kq.h): a bf16 [128, 32], b bf16 [32, 128], d1/d2 fp32 [128, 128],
+    status one int32 (0 = the waits completed)."""
+    _check(lib().kq_diag_tc_steps(_ptr(a), _ptr(b), _ptr(d1), _ptr(d2), _ptr(status),
+                                  _stream(stream)), "kq_diag_tc_steps")
 
 
 def kq_workspace_size(tokens: int, dim: int, block: int) -> int:

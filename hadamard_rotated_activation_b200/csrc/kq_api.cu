@@ -212,4 +212,14 @@ KQ_API int kq_last_cuda_error(void) { return g_last_cuda_error; }
 
 KQ_API int kq_version(void) { return (1 << 16) | 0; }
 
+KQ_API kq_status kq_diag_tc_steps(const uint16_t* a, const uint16_t* b, float* d1, float* d2,
+                                  unsigned int* status, kq_stream_t stream) {
+  if (!a || !b || !d1 || !d2 || !status) return KQ_ERR_INVALID_ARG;
+  if (!aligned(a, 2) || !aligned(b, 2) || !aligned(d1, 4) || !aligned(d2, 4) ||
+      !aligned(status, 4))
+    return KQ_ERR_MISALIGNED;
+  return finish(kq::launch_diag_tc_steps(a, b, d1, d2, status,
+                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -63,6 +63,8 @@ cudaError_t launch_tc_nvfp4(const void* x, int64_t tokens, const Geometry& g,
 cudaError_t launch_tc_rot(const void* x, int64_t tokens, const Geometry& g, const int8_t* signs,
                           float* out, cudaStream_t s);
 int tc_error_flag();
+cudaError_t launch_diag_tc_steps(const uint16_t* a, const uint16_t* b, float* d1, float* d2,
+                                 unsigned int* status, cudaStream_t s);
 
 cudaError_t launch_dequant(int fmt, const uint8_t* codes, const void* scales,
                            const void* zeros, const float* tensor_scale, int64_t tokens,

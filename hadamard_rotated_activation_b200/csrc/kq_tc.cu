@@ -736,6 +736,76 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
   }
 }
 
+// ------------------------------------------------------------ diagnostic
+// Two accumulation steps of the kernel's MMA on caller data, with the same
+// operand layouts, descriptors and instruction: D = A[:, 0:16] B[0:16, :]
+// (from zero), written to d1, then D += A[:, 16:32] B[16:32, :], written to
+// d2.  B's 128 columns are four 32-column blocks laid out like four staged
+// tokens.  One CTA of 128 threads.
+__global__ void __launch_bounds__(128, 1)
+k_diag_steps(const uint16_t* __restrict__ a, const uint16_t* __restrict__ b, float* d1,
+             float* d2, unsigned int* status) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sA = smem;                       // 32 KB
+  uint8_t* sB = smem + 32768;               // 32 KB: four 8 KB column blocks
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sB + kStageBytes);
+  uint32_t* slot = reinterpret_cast<uint32_t*>(bar + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < 128 * 128; i += blockDim.x) {
+    const int m = i >> 7, k = i & 127;
+    *reinterpret_cast<uint16_t*>(sA + a_off(m, k)) = k < 32 ? a[m * 32 + k] : 0;
+  }
+  for (int i = threadIdx.x; i < 128 * 128; i += blockDim.x) {
+    const int k = i >> 7, n = i & 127, blk = n >> 5, beta = n & 31;
+    *reinterpret_cast<uint16_t*>(sB + blk * kTokBytes + tok_chunk(k, beta >> 3) + (beta & 7) * 2) =
+        k < 32 ? b[k * 128 + n] : 0;
+  }
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 :: "r"(smem_u32(slot)), "n"(kAccCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *slot;
+  bool ok = true;
+  for (int step = 0; step < 2; ++step) {
+    if (threadIdx.x == 0) {
+      const uint64_t adesc = smem_desc(smem_u32(sA) + step * 32, 16, 1024, 2);
+      const uint64_t bdesc = smem_desc(smem_u32(sB) + step * 1024, kTokBytes, 512, 4);
+      mma_bf16(tmem, adesc, bdesc, (uint32_t)step);
+      mma_commit(bar);
+    }
+    ok = mbar_wait(bar, (uint32_t)step) && ok;
+    tc_fence_after();
+    float* d = step == 0 ? d1 : d2;
+    for (int cb = 0; cb < 4; ++cb) {
+      uint32_t r[32];
+      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + cb * 32, r);
+      tmem_wait_ld();
+      const int m = warp * 32 + lane;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) d[m * 128 + cb * 32 + j] = __uint_as_float(r[j]);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  }
+  if (threadIdx.x == 0) *status = ok ? 0u : 1u;
+  __syncthreads();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;"
+                 :: "r"(tmem), "n"(kAccCols));
+}
+
 }  // namespace tc
 
 // ------------------------------------------------------------- launchers
@@ -825,6 +895,15 @@ cudaError_t launch_tc_rot(const void* x, int64_t tokens, const Geometry& g, cons
   P.tokens = tokens;
   (void)g;
   return launch_tc<tc::kRot>(x, signs, P, s);
+}
+
+cudaError_t launch_diag_tc_steps(const uint16_t* a, const uint16_t* b, float* d1, float* d2,
+                                 unsigned int* status, cudaStream_t s) {
+  constexpr int kDiagSmem = 1024 + 32768 + (int)tc::kStageBytes + 64;
+  cudaFuncSetAttribute((const void*)tc::k_diag_steps, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       kDiagSmem);
+  tc::k_diag_steps<<<1, 128, kDiagSmem, s>>>(a, b, d1, d2, status);
+  return cudaGetLastError();
 }
 
 int tc_error_flag() {

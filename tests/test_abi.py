@@ -101,6 +101,10 @@ def test_argument_errors(L):
     assert L.kq_rht(None, 1, 0, 4096, 0, None, None, 0, None) == kq.KQ_OK
     assert d(2, None, None, None, None, 0, 4096, 0, None, None) == kq.KQ_OK
     assert L.kq_workspace_size(4, 4095, 0) == 0
+    t = L.kq_diag_tc_steps
+    assert t(None, P, P, P, P, None) == kq.KQ_ERR_INVALID_ARG
+    assert t(P + 1, P, P, P, P, None) == kq.KQ_ERR_MISALIGNED
+    assert t(P, P, P + 2, P, P, None) == kq.KQ_ERR_MISALIGNED
 
 
 def test_python_binding_rejects_host_tensors(L):
