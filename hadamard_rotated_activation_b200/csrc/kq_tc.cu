@@ -34,15 +34,17 @@
 // there, each losing less than 2^-25 P_k); the 5 u term bounds the five fp32
 // butterfly stages.  The sign-flip warps compute W, sum|x| and R for each
 // token while they touch the tile.  Block scales that E leaves undecided are
-// recomputed exactly (fp64)
-// from the staged input, which stays in shared memory until the epilogue
-// releases its stage.
+// recomputed exactly (fp64) from the input row in global memory.
 //
-// Warp roles (18 warps): 0 TMA producer, 1 MMA issuer + TMEM owner, 2-9 sign
+// Warp roles (19 warps): 0 TMA producer, 1 MMA issuer + TMEM owner, 2-9 sign
 // flip and error bound (two per token of a tile), 10-17 epilogue (two groups
-// of four warps; warp w reads TMEM lane quarter w % 4).  Every wait on an
-// mbarrier is bounded; on timeout the kernel records an error code and
-// returns.
+// of four warps; warp w reads TMEM lane quarter w % 4), 18 fix-up: blocks
+// whose scale the bound leaves undecided are stored provisionally by the
+// epilogue and queued (shared memory); the fix-up warp decides them exactly
+// and rewrites their scale and codes.  A shared-memory stage
+// is recycled as soon as the MMAs have read it (tcgen05.commit); the tile's
+// error bounds travel with its accumulator.  Every wait on an mbarrier is
+// bounded; on timeout the kernel records an error code and returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -67,17 +69,21 @@ constexpr int kAccCols = 32 * kTok;            // fp32 columns per accumulator
 constexpr int kTmemCols = kAcc * kAccCols;     // power of two >= 32
 constexpr int kSignWarps = 2 * kTok;           // two per token
 constexpr int kEpiWarps = 4 * kGroups;
-constexpr int kThreads = 32 * (2 + kSignWarps + kEpiWarps);
+constexpr int kFixWarp = 2 + kSignWarps + kEpiWarps;   // finishes undecided blocks
+constexpr int kThreads = 32 * (kFixWarp + 1);
+constexpr int kQ = 32;                         // fix-up queue entries
 constexpr long long kWaitCycles = 4000000000ll;   // about 2 s at 2 GHz
 static_assert(kAcc % kGroups == 0 && (kTmemCols & (kTmemCols - 1)) == 0 && kTmemCols <= 512,
               "accumulators: a multiple of the groups, a power-of-two column count <= 512");
 static_assert((3 * kStages + 2 * kAcc) * 8 + 4 <= 512, "barrier area");
+constexpr int kBoundFloats = (kStages + kAcc) * kTok * 2;   // sE + sEacc
 
 __device__ unsigned int g_tc_error = 0;        // nonzero: a wait timed out
 
 enum { kNvfp4 = 0, kNvStats = 1, kRot = 2 };
 
 struct Params {
+  const uint16_t* x;            // bf16 [T, n]: read by the exact fix-ups
   uint8_t* codes;               // [T, n/2]
   uint8_t* scales8;             // [T, n/16]
   float* tensor_scale;
@@ -273,14 +279,16 @@ __device__ __forceinline__ uint32_t tok_chunk(int a, int c) {
   return (uint32_t)(a * 64 + ((c ^ ((a >> 1) & 3)) << 4));
 }
 
-// Exact S_i of a staged token (sign-flipped, 64-byte swizzled), warp-
-// cooperative fp64.  Lane l reads the 16-byte chunks l, l+32, ...: chunk
-// (a, c) holds x'[a*32 + c*8 .. +7], and H[i][j] for those j is
-// (-1)^(popc(i_hi & a) + popc(i_mid & c) + popc(i_lo & e)) with i = i_hi*32 +
-// i_mid*8 + i_lo, so the Hadamard signs are two bit masks per word selected
-// per chunk.  Values enter fp64 exactly through bf16x2_to_f64_scaled, into
-// four independent accumulators.  Every lane gets the result.  Finite inputs.
-__device__ __noinline__ double warp_exact_S(const uint8_t* tok, int i) {
+// Exact S_i of token row `row` (bf16, natural order, in global memory),
+// warp-cooperative fp64.  Lane l reads the 16-byte chunks l, l+32, ...: chunk
+// (a, c) holds x[a*32 + c*8 .. +7] and its sign-flip masks are smask[a*4 + c];
+// H[i][j] for those j is (-1)^(popc(i_hi & a) + popc(i_mid & c) + popc(i_lo &
+// e)) with i = i_hi*32 + i_mid*8 + i_lo, so the Hadamard signs are two bit
+// masks per word selected per chunk.  Values enter fp64 exactly through
+// bf16x2_to_f64_scaled, into four independent accumulators.  Every lane gets
+// the result.  Finite inputs.
+__device__ __noinline__ double warp_exact_S(const uint4* __restrict__ row,
+                                            const uint4* __restrict__ smask, int i) {
   const int lane = threadIdx.x & 31;
   const int ihi = i >> 5, imid = (i >> 3) & 3, ilo = i & 7;
   uint32_t em[4];                   // sign bits of elements 2w, 2w+1 of a chunk
@@ -288,15 +296,15 @@ __device__ __noinline__ double warp_exact_S(const uint8_t* tok, int i) {
   for (int w = 0; w < 4; ++w)
     em[w] = ((uint32_t)(__popc(ilo & (2 * w)) & 1) << 15) |
             ((uint32_t)(__popc(ilo & (2 * w + 1)) & 1) << 31);
-  const uint4* base = reinterpret_cast<const uint4*>(tok);
   double acc[4] = {0.0, 0.0, 0.0, 0.0};
-#pragma unroll 4
+#pragma unroll 8
   for (int k = 0; k < 16; ++k) {
-    const int idx = lane + 32 * k;            // physical chunk: row a, slot pc
-    const int a = idx >> 2, c = (idx & 3) ^ ((a >> 1) & 3);
+    const int idx = lane + 32 * k;            // chunk (a, c)
+    const int a = idx >> 2, c = idx & 3;
     const uint32_t flip = ((__popc(ihi & a) ^ __popc(imid & c)) & 1) ? 0x80008000u : 0u;
-    const uint4 v = base[idx];
-    const uint32_t ww[4] = {v.x, v.y, v.z, v.w};
+    const uint4 v = __ldg(row + idx);
+    const uint4 m = smask[idx];
+    const uint32_t ww[4] = {v.x ^ m.x, v.y ^ m.y, v.z ^ m.z, v.w ^ m.w};
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
       double lo, hi;
@@ -308,18 +316,75 @@ __device__ __noinline__ double warp_exact_S(const uint8_t* tok, int i) {
   return warp_sum_d((acc[0] + acc[1]) + (acc[2] + acc[3])) * kF64Unscale;
 }
 
-// The same for tokens that hold an infinity or NaN (IEEE conversions, slow).
-__device__ __noinline__ double warp_exact_S_ieee(const uint8_t* tok, int i) {
+// The same for rows that hold an infinity or NaN (IEEE conversions, slow).
+__device__ __noinline__ double warp_exact_S_ieee(const uint16_t* __restrict__ row,
+                                                 const int8_t* __restrict__ signs, int i) {
   const int lane = threadIdx.x & 31;
   double acc = 0.0;
-  for (int a = 0; a < 128; ++a) {
-    const int beta = lane;
-    const uint8_t* p = tok + tok_chunk(a, beta >> 3) + (beta & 7) * 2;
-    const double xv =
-        (double)__uint_as_float((uint32_t)(*reinterpret_cast<const uint16_t*>(p)) << 16);
-    acc += (__popc(i & (a * 32 + beta)) & 1) ? -xv : xv;
+  for (int j = lane; j < 4096; j += 32) {
+    double xv = (double)__uint_as_float((uint32_t)row[j] << 16);
+    if (signs && signs[j] < 0) xv = -xv;
+    acc += (__popc(i & j) & 1) ? -xv : xv;
   }
   return warp_sum_d(acc);
+}
+
+// One NVFP4 block whose scale the error bound leaves undecided: the epilogue
+// stores a provisional scale and codes and hands the block to the fix-up
+// warp, which decides the scale exactly and rewrites both.
+struct FixEntry {
+  float v[16];        // the block's S_hat values
+  float bm;           // max |S_hat| of the block
+  float E;            // |S_hat - S| <= E (per output of the token)
+  long long token;
+  int block;          // 16-element block index within the row
+  int pad_;
+};
+struct FixQueue {
+  FixEntry e[kQ];
+  unsigned int seq[kQ];   // slot k holds entry h when seq[k] == h + 1
+  unsigned int tail;      // entries reserved by the epilogue
+  unsigned int head;      // entries finished by the fix-up warp
+  unsigned int done;      // epilogue warps that will enqueue nothing more
+};
+
+__device__ __forceinline__ unsigned int ld_acquire(const unsigned int* p) {
+  unsigned int v;
+  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release(unsigned int* p, unsigned int v) {
+  asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" :: "r"(smem_u32(p)), "r"(v) : "memory");
+}
+
+// E2M1 codes of one 16-element block (v: 8 pairs) for the E4M3 scale `code`:
+// two words, element k in bits 4k..4k+3.  A zero scale (or tensor scale)
+// leaves only the signs.
+__device__ __forceinline__ void nvfp4_block_words(const float2* v, uint32_t code, float inv_bt,
+                                                  float ts, uint32_t& w0, uint32_t& w1) {
+  if (code != 0 && ts > 0.0f) {
+    const float cs = inv_bt * e4m3_recip(code);
+    const float2 c2 = make_float2(cs, cs), zero2 = make_float2(0.0f, 0.0f);
+    float qv[16];
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      const float2 a = fma2(v[p], c2, zero2);   // + 0 turns -0 into +0
+      qv[2 * p] = a.x;
+      qv[2 * p + 1] = a.y;
+    }
+    w0 = e2m1x8_hw(qv);
+    w1 = e2m1x8_hw(qv + 8);
+  } else {
+    w0 = 0;
+    w1 = 0;
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      w0 |= (v[p].x < 0.0f ? 8u : 0u) << (8 * p);
+      w0 |= (v[p].y < 0.0f ? 8u : 0u) << (8 * p + 4);
+      w1 |= (v[4 + p].x < 0.0f ? 8u : 0u) << (8 * p);
+      w1 |= (v[4 + p].y < 0.0f ? 8u : 0u) << (8 * p + 4);
+    }
+  }
 }
 
 // ---------------------------------------------------------------- kernel
@@ -335,13 +400,15 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
   uint8_t* sB = smem + 32768;                           // kStages x 32 KB
   uint4* smask = reinterpret_cast<uint4*>(sB + kStages * kStageBytes);   // 512 chunks
   float* sE = reinterpret_cast<float*>(smask + 512);   // error bound halves per (stage, token)
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sE + kStages * kTok * 2);
+  float* sEacc = sE + kStages * kTok * 2;              // the same, handed to the epilogue per accumulator
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sE + kBoundFloats);
   uint64_t* full = bars;                                // TMA landed
   uint64_t* ready = bars + kStages;                     // signs applied, bounds written
-  uint64_t* empty = bars + 2 * kStages;                 // epilogue done with the stage
-  uint64_t* tfull = bars + 3 * kStages;                 // accumulator written (kAcc)
+  uint64_t* empty = bars + 2 * kStages;                 // MMAs done reading the stage
+  uint64_t* tfull = bars + 3 * kStages;                 // accumulator written + bounds (kAcc)
   uint64_t* tempty = tfull + kAcc;                      // accumulator read (kAcc)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + kAcc);
+  FixQueue* fq = reinterpret_cast<FixQueue*>(bars + 64);   // after the 512-byte barrier area
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -367,14 +434,18 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&ready[s], 32 * kSignWarps);
-      mbar_init(&empty[s], 128);
+      mbar_init(&empty[s], 1);
     }
     for (int d = 0; d < kAcc; ++d) {
-      mbar_init(&tfull[d], 1);
+      mbar_init(&tfull[d], 2);
       mbar_init(&tempty[d], 128);
     }
+    fq->tail = 0;
+    fq->head = 0;
+    fq->done = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  for (int i = threadIdx.x; i < kQ; i += blockDim.x) fq->seq[i] = 0;
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                  :: "r"(smem_u32(tmem_slot)), "n"(kTmemCols));
@@ -419,6 +490,10 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
         if (!mbar_wait(&ready[s], (uint32_t)(k / kStages) & 1)) break;
         if (k >= kAcc && !mbar_wait(&tempty[d], (uint32_t)(k / kAcc - 1) & 1)) break;
         tc_fence_after();
+        // the tile's error bounds move to the accumulator's slot: the stage
+        // is recycled as soon as the MMAs below have read it
+#pragma unroll
+        for (int e = 0; e < kTok * 2; ++e) sEacc[d * kTok * 2 + e] = sE[s * kTok * 2 + e];
         const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB + s * kStageBytes);
         const uint32_t tmem_d = tmem_base + (uint32_t)(d * kAccCols);
 #pragma unroll
@@ -430,7 +505,9 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
           const uint64_t bdesc = smem_desc(b0 + ks * 1024, kTokBytes, 512, 4);
           mma_bf16(tmem_d, adesc, bdesc, ks > 0 ? 1u : 0u);
         }
+        mma_commit(&empty[s]);
         mma_commit(&tfull[d]);
+        mbar_arrive(&tfull[d]);          // publishes sEacc[d] (release)
         issued = k + 1;
       }
       // the accumulators must not be released with MMAs still running
@@ -546,7 +623,7 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
       __syncwarp();
       mbar_arrive(&ready[s]);
     }
-  } else {
+  } else if (warp < kFixWarp) {
     // ================= epilogue: group g of warps 10+4g .. 13+4g
     const int g = (warp - 2 - kSignWarps) >> 2;
     const int q = warp & 3;                   // TMEM lane quarter
@@ -565,19 +642,18 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
       inv_bt = (ts > 0.0f) ? (float)(1.0 / (kSqrtN * (double)ts)) : 0.0f;
     }
     for (int64_t k = g; k < my_tiles; k += kGroups) {
-      const int s = (int)(k % kStages);
       const int d = (int)(k % kAcc);
       const int64_t tile = blockIdx.x + k * gridDim.x;
       // A timed-out wait does not leave the loop: the failure is recorded
       // (g_tc_error) and the tile's outputs are not written.
-      bool ok = mbar_wait(&tfull[d], (uint32_t)(k / kAcc) & 1);
-      // the staged input (read by the fix-ups) and the bounds are final once
-      // the sign warps have arrived
-      ok = mbar_wait(&ready[s], (uint32_t)(k / kStages) & 1) && ok;
+      const bool ok = mbar_wait(&tfull[d], (uint32_t)(k / kAcc) & 1);
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(d * kAccCols);
 #pragma unroll 1
       for (int t = 0; t < kTok; ++t) {
+        // |S_hat - S| <= E for every output of the token; read before the
+        // accumulator (and with it the bound slot) is handed back below
+        const float E = __fadd_ru(sEacc[(d * kTok + t) * 2], sEacc[(d * kTok + t) * 2 + 1]);
         float2 v[16];
         {
           uint32_t r[32];
@@ -613,8 +689,6 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
           for (int p = 8 * j; p < 8 * j + 8; ++p) mm = fmax3(mm, fabsf(v[p].x), fabsf(v[p].y));
           bm[j] = mm;
         }
-        // |S_hat - S| <= E for every output of the token
-        const float E = __fadd_ru(sE[(s * kTok + t) * 2], sE[(s * kTok + t) * 2 + 1]);
 
         if (kMode == kRot) {
           if (valid) {
@@ -640,7 +714,8 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
           continue;
         }
 
-        // ---- NVFP4 block scales, exact where undecided
+        // ---- NVFP4 block scales; a block whose scale the bound leaves
+        // undecided is stored provisionally and finished by the fix-up warp
         uint32_t sc = 0, undecided = 0;
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
@@ -651,79 +726,99 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
           if ((cc & 0xffu) != (cc >> 8)) undecided |= 1u << j;
         }
         if (ts <= 0.0f || !valid) undecided = 0;
-        const bool finite = isfinite(E);   // sum|x| finite: every input finite
-        unsigned todo = __ballot_sync(0xffffffffu, undecided != 0);
-        const uint8_t* tok = sB + s * kStageBytes + t * kTokBytes;
-        while (todo) {
-          const int src = __ffs(todo) - 1;
-          todo &= todo - 1;
-          const uint32_t und = __shfl_sync(0xffffffffu, undecided, src);
-          const int src_o = q * 32 + src;
-          for (int j = 0; j < 2; ++j) {
-            if (!((und >> j) & 1u)) continue;
-            uint32_t cand = 0;
-            if (lane == src) {
-              const float thr = (j ? bm[1] : bm[0]) - 2.0f * E;
-#pragma unroll
-              for (int p = 0; p < 8; ++p) {
-                const float2 a = j ? v[8 + p] : v[p];
-                if (fabsf(a.x) >= thr) cand |= 1u << (2 * p);
-                if (fabsf(a.y) >= thr) cand |= 1u << (2 * p + 1);
-              }
-            }
-            cand = __shfl_sync(0xffffffffu, cand, src);
-            double best = 0.0;
-            while (cand) {
-              const int e = __ffs(cand) - 1;
-              cand &= cand - 1;
-              const int ii = src_o * 32 + 16 * j + e;
-              best = fmax(best, fabs(finite ? warp_exact_S(tok, ii) : warp_exact_S_ieee(tok, ii)));
-            }
-            const float rr = __double2float_rn((best / kSqrtN) / (6.0 * (double)ts));
-            const uint32_t code = e4m3_pair(rr, rr) & 0xffu;
-            if (lane == src) sc = (sc & ~(0xffu << (8 * j))) | (code << (8 * j));
-          }
-        }
 
         // ---- codes: 16 bytes per lane, contiguous across the warp
-        const float2 zero2 = make_float2(0.0f, 0.0f);
         uint32_t words[4];
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const uint32_t code = (sc >> (8 * j)) & 0xffu;
-          if (code != 0 && ts > 0.0f) {
-            const float cs = inv_bt * e4m3_recip(code);
-            const float2 c2 = make_float2(cs, cs);
-            float qv[16];
-#pragma unroll
-            for (int p = 0; p < 8; ++p) {
-              const float2 a = fma2(v[8 * j + p], c2, zero2);   // + 0 turns -0 into +0
-              qv[2 * p] = a.x;
-              qv[2 * p + 1] = a.y;
-            }
-            words[2 * j] = e2m1x8_hw(qv);
-            words[2 * j + 1] = e2m1x8_hw(qv + 8);
-          } else {
-            uint32_t w0 = 0, w1 = 0;
-#pragma unroll
-            for (int p = 0; p < 4; ++p) {
-              w0 |= (v[8 * j + p].x < 0.0f ? 8u : 0u) << (8 * p);
-              w0 |= (v[8 * j + p].y < 0.0f ? 8u : 0u) << (8 * p + 4);
-              w1 |= (v[8 * j + 4 + p].x < 0.0f ? 8u : 0u) << (8 * p);
-              w1 |= (v[8 * j + 4 + p].y < 0.0f ? 8u : 0u) << (8 * p + 4);
-            }
-            words[2 * j] = w0;
-            words[2 * j + 1] = w1;
-          }
-        }
+        nvfp4_block_words(v, sc & 0xffu, inv_bt, ts, words[0], words[1]);
+        nvfp4_block_words(v + 8, sc >> 8, inv_bt, ts, words[2], words[3]);
         if (valid) {
           *reinterpret_cast<uint4*>(P.codes + token * (N / 2) + o * 16) =
               make_uint4(words[0], words[1], words[2], words[3]);
           *reinterpret_cast<uint16_t*>(P.scales8 + token * (N / 16) + o * 2) = (uint16_t)sc;
         }
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          if (!((undecided >> j) & 1u)) continue;
+          const unsigned int slot = atomicAdd(&fq->tail, 1u);
+          const long long t0 = clock64();
+          bool room = true;
+          while (slot - ld_acquire(&fq->head) >= (unsigned int)kQ) {
+            if (clock64() - t0 > kWaitCycles) { room = false; break; }
+            __nanosleep(64);
+          }
+          if (!room) {                 // the block keeps its provisional scale
+            atomicOr(&g_tc_error, 2u);
+            continue;
+          }
+          FixEntry& fe = fq->e[slot % kQ];
+#pragma unroll
+          for (int p = 0; p < 8; ++p) {
+            fe.v[2 * p] = v[8 * j + p].x;
+            fe.v[2 * p + 1] = v[8 * j + p].y;
+          }
+          fe.bm = bm[j];
+          fe.E = E;
+          fe.token = token;
+          fe.block = o * 2 + j;
+          __threadfence_block();       // the provisional stores above come first
+          st_release(&fq->seq[slot % kQ], slot + 1);
+        }
       }
-      __syncwarp();
-      mbar_arrive(&empty[s]);        // staged input no longer needed
+    }
+    __syncwarp();
+    __threadfence_block();
+    if (lane == 0) atomicAdd(&fq->done, 1u);
+  } else if (warp == kFixWarp) {
+    // ================= fix-up warp: exact scales of the queued blocks
+    if (kMode == kNvfp4) {
+      float ts = 0.0f, inv_bt = 0.0f;
+      if (P.ws) {
+        const double gm = __longlong_as_double((long long)P.ws->gmax_bits);
+        ts = __double2float_rn((gm / kSqrtN) / 2688.0);
+      } else {
+        ts = *P.tensor_scale;
+      }
+      inv_bt = (ts > 0.0f) ? (float)(1.0 / (kSqrtN * (double)ts)) : 0.0f;
+      unsigned int h = 0;
+      long long idle0 = clock64();
+      for (;;) {
+        if (ld_acquire(&fq->seq[h % kQ]) == h + 1) {
+          const FixEntry& fe = fq->e[h % kQ];
+          const float thr = fe.bm - 2.0f * fe.E;
+          const bool finite = isfinite(fe.E);   // sum|x| finite: every input finite
+          uint32_t cand = __ballot_sync(0xffffffffu, lane < 16 && fabsf(fe.v[lane & 15]) >= thr);
+          const long long token = fe.token;
+          const int blk = fe.block;
+          double best = 0.0;
+          while (cand) {
+            const int e = __ffs(cand) - 1;
+            cand &= cand - 1;
+            const int ii = blk * 16 + e;
+            best = fmax(best, fabs(finite
+                ? warp_exact_S(reinterpret_cast<const uint4*>(P.x + token * N), smask, ii)
+                : warp_exact_S_ieee(P.x + token * N, signs, ii)));
+          }
+          const float rr = __double2float_rn((best / kSqrtN) / (6.0 * (double)ts));
+          const uint32_t code = e4m3_pair(rr, rr) & 0xffu;
+          if (lane == 0) {
+            uint32_t w0, w1;
+            nvfp4_block_words(reinterpret_cast<const float2*>(fe.v), code, inv_bt, ts, w0, w1);
+            *reinterpret_cast<uint2*>(P.codes + token * (N / 2) + blk * 8) = make_uint2(w0, w1);
+            P.scales8[token * (N / 16) + blk] = (uint8_t)code;
+          }
+          __syncwarp();
+          if (lane == 0) st_release(&fq->head, h + 1);
+          ++h;
+          idle0 = clock64();
+          continue;
+        }
+        if (ld_acquire(&fq->done) == (unsigned int)kEpiWarps && ld_acquire(&fq->tail) == h) break;
+        if (clock64() - idle0 > kWaitCycles) {
+          atomicOr(&g_tc_error, 4u);
+          break;
+        }
+        __nanosleep(128);
+      }
     }
   }
 
@@ -841,7 +936,7 @@ bool make_tmap(CUtensorMap* map, const void* x, int64_t rows) {
 }
 
 constexpr size_t kSmemBytes = 1024 + 32768 + tc::kStages * tc::kStageBytes + 512 * 16 +
-                              tc::kStages * tc::kTok * 8 + 512;
+                              tc::kBoundFloats * 4 + 512 + sizeof(tc::FixQueue);
 
 template <int kMode>
 cudaError_t launch_tc(const void* x, const int8_t* signs, tc::Params& P, cudaStream_t s) {
@@ -871,6 +966,7 @@ cudaError_t launch_tc_nvfp4(const void* x, int64_t tokens, const Geometry& g,
                             const int8_t* signs, uint8_t* codes, uint8_t* bscales,
                             float* tensor_scale, NvWorkspace* ws, cudaStream_t s) {
   tc::Params P{};
+  P.x = static_cast<const uint16_t*>(x);
   P.codes = codes;
   P.scales8 = bscales;
   P.tensor_scale = tensor_scale;
@@ -891,6 +987,7 @@ cudaError_t launch_tc_nvfp4(const void* x, int64_t tokens, const Geometry& g,
 cudaError_t launch_tc_rot(const void* x, int64_t tokens, const Geometry& g, const int8_t* signs,
                           float* out, cudaStream_t s) {
   tc::Params P{};
+  P.x = static_cast<const uint16_t*>(x);
   P.out = out;
   P.tokens = tokens;
   (void)g;
