@@ -33,7 +33,8 @@
 // (step, column) pairs that hold an input below 2^-18 P_k: at most 16 inputs
 // there, each losing less than 2^-25 P_k); the 5 u term bounds the five fp32
 // butterfly stages.  The sign-flip warps compute W, sum|x| and R for each
-// token while they touch the tile.  Block scales that E leaves undecided are
+// token while they touch the tile (bf16 partial sums of |x|, made upper
+// bounds by a 2^-4 relative margin).  Block scales that E leaves undecided are
 // recomputed exactly (fp64) from the input row in global memory.
 //
 // Warp roles (19 warps): 0 TMA producer, 1 MMA issuer + TMEM owner, 2-9 sign
@@ -214,6 +215,11 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
 __device__ __forceinline__ uint32_t min_bf16x2(uint32_t a, uint32_t b) {
   uint32_t d;
   asm("min.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t add_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
   return d;
 }
 __device__ __forceinline__ uint32_t redux_max(uint32_t v) {
@@ -534,11 +540,10 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
       const int s = (int)(k % kStages);
       if (!mbar_wait(&full[s], (uint32_t)(k / kStages) & 1)) break;
       uint8_t* tok = sB + s * kStageBytes + t * kTokBytes;
-      float2 acc[4];
-      uint32_t mn[4];
+      uint32_t sacc[4], mn[4];                    // bf16x2 sums and minima of |x'|
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
-        acc[h] = make_float2(0.0f, 0.0f);
+        sacc[h] = 0u;
         mn[h] = 0x7f807f80u;                        // +inf, +inf
       }
 #pragma unroll
@@ -564,11 +569,18 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
           for (int h = 0; h < 4; ++h) {
             const uint32_t ab = ww[h] & 0x7fff7fffu;   // |x'| of columns 2h, 2h+1
             mn[h] = min_bf16x2(mn[h], ab);
-            acc[h] = add2(acc[h], make_float2(__uint_as_float(ab << 16),
-                                              __uint_as_float(ab & 0xffff0000u)));
+            sacc[h] = add_bf16x2(sacc[h], ab);
           }
         }
       }
+      // Each bf16 sum of 8 non-negative terms is at least (1 - 2^-8)^7 of the
+      // exact sum (round to nearest), so x (1 + 2^-4) bounds it from above,
+      // with room for the fp32 additions below.
+      float2 acc[4];
+#pragma unroll
+      for (int h = 0; h < 4; ++h)
+        acc[h] = make_float2(__uint_as_float(sacc[h] << 16) * (1.0f + 0x1p-4f),
+                             __uint_as_float(sacc[h] & 0xffff0000u) * (1.0f + 0x1p-4f));
       float own = 0.0f;                       // this lane's sum |x'|
 #pragma unroll
       for (int h = 0; h < 4; ++h) own += acc[h].x + acc[h].y;
