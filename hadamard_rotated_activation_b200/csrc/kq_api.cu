@@ -88,6 +88,9 @@ KQ_API kq_status kq_rht(const void* x, int dtype, int64_t tokens, int dim, int b
   if (!(flags & KQ_INVERSE) && kq::tc_row_supported(g, dtype, x, tokens))
     return finish(kq::launch_tc_rot(x, tokens, g, signs, out,
                                     reinterpret_cast<cudaStream_t>(stream)));
+  if (!(flags & KQ_INVERSE) && kq::tcp_supported(g, dtype, x, tokens) && aligned(signs, 8))
+    return finish(kq::launch_tcp_rot(x, tokens, g, signs, out,
+                                     reinterpret_cast<cudaStream_t>(stream)));
   return finish(kq::launch_rht(x, dtype, tokens, g, signs, out, (flags & KQ_INVERSE) ? 1 : 0,
                                reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -117,6 +120,9 @@ KQ_API kq_status kq_rht_quant_int4(const void* x, int dtype, int64_t tokens, int
     return finish(kq::launch_blk128_asym(x, tokens, g, signs, codes,
                                          static_cast<uint16_t*>(scales),
                                          static_cast<uint16_t*>(zeros), s));
+  if (asym == 0 && kq::tcp_supported(g, dtype, x, tokens) && aligned(signs, 8))
+    return finish(kq::launch_tcp_int4(x, tokens, g, signs, codes, static_cast<float*>(scales),
+                                      s));
   if (asym == 0 && kq::rowwarp_supported(g, dtype))
     return finish(kq::launch_rowwarp_int4(x, dtype, tokens, g, signs, codes,
                                           static_cast<float*>(scales), s));

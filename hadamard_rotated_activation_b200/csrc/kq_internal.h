@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "kq_device.cuh"
@@ -19,6 +20,12 @@ struct NvWorkspace {
   float2 rows[1];
 };
 constexpr size_t kNvWorkspaceHeader = 16;
+
+// 2-D bf16 tensor map over a row-major [rows, cols] array (cols * 2 bytes a
+// row, a multiple of 16), boxes of box_cols x box_rows.  False when the driver
+// refuses it.
+bool encode_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
+                         uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swizzle);
 
 // Records a CUDA error for kq_last_cuda_error() on the calling thread.
 void set_last_cuda_error(int err);
@@ -63,6 +70,13 @@ cudaError_t launch_tc_nvfp4(const void* x, int64_t tokens, const Geometry& g,
 cudaError_t launch_tc_rot(const void* x, int64_t tokens, const Geometry& g, const int8_t* signs,
                           float* out, cudaStream_t s);
 int tc_error_flag();
+
+// Tensor-core kernels for 12288-wide rows (H_12 kron H_1024) of bf16 input (kq_tcp.cu).
+bool tcp_supported(const Geometry& g, int dtype, const void* x, int64_t tokens);
+cudaError_t launch_tcp_int4(const void* x, int64_t tokens, const Geometry& g,
+                            const int8_t* signs, uint8_t* codes, float* scales, cudaStream_t s);
+cudaError_t launch_tcp_rot(const void* x, int64_t tokens, const Geometry& g,
+                           const int8_t* signs, float* out, cudaStream_t s);
 cudaError_t launch_diag_tc_steps(const uint16_t* a, const uint16_t* b, float* d1, float* d2,
                                  unsigned int* status, cudaStream_t s);
 

@@ -56,6 +56,7 @@
 
 #include "kq_device.cuh"
 #include "kq_internal.h"
+#include "kq_sm100.cuh"
 
 namespace kq {
 namespace tc {
@@ -73,7 +74,6 @@ constexpr int kEpiWarps = 4 * kGroups;
 constexpr int kFixWarp = 2 + kSignWarps + kEpiWarps;   // finishes undecided blocks
 constexpr int kThreads = 32 * (kFixWarp + 1);
 constexpr int kQ = 32;                         // fix-up queue entries
-constexpr long long kWaitCycles = 4000000000ll;   // about 2 s at 2 GHz
 static_assert(kAcc % kGroups == 0 && (kTmemCols & (kTmemCols - 1)) == 0 && kTmemCols <= 512,
               "accumulators: a multiple of the groups, a power-of-two column count <= 512");
 static_assert((3 * kStages + 2 * kAcc) * 8 + 4 <= 512, "barrier area");
@@ -95,190 +95,20 @@ struct Params {
 };
 
 // --------------------------------------------------------------- helpers
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return (uint32_t)__cvta_generic_to_shared(p);
-}
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(smem_u32(bar)), "r"(count));
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" :: "r"(smem_u32(bar))
-               : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;"
-               :: "r"(smem_u32(bar)), "r"(bytes) : "memory");
-}
-// Bounded wait for the phase with the given parity; false on timeout (about
-// two seconds).  try_wait suspends the thread for up to the hint (ns) instead
-// of spinning.
+using namespace sm100;
+
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  const uint32_t a = smem_u32(bar);
-  const long long start = clock64();
-  for (;;) {
-    uint32_t ok;
-    asm volatile("{\n\t.reg .pred p;\n\t"
-                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-                 "selp.u32 %0, 1, 0, p;\n\t}"
-                 : "=r"(ok) : "r"(a), "r"(parity), "r"(20000u) : "memory");
-    if (ok) return true;
-    if (clock64() - start > kWaitCycles) break;
-  }
-  atomicOr(&g_tc_error, 1u);
-  return false;
-}
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
-                                            uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];"
-      :: "r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y),
-         "r"(smem_u32(bar)) : "memory");
-}
-__device__ __forceinline__ void fence_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  return sm100::mbar_wait(bar, parity, &g_tc_error);
 }
 
-// Shared-memory matrix descriptor (tcgen05): start >> 4, leading and stride
-// byte offsets >> 4, version 1, swizzle layout (2 = 128-byte, 4 = 64-byte).
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo,
-                                              uint32_t layout) {
-  uint64_t d = 0;
-  d |= (uint64_t)((addr >> 4) & 0x3FFFu);
-  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
-  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
-  d |= (uint64_t)1 << 46;           // version
-  d |= (uint64_t)layout << 61;
-  return d;
-}
-
-// kind::f16 instruction descriptor: D fp32, A and B bf16, A K-major,
-// B MN-major, N = 128 (four tokens x 32), M = 128.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) | (1u << 16) |
-                            ((uint32_t)(kAccCols >> 3) << 17) | ((128u >> 4) << 24);
+// D fp32, A = H_128 (K-major), B = staged tokens (MN-major), M = 128, N = 128.
+constexpr uint32_t kIdesc = idesc_bf16(128, kAccCols, 1);
 
 __device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
                                          uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-      :: "r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate));
-}
-__device__ __forceinline__ void mma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
-               :: "r"(smem_u32(bar)) : "memory");
+  sm100::mma_bf16(tmem_d, adesc, bdesc, kIdesc, accumulate);
 }
 
-// 32 consecutive TMEM columns of this thread's lane.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-        "=r"(r[31])
-      : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_wait_ld() {
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ void bfly2(float2& a, float2& b) {
-  uint64_t ua = *reinterpret_cast<uint64_t*>(&a), ub = *reinterpret_cast<uint64_t*>(&b), s, d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(s) : "l"(ua), "l"(ub));
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(ua), "l"(ub));
-  a = *reinterpret_cast<float2*>(&s);
-  b = *reinterpret_cast<float2*>(&d);
-}
-__device__ __forceinline__ float2 add2(float2 a, float2 b) {
-  uint64_t ua = *reinterpret_cast<uint64_t*>(&a), ub = *reinterpret_cast<uint64_t*>(&b), r;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(ua), "l"(ub));
-  return *reinterpret_cast<float2*>(&r);
-}
-__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
-  uint64_t ua = *reinterpret_cast<uint64_t*>(&a), ub = *reinterpret_cast<uint64_t*>(&b),
-           uc = *reinterpret_cast<uint64_t*>(&c), r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(ua), "l"(ub), "l"(uc));
-  return *reinterpret_cast<float2*>(&r);
-}
-__device__ __forceinline__ uint32_t min_bf16x2(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("min.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-__device__ __forceinline__ uint32_t add_bf16x2(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-__device__ __forceinline__ uint32_t redux_max(uint32_t v) {
-  uint32_t r;
-  asm volatile("redux.sync.max.u32 %0, %1, 0xffffffff;" : "=r"(r) : "r"(v));
-  return r;
-}
-__device__ __forceinline__ uint32_t redux_add(uint32_t v) {
-  uint32_t r;
-  asm volatile("redux.sync.add.u32 %0, %1, 0xffffffff;" : "=r"(r) : "r"(v));
-  return r;
-}
-__device__ __forceinline__ float pow2f(int j) {   // 2^j, -126 <= j <= 127
-  return __uint_as_float((uint32_t)(127 + j) << 23);
-}
-// Upper bound of the warp sum of v >= 0 (every lane gets it), with integer
-// reductions: each lane's value is rounded up onto the grid 2^-k, where k
-// makes the warp maximum (bit pattern mbits) less than 2^26 units, so the 32
-// terms add exactly in 32 bits.  A non-finite maximum passes through.
-__device__ __forceinline__ float warp_sum_up(float v, uint32_t mbits) {
-  if (mbits >= 0x7f800000u) return __uint_as_float(mbits);
-  if (mbits == 0) return 0.0f;
-  const int e = max((int)(mbits >> 23), 1) - 127;
-  const int k = 25 - e, k1 = k / 2, k2 = k - k1;
-  const uint32_t q = __float2uint_ru(__fmul_ru(__fmul_ru(v, pow2f(k1)), pow2f(k2)));
-  const uint32_t sum = redux_add(q);
-  return __fmul_ru(__fmul_ru(__uint2float_ru(sum), pow2f(-k1)), pow2f(-k2));
-}
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-  float d;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-  return d;
-}
-__device__ __forceinline__ uint32_t e4m3_pair(float r_lo, float r_hi) {
-  uint32_t out;
-  asm("{.reg .b16 t; cvt.rn.satfinite.e4m3x2.f32 t, %1, %2; cvt.u32.u16 %0, t;}"
-      : "=r"(out) : "f"(r_hi), "f"(r_lo));
-  return out;
-}
-// 1 / value of a non-zero E4M3 code: a rounded reciprocal of the significand
-// (table folded at compile time) scaled by an exact power of two.
-__device__ __forceinline__ float e4m3_recip(uint32_t c) {
-  const uint32_t e = (c >> 3) & 15u, m = c & 7u;
-  if (e == 0) return 512.0f / (float)m;                 // subnormal: m * 2^-9
-  constexpr float kR0 = 1.0f / 1.0f, kR1 = 1.0f / 1.125f, kR2 = 1.0f / 1.25f,
-                  kR3 = 1.0f / 1.375f, kR4 = 1.0f / 1.5f, kR5 = 1.0f / 1.625f,
-                  kR6 = 1.0f / 1.75f, kR7 = 1.0f / 1.875f;
-  const float r = m < 4 ? (m < 2 ? (m == 0 ? kR0 : kR1) : (m == 2 ? kR2 : kR3))
-                        : (m < 6 ? (m == 4 ? kR4 : kR5) : (m == 6 ? kR6 : kR7));
-  return __uint_as_float(__float_as_uint(r) + ((7u - e) << 23));   // r * 2^(7-e)
-}
-
-// Byte offset of element (row m, column k) of the 128 x 128 A operand: two
-// 16 KB halves of 128 rows x 64 columns (bf16), 128-byte swizzle (16-byte
-// chunk c of row m at chunk position c ^ (m & 7)).
-__device__ __forceinline__ uint32_t a_off(int m, int k) {
-  const int h = k >> 6, c = (k >> 3) & 7, e = k & 7;
-  return (uint32_t)(h * 16384 + m * 128 + ((c ^ (m & 7)) << 4) + e * 2);
-}
 // Byte offset of 16-byte chunk c (0..3) of row a of a staged token (128 rows
 // of 64 bytes, 64-byte swizzle: chunk position c ^ ((a >> 1) & 3)).
 __device__ __forceinline__ uint32_t tok_chunk(int a, int c) {
@@ -353,15 +183,6 @@ struct FixQueue {
   unsigned int head;      // entries finished by the fix-up warp
   unsigned int done;      // epilogue warps that will enqueue nothing more
 };
-
-__device__ __forceinline__ unsigned int ld_acquire(const unsigned int* p) {
-  unsigned int v;
-  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_release(unsigned int* p, unsigned int v) {
-  asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" :: "r"(smem_u32(p)), "r"(v) : "memory");
-}
 
 // E2M1 codes of one 16-element block (v: 8 pairs) for the E4M3 scale `code`:
 // two words, element k in bits 4k..4k+3.  A zero scale (or tensor scale)
@@ -935,16 +756,7 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 // [rows, 32] bf16 view of the input (rows of 64 bytes), 32 x 128 boxes (one
 // token), 64-byte swizzle.
 bool make_tmap(CUtensorMap* map, const void* x, int64_t rows) {
-  auto enc = get_encode();
-  if (!enc) return false;
-  cuuint64_t gdim[2] = {32, (cuuint64_t)rows};
-  cuuint64_t gstride[1] = {64};
-  cuuint32_t box[2] = {32, 128};
-  cuuint32_t estride[2] = {1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), gdim, gstride,
-                   box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  return encode_tmap_bf16_2d(map, x, 32, (uint64_t)rows, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
 constexpr size_t kSmemBytes = 1024 + 32768 + tc::kStages * tc::kStageBytes + 512 * 16 +
@@ -967,6 +779,20 @@ cudaError_t launch_tc(const void* x, const int8_t* signs, tc::Params& P, cudaStr
 }
 
 }  // namespace
+
+bool encode_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
+                         uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swizzle) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t gstride[1] = {(cuuint64_t)cols * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estride[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim,
+                   gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
 
 bool tc_row_supported(const Geometry& g, int dtype, const void* x, int64_t tokens) {
   // TMA: 16-byte aligned base, int32 row coordinates

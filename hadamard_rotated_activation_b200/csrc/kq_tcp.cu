@@ -1,0 +1,525 @@
+// Tensor-core (tcgen05) kernel for 12288-wide rows (the intermediate size of
+// "Bug: Qwen3-8B integration issue", Model Details: 12288 = 12 x 1024 is
+// Hadamard-compatible), rotated by H_12 (Paley) kron H_1024 (Sylvester) and
+// quantized to per-token symmetric INT4 (QuaRot reviews, review 2 Summary:
+// RTN INT4 of the rotated activations), or written out rotated (fp32).
+//
+// A row of n = 12288 values is viewed as 96 rows of 128 (index j = a*128 +
+// beta, a = a12*8 + a8).  Since H_1024 = H_8 kron H_128 (Sylvester, natural
+// order), H_12 kron H_1024 = H_96 kron H_128 with H_96 = H_12 kron H_8, and the
+// transform splits into
+//   (1) a mix over a: D[o][beta] = sum_a H_96[o][a] x'[a*128+beta], run on the
+//       tensor cores: D (TMEM, fp32) = A * B with A = H_96 zero-padded to 128 x
+//       128 (bf16 +-1, K-major, built in shared memory once) and B = the
+//       sign-flipped token (K = a, N = beta; MN-major, 128-byte swizzle, two
+//       TMA boxes of 64 columns);
+//   (2) the H_128 over beta, run by the epilogue thread that owns TMEM lane o
+//       (o < 96): 128 columns in registers, seven butterfly stages in fp32.
+// That thread then holds the 128 contiguous outputs o*128 .. o*128+127.
+//
+// Exact scale.  The per-token scale fp32(max|y| / 7), y = S / sqrt(n), needs
+// max|S| exactly.  With the accumulation model of tcgen05.mma (see the
+// 4096-wide kernel: step k adds at most 2.5 u P_k plus the truncation of
+// inputs far below the step's largest term, at most 8 u P_k more; P_k =
+// partial column sum of |x|) the six steps err by at most 63 u C_beta per
+// column (C_beta = sum_a |x'[a][beta]|), and the seven fp32 stages by 7.01 u
+// sum|x| more, so |S_hat_i - S_i| <= 70.1 u sum|x| <= 70.1 u ||S||_2 (Cauchy-
+// Schwarz and ||S||_2 = sqrt(n) ||x||_2) <= E = 72 u ||S_hat||_2.  Every
+// output within 2E of the largest |S_hat| is recomputed exactly in fp64 by
+// the whole epilogue group from the input row in global memory.
+//
+// Warp roles (12 warps, three per scheduler, so a thread may hold 168
+// registers): 0 TMA producer, 1 MMA issuer + TMEM owner, 2-3 sign flip, 4-7
+// and 8-11 two epilogue groups taking alternate tokens (warp w reads TMEM
+// lane quarter w % 4; quarter 3 holds the zero padding of A and only helps
+// with reductions and fix-ups).  Every wait is bounded; on timeout the kernel
+// records an error code and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "kq_device.cuh"
+#include "kq_internal.h"
+#include "kq_sm100.cuh"
+
+namespace kq {
+namespace tcp {
+
+using namespace sm100;
+
+constexpr int N = 12288;
+constexpr int kRows = 96;                          // a
+constexpr int kCols = 128;                         // beta
+constexpr uint32_t kHalfBytes = kRows * 128;       // 96 rows x 64 columns (bf16)
+constexpr uint32_t kStageBytes = 2 * kHalfBytes;   // one token, 24 KB
+constexpr int kStages = 5;
+constexpr int kAcc = 4;                            // TMEM accumulators (128 columns each)
+constexpr int kTmemCols = kAcc * kCols;
+constexpr int kSignWarps = 2;
+constexpr int kThreads = 32 * 12;
+constexpr int kChunks = N / 8;                     // 16-byte chunks per token
+constexpr int kMaxCand = 32;                       // fix-up candidates handled per token
+constexpr double kBoundC = 72.0 * 0x1p-24;         // E = kBoundC ||S_hat||_2
+static_assert(kChunks % (32 * kSignWarps) == 0, "sign warps split the chunks evenly");
+static_assert(kChunks % 128 == 0, "an epilogue group splits the chunks evenly");
+
+__device__ unsigned int g_tcp_error = 0;           // nonzero: a wait timed out
+
+enum { kInt4 = 0, kRot = 1 };
+
+struct Params {
+  const uint16_t* x;     // bf16 [T, n]
+  uint8_t* codes;        // kInt4: [T, n/2]
+  float* scales;         // kInt4: [T]
+  float* out;            // kRot: fp32 [T, n]
+  int64_t tokens;
+  double sqrt_n;         // IEEE sqrt(12288)
+};
+
+// Per-group scratch for the token reductions.
+struct GroupScratch {
+  float wmax[4];
+  float wsq[4];
+  double part[4];
+  int wcnt[4];
+  int cand[kMaxCand];
+};
+
+__device__ __forceinline__ bool wait(uint64_t* bar, uint32_t parity) {
+  return sm100::mbar_wait(bar, parity, &g_tcp_error);
+}
+__device__ __forceinline__ void group_sync(int g) {
+  asm volatile("bar.sync %0, 128;" :: "r"(1 + g) : "memory");
+}
+
+// H_96[m][k] = H_12[m/8][k/8] (-1)^popc((m%8) & (k%8)), negative?
+__device__ __forceinline__ bool h96_negative(int m, int k) {
+  return paley_negative(m >> 3, k >> 3) ^ (__popc((m & 7) & (k & 7)) & 1);
+}
+
+// Exact S_i (fp64) of the token row `row` (bf16, global memory), computed by
+// the 128 threads of an epilogue group: thread tau takes the 16-byte chunks
+// tau, tau + 128, ...; chunk ch holds x[a*128 + c16*8 .. +7] (a = ch / 16, c16
+// = ch % 16) and its sign masks are smask[ch].  H[i][j] for i = o*128 + b,
+// j = a*128 + c16*8 + e is H_96[o][a] (-1)^(popc(b_hi & c16) + popc(b_lo & e)),
+// b_hi = b / 8, b_lo = b % 8.  Returns this thread's partial sum.
+__device__ __forceinline__ double exact_partial(const uint4* __restrict__ row,
+                                                const uint4* __restrict__ smask, int i,
+                                                int tau) {
+  const int o = i >> 7, bhi = (i >> 3) & 15, blo = i & 7;
+  uint32_t em[4];
+#pragma unroll
+  for (int w = 0; w < 4; ++w)
+    em[w] = ((uint32_t)(__popc(blo & (2 * w)) & 1) << 15) |
+            ((uint32_t)(__popc(blo & (2 * w + 1)) & 1) << 31);
+  double acc[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll 1
+  for (int k = 0; k < kChunks / 128; ++k) {
+    const int ch = tau + 128 * k;
+    const int a = ch >> 4, c16 = ch & 15;
+    const uint32_t flip =
+        (h96_negative(o, a) ^ (__popc(bhi & c16) & 1)) ? 0x80008000u : 0u;
+    const uint4 v = __ldg(row + ch);
+    const uint4 m = smask[ch];
+    const uint32_t ww[4] = {v.x ^ m.x, v.y ^ m.y, v.z ^ m.z, v.w ^ m.w};
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      double lo, hi;
+      bf16x2_to_f64_scaled(ww[w] ^ em[w] ^ flip, lo, hi);
+      acc[w] += lo;
+      acc[(w + 2) & 3] += hi;
+    }
+  }
+  return ((acc[0] + acc[1]) + (acc[2] + acc[3])) * kF64Unscale;
+}
+
+// Byte offset of 16-byte chunk c16 (0..15) of row a of a staged token: two
+// halves of 96 rows x 128 bytes (columns 64h .. 64h+63), 128-byte swizzle
+// (chunk c of row a at chunk position c ^ (a & 7)).
+__device__ __forceinline__ uint32_t b_chunk(int a, int c16) {
+  return (uint32_t)((c16 >> 3) * kHalfBytes + a * 128 + (((c16 & 7) ^ (a & 7)) << 4));
+}
+
+// Seven butterfly stages (H_128, natural order) on f[0..63] (f[p] holds
+// elements 2p, 2p + 1) in place.
+__device__ __forceinline__ void h128(float2 (&f)[64]) {
+#pragma unroll
+  for (int p = 0; p < 64; ++p) {
+    const float a = f[p].x, b = f[p].y;
+    f[p] = make_float2(a + b, a - b);
+  }
+#pragma unroll
+  for (int hh = 1; hh < 64; hh <<= 1)
+#pragma unroll
+    for (int p = 0; p < 64; ++p)
+      if (!(p & hh)) bfly2(f[p], f[p | hh]);
+}
+
+// Two's-complement INT4 nibble in the low 4 bits of the fp32 value
+// t = v * c + 1.5 * 2^23 (one rounding: the integer nearest v * c, ties to
+// even, for |v * c| < 2^22).
+constexpr float kRneMagic = 12582912.0f;
+
+// Eight values (4 pairs) -> 8 nibbles, element k in bits 4k .. 4k + 3.
+__device__ __forceinline__ uint32_t int4x8(const float2* f, float2 c2) {
+  const float2 m2 = make_float2(kRneMagic, kRneMagic);
+  uint32_t byte[4];
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    const float2 t = fma2(f[p], c2, m2);
+    byte[p] = (__float_as_uint(t.x) & 0xFu) | ((__float_as_uint(t.y) & 0xFu) << 4);
+  }
+  return __byte_perm(__byte_perm(byte[0], byte[1], 0x0040), __byte_perm(byte[2], byte[3], 0x0040),
+                     0x5410);
+}
+
+template <int kMode>
+__global__ void __launch_bounds__(kThreads, 1)
+k_tc12288(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ signs, Params P) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sA = smem;                                    // 32 KB: A = H_96, zero-padded
+  uint8_t* sB = smem + 32768;                            // kStages x 24 KB
+  uint4* smask = reinterpret_cast<uint4*>(sB + kStages * kStageBytes);   // kChunks
+  GroupScratch* gs = reinterpret_cast<GroupScratch*>(smask + kChunks);   // 2 groups
+  uint64_t* bars = reinterpret_cast<uint64_t*>(gs + 2);
+  uint64_t* full = bars;                                 // TMA landed
+  uint64_t* ready = bars + kStages;                      // signs applied
+  uint64_t* empty = bars + 2 * kStages;                  // MMAs done reading the stage
+  uint64_t* tfull = bars + 3 * kStages;                  // accumulator written (kAcc)
+  uint64_t* tempty = tfull + kAcc;                       // accumulator read (kAcc)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + kAcc);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---- set-up: A operand, sign masks, barriers, TMEM
+  for (int idx = threadIdx.x; idx < 128 * 128; idx += blockDim.x) {
+    const int m = idx >> 7, k = idx & 127;
+    uint16_t v = 0;                                       // zero padding
+    if (m < kRows && k < kRows) v = h96_negative(m, k) ? 0xBF80 : 0x3F80;   // -1 / +1
+    *reinterpret_cast<uint16_t*>(sA + a_off(m, k)) = v;
+  }
+  for (int i = threadIdx.x; i < kChunks; i += blockDim.x) {
+    uint4 m4 = make_uint4(0, 0, 0, 0);
+    if (signs) {
+      const uint2 sv = __ldg(reinterpret_cast<const uint2*>(signs) + i);
+      m4 = make_uint4(__byte_perm(sv.x, 0, 0x1404) & 0x80008000u,
+                      __byte_perm(sv.x, 0, 0x3424) & 0x80008000u,
+                      __byte_perm(sv.y, 0, 0x1404) & 0x80008000u,
+                      __byte_perm(sv.y, 0, 0x3424) & 0x80008000u);
+    }
+    smask[i] = m4;
+  }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&ready[s], 32 * kSignWarps);
+      mbar_init(&empty[s], 1);
+    }
+    for (int d = 0; d < kAcc; ++d) {
+      mbar_init(&tfull[d], 1);
+      mbar_init(&tempty[d], 128);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 :: "r"(smem_u32(tmem_slot)), "n"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int64_t my_tiles = (P.tokens - blockIdx.x + gridDim.x - 1) / gridDim.x;
+
+  if (warp == 0) {
+    // ================= TMA producer: two 96-row boxes per token
+    if (lane == 0) {
+      int64_t issued = 0;
+      for (int64_t k = 0; k < my_tiles; ++k) {
+        const int s = (int)(k % kStages);
+        if (k >= kStages && !wait(&empty[s], (uint32_t)(k / kStages - 1) & 1)) break;
+        const int64_t token = blockIdx.x + k * gridDim.x;
+        mbar_expect_tx(&full[s], kStageBytes);
+        tma_load_2d(sB + s * kStageBytes, &tmap, 0, (int)(token * kRows), &full[s]);
+        tma_load_2d(sB + s * kStageBytes + kHalfBytes, &tmap, 64, (int)(token * kRows),
+                    &full[s]);
+        issued = k + 1;
+      }
+      // no copy may still be in flight when the CTA exits
+      for (int64_t k = issued > kStages ? issued - kStages : 0; k < issued; ++k)
+        wait(&full[k % kStages], (uint32_t)(k / kStages) & 1);
+    }
+  } else if (warp == 1) {
+    // ================= MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(128, kCols, 1);
+      int64_t issued = 0;
+      for (int64_t k = 0; k < my_tiles; ++k) {
+        const int s = (int)(k % kStages);
+        const int d = (int)(k % kAcc);
+        if (!wait(&ready[s], (uint32_t)(k / kStages) & 1)) break;
+        if (k >= kAcc && !wait(&tempty[d], (uint32_t)(k / kAcc - 1) & 1)) break;
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB + s * kStageBytes);
+        const uint32_t tmem_d = tmem_base + (uint32_t)(d * kCols);
+#pragma unroll
+        for (int ks = 0; ks < kRows / 16; ++ks) {
+          // A: K-major, K step of 16 = 32 bytes inside a 128-byte swizzle row
+          const uint64_t adesc = smem_desc(a0 + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, 2);
+          // B: MN-major 128-byte swizzle atoms of 64 columns (the two halves,
+          // kHalfBytes apart), 8-row groups 1 KB apart; K step of 16 rows = 2 KB
+          const uint64_t bdesc = smem_desc(b0 + ks * 2048, kHalfBytes, 1024, 2);
+          mma_bf16(tmem_d, adesc, bdesc, idesc, ks > 0 ? 1u : 0u);
+        }
+        mma_commit(&empty[s]);
+        mma_commit(&tfull[d]);
+        issued = k + 1;
+      }
+      for (int64_t k = issued > kAcc ? issued - kAcc : 0; k < issued; ++k)
+        wait(&tfull[k % kAcc], (uint32_t)(k / kAcc) & 1);
+    }
+  } else if (warp < 2 + kSignWarps) {
+    // ================= sign flip: lane l of sign warp w takes the physical
+    // chunks l + 32 w + 64 i (conflict-free), whatever logical chunk they hold
+    const int t0 = (warp - 2) * 32 + lane;
+    for (int64_t k = 0; k < my_tiles; ++k) {
+      const int s = (int)(k % kStages);
+      if (!wait(&full[s], (uint32_t)(k / kStages) & 1)) break;
+      if (signs) {
+        uint8_t* st = sB + s * kStageBytes;
+#pragma unroll 4
+        for (int i = 0; i < kChunks / 64; ++i) {
+          const int pc = t0 + 64 * i;                 // physical chunk
+          const int h = pc / (kRows * 8), r = pc % (kRows * 8);
+          const int a = r >> 3, c16 = h * 8 + ((r & 7) ^ (a & 7));
+          uint4* p = reinterpret_cast<uint4*>(st) + pc;
+          uint4 w = *p;
+          const uint4 m = smask[a * 16 + c16];
+          w.x ^= m.x;
+          w.y ^= m.y;
+          w.z ^= m.z;
+          w.w ^= m.w;
+          *p = w;
+        }
+        fence_async_smem();
+      }
+      __syncwarp();
+      mbar_arrive(&ready[s]);
+    }
+  } else {
+    // ================= epilogue: group g of warps 4+4g .. 7+4g
+    const int g = (warp - 4) >> 2;
+    const int q = warp & 3;                   // TMEM lane quarter
+    const int o = q * 32 + lane;              // accumulator row = thread within group
+    const bool rowv = o < kRows;
+    GroupScratch& S = gs[g];
+    for (int64_t k = g; k < my_tiles; k += 2) {
+      const int d = (int)(k % kAcc);
+      const int64_t token = blockIdx.x + k * gridDim.x;
+      // A timed-out wait does not leave the loop: the failure is recorded and
+      // the token's outputs are not written.
+      const bool ok = wait(&tfull[d], (uint32_t)(k / kAcc) & 1);
+      tc_fence_after();
+      float2 f[64];
+      if (rowv) {
+        const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(d * kCols);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          tmem_ld32(taddr + c * 32, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            f[16 * c + e] = make_float2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
+        }
+      } else {
+#pragma unroll
+        for (int p = 0; p < 64; ++p) f[p] = make_float2(0.0f, 0.0f);
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[d]);
+      h128(f);
+
+      if (kMode == kRot) {
+        if (ok && rowv) {
+          const float inv = (float)(1.0 / P.sqrt_n);
+          float4* dst = reinterpret_cast<float4*>(P.out + token * N + o * 128);
+#pragma unroll
+          for (int p = 0; p < 32; ++p)
+            dst[p] = make_float4(f[2 * p].x * inv, f[2 * p].y * inv, f[2 * p + 1].x * inv,
+                                 f[2 * p + 1].y * inv);
+        }
+        continue;
+      }
+
+      // ---- token maximum and ||S_hat||_2^2 over the group
+      float mx = 0.0f, sq = 0.0f;
+#pragma unroll
+      for (int p = 0; p < 64; ++p) {
+        mx = fmax3(mx, fabsf(f[p].x), fabsf(f[p].y));
+        sq = fmaf(f[p].x, f[p].x, fmaf(f[p].y, f[p].y, sq));
+      }
+      const float own_mx = mx;
+      mx = warp_max(mx);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
+      group_sync(g);                           // the previous token's scratch reads are done
+      if (lane == 0) {
+        S.wmax[q] = mx;
+        S.wsq[q] = sq;
+      }
+      group_sync(g);
+      const float M = fmaxf(fmaxf(S.wmax[0], S.wmax[1]), fmaxf(S.wmax[2], S.wmax[3]));
+      const float Q = (S.wsq[0] + S.wsq[1]) + (S.wsq[2] + S.wsq[3]);
+      const bool finite = isfinite(M) && isfinite(Q);
+      // fp32 sums of 12288 squares err by far less than 2^-10 relative
+      const double E = kBoundC * sqrt((double)Q * (1.0 + 0x1p-10));
+      const float thr = __double2float_rd((double)M - 2.0 * E);
+
+      // ---- candidates: every output within 2E of the maximum, ranked
+      uint32_t cm[4] = {0u, 0u, 0u, 0u};
+      if (rowv && finite && M > 0.0f && own_mx >= thr) {
+#pragma unroll
+        for (int p = 0; p < 64; ++p) {
+          if (fabsf(f[p].x) >= thr) cm[p >> 4] |= 1u << (2 * (p & 15));
+          if (fabsf(f[p].y) >= thr) cm[p >> 4] |= 1u << (2 * (p & 15) + 1);
+        }
+      }
+      const int myc = __popc(cm[0]) + __popc(cm[1]) + __popc(cm[2]) + __popc(cm[3]);
+      int incl = myc;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+      }
+      if (lane == 31) S.wcnt[q] = incl;
+      group_sync(g);
+      int base = 0, total = 0;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        base += (w < q) ? S.wcnt[w] : 0;
+        total += S.wcnt[w];
+      }
+      const int rank0 = base + incl - myc;
+
+      // ---- exact maximum over the candidates, kMaxCand at a time
+      double best = 0.0;
+      const uint16_t* xrow = P.x + token * N;
+      for (int r0 = 0; r0 < total; r0 += kMaxCand) {
+        if (myc > 0 && rank0 < r0 + kMaxCand && rank0 + myc > r0) {
+          int rk = rank0;
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            uint32_t bits = cm[w];
+            while (bits) {
+              const int b = __ffs(bits) - 1;
+              bits &= bits - 1;
+              if (rk >= r0 && rk < r0 + kMaxCand) S.cand[rk - r0] = o * 128 + w * 32 + b;
+              ++rk;
+            }
+          }
+        }
+        group_sync(g);
+        const int nc = min(kMaxCand, total - r0);
+        for (int c = 0; c < nc; ++c) {
+          const int i = S.cand[c];
+          double part = exact_partial(reinterpret_cast<const uint4*>(xrow), smask, i, o);
+          part = warp_sum_d(part);
+          if (lane == 0) S.part[q] = part;
+          group_sync(g);
+          best = fmax(best, fabs((S.part[0] + S.part[1]) + (S.part[2] + S.part[3])));
+          group_sync(g);
+        }
+      }
+
+      // ---- scale and codes: 64 bytes per row thread.  A row holding an
+      // infinity or NaN gets the scale of its computed maximum (not exact).
+      if (!finite) best = (double)M;
+      const float scale = (M > 0.0f || !finite) ? __double2float_rn((best / P.sqrt_n) / 7.0)
+                                                : 0.0f;
+      if (ok && rowv) {
+        const float cq = scale > 0.0f ? __double2float_rn(1.0 / (P.sqrt_n * (double)scale)) : 0.0f;
+        const float2 c2 = make_float2(cq, cq);
+        uint4* dst = reinterpret_cast<uint4*>(P.codes + token * (N / 2) + o * 64);
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+          dst[w] = make_uint4(int4x8(f + 16 * w, c2), int4x8(f + 16 * w + 4, c2),
+                              int4x8(f + 16 * w + 8, c2), int4x8(f + 16 * w + 12, c2));
+      }
+      if (ok && o == 0) P.scales[token] = scale;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;"
+                 :: "r"(tmem_base), "n"(kTmemCols));
+  }
+}
+
+}  // namespace tcp
+
+// ------------------------------------------------------------- launchers
+namespace {
+
+constexpr size_t kTcpSmem = 1024 + 32768 + tcp::kStages * tcp::kStageBytes +
+                            tcp::kChunks * 16 + 2 * sizeof(tcp::GroupScratch) + 256;
+
+template <int kMode>
+cudaError_t launch_tcp(const void* x, const int8_t* signs, tcp::Params& P, const Geometry& g,
+                       cudaStream_t s) {
+  CUtensorMap map;
+  // [tokens * 96, 128] view: rows of 256 bytes, 64 x 96 boxes (half a token)
+  if (!encode_tmap_bf16_2d(&map, x, tcp::kCols, (uint64_t)P.tokens * tcp::kRows, 64,
+                           tcp::kRows, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorNotSupported;
+  P.sqrt_n = g.sqrt_b;
+  auto k = tcp::k_tc12288<kMode>;
+  cudaFuncSetAttribute((const void*)k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       (int)kTcpSmem);
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t grid = P.tokens < sms ? P.tokens : sms;
+  k<<<(int)grid, tcp::kThreads, kTcpSmem, s>>>(map, signs, P);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool tcp_supported(const Geometry& g, int dtype, const void* x, int64_t tokens) {
+  // TMA: 16-byte aligned base, int32 row coordinates (tokens * 96)
+  return dtype == 1 && g.paley && g.b == g.n && g.n == tcp::N &&
+         (reinterpret_cast<uintptr_t>(x) & 15) == 0 && tokens < (int64_t(1) << 24);
+}
+
+cudaError_t launch_tcp_int4(const void* x, int64_t tokens, const Geometry& g,
+                            const int8_t* signs, uint8_t* codes, float* scales, cudaStream_t s) {
+  tcp::Params P{};
+  P.x = static_cast<const uint16_t*>(x);
+  P.codes = codes;
+  P.scales = scales;
+  P.tokens = tokens;
+  return launch_tcp<tcp::kInt4>(x, signs, P, g, s);
+}
+
+cudaError_t launch_tcp_rot(const void* x, int64_t tokens, const Geometry& g,
+                           const int8_t* signs, float* out, cudaStream_t s) {
+  tcp::Params P{};
+  P.x = static_cast<const uint16_t*>(x);
+  P.out = out;
+  P.tokens = tokens;
+  return launch_tcp<tcp::kRot>(x, signs, P, g, s);
+}
+
+}  // namespace kq
