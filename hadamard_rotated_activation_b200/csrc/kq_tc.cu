@@ -239,24 +239,11 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // ---- set-up: A operand, sign masks, barriers, TMEM
-  for (int idx = threadIdx.x; idx < 128 * 128; idx += blockDim.x) {
-    const int m = idx >> 7, k = idx & 127;
-    const uint16_t v = (__popc(m & k) & 1) ? 0xBF80 : 0x3F80;    // -1 / +1 in bf16
-    *reinterpret_cast<uint16_t*>(sA + a_off(m, k)) = v;
-  }
-  for (int i = threadIdx.x; i < 512; i += blockDim.x) {
-    // chunk i = (a, c): elements 8i .. 8i+7 = a*32 + c*8 .. +7
-    uint4 m4 = make_uint4(0, 0, 0, 0);
-    if (signs) {
-      const uint2 sv = __ldg(reinterpret_cast<const uint2*>(signs) + i);
-      m4 = make_uint4(__byte_perm(sv.x, 0, 0x1404) & 0x80008000u,
-                      __byte_perm(sv.x, 0, 0x3424) & 0x80008000u,
-                      __byte_perm(sv.y, 0, 0x1404) & 0x80008000u,
-                      __byte_perm(sv.y, 0, 0x3424) & 0x80008000u);
-    }
-    smask[i] = m4;
-  }
+  const int64_t my_tiles = (P.tiles - blockIdx.x + gridDim.x - 1) / gridDim.x;
+
+  // ---- set-up.  The producer thread initialises the barriers and starts the
+  // first copies before the rest of the set-up, so they overlap it.
+  int64_t prefilled = 0;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
@@ -271,6 +258,39 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
     fq->head = 0;
     fq->done = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    prefilled = my_tiles < kStages ? my_tiles : kStages;
+    for (int64_t k = 0; k < prefilled; ++k) {
+      const int64_t tile = blockIdx.x + k * gridDim.x;
+      mbar_expect_tx(&full[k], kStageBytes);
+#pragma unroll
+      for (int t = 0; t < kTok; ++t)
+        tma_load_2d(sB + k * kStageBytes + t * kTokBytes, &tmap, 0,
+                    (int)((tile * kTok + t) * 128), &full[k]);
+    }
+  }
+  // A = H_128, one 16-byte chunk (8 columns) per step
+  for (int idx = threadIdx.x; idx < 128 * 16; idx += blockDim.x) {
+    const int m = idx >> 4, k0 = (idx & 15) * 8;
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t lo = (__popc(m & (k0 + 2 * e)) & 1) ? 0xBF80u : 0x3F80u;   // -1 / +1
+      const uint32_t hi = (__popc(m & (k0 + 2 * e + 1)) & 1) ? 0xBF80u : 0x3F80u;
+      w[e] = lo | (hi << 16);
+    }
+    *reinterpret_cast<uint4*>(sA + a_off(m, k0)) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  for (int i = threadIdx.x; i < 512; i += blockDim.x) {
+    // chunk i = (a, c): elements 8i .. 8i+7 = a*32 + c*8 .. +7
+    uint4 m4 = make_uint4(0, 0, 0, 0);
+    if (signs) {
+      const uint2 sv = __ldg(reinterpret_cast<const uint2*>(signs) + i);
+      m4 = make_uint4(__byte_perm(sv.x, 0, 0x1404) & 0x80008000u,
+                      __byte_perm(sv.x, 0, 0x3424) & 0x80008000u,
+                      __byte_perm(sv.y, 0, 0x1404) & 0x80008000u,
+                      __byte_perm(sv.y, 0, 0x3424) & 0x80008000u);
+    }
+    smask[i] = m4;
   }
   for (int i = threadIdx.x; i < kQ; i += blockDim.x) fq->seq[i] = 0;
   if (warp == 1) {
@@ -284,13 +304,12 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int64_t my_tiles = (P.tiles - blockIdx.x + gridDim.x - 1) / gridDim.x;
 
   if (warp == 0) {
     // ================= TMA producer: one 128-row box per token
     if (lane == 0) {
-      int64_t issued = 0;
-      for (int64_t k = 0; k < my_tiles; ++k) {
+      int64_t issued = prefilled;
+      for (int64_t k = prefilled; k < my_tiles; ++k) {
         const int s = (int)(k % kStages);
         const uint32_t use = (uint32_t)(k / kStages);
         if (k >= kStages && !mbar_wait(&empty[s], (use - 1) & 1)) break;

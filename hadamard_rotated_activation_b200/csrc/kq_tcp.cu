@@ -26,7 +26,8 @@
 // sum|x| more, so |S_hat_i - S_i| <= 70.1 u sum|x| <= 70.1 u ||S||_2 (Cauchy-
 // Schwarz and ||S||_2 = sqrt(n) ||x||_2) <= E = 72 u ||S_hat||_2.  Every
 // output within 2E of the largest |S_hat| is recomputed exactly in fp64 by
-// the whole epilogue group from the input row in global memory.
+// the whole epilogue group from the staged token, which the epilogue holds
+// until then.
 //
 // Warp roles (12 warps, three per scheduler, so a thread may hold 168
 // registers): 0 TMA producer, 1 MMA issuer + TMEM owner, 2-3 sign flip, 4-7
@@ -71,7 +72,6 @@ __device__ unsigned int g_tcp_error = 0;           // nonzero: a wait timed out
 enum { kInt4 = 0, kRot = 1 };
 
 struct Params {
-  const uint16_t* x;     // bf16 [T, n]
   uint8_t* codes;        // kInt4: [T, n/2]
   float* scales;         // kInt4: [T]
   float* out;            // kRot: fp32 [T, n]
@@ -100,15 +100,21 @@ __device__ __forceinline__ bool h96_negative(int m, int k) {
   return paley_negative(m >> 3, k >> 3) ^ (__popc((m & 7) & (k & 7)) & 1);
 }
 
-// Exact S_i (fp64) of the token row `row` (bf16, global memory), computed by
-// the 128 threads of an epilogue group: thread tau takes the 16-byte chunks
-// tau, tau + 128, ...; chunk ch holds x[a*128 + c16*8 .. +7] (a = ch / 16, c16
-// = ch % 16) and its sign masks are smask[ch].  H[i][j] for i = o*128 + b,
-// j = a*128 + c16*8 + e is H_96[o][a] (-1)^(popc(b_hi & c16) + popc(b_lo & e)),
-// b_hi = b / 8, b_lo = b % 8.  Returns this thread's partial sum.
-__device__ __forceinline__ double exact_partial(const uint4* __restrict__ row,
-                                                const uint4* __restrict__ smask, int i,
-                                                int tau) {
+// Byte offset of 16-byte chunk c16 (0..15) of row a of a staged token: two
+// halves of 96 rows x 128 bytes (columns 64h .. 64h+63), 128-byte swizzle
+// (chunk c of row a at chunk position c ^ (a & 7)).
+__device__ __forceinline__ uint32_t b_chunk(int a, int c16) {
+  return (uint32_t)((c16 >> 3) * kHalfBytes + a * 128 + (((c16 & 7) ^ (a & 7)) << 4));
+}
+
+// Exact S_i (fp64) of a staged, sign-flipped token, computed by the 128
+// threads of an epilogue group: thread tau takes the 16-byte chunks tau,
+// tau + 128, ...; chunk ch holds x'[a*128 + c16*8 .. +7] (a = ch / 16, c16 =
+// ch % 16).  H[i][j] for i = o*128 + b, j = a*128 + c16*8 + e is H_96[o][a]
+// (-1)^(popc(b_hi & c16) + popc(b_lo & e)), b_hi = b / 8, b_lo = b % 8.
+// Values enter fp64 exactly through bf16x2_to_f64_scaled.  Returns this
+// thread's partial sum.
+__device__ __forceinline__ double exact_partial(const uint8_t* tok, int i, int tau) {
   const int o = i >> 7, bhi = (i >> 3) & 15, blo = i & 7;
   uint32_t em[4];
 #pragma unroll
@@ -116,15 +122,14 @@ __device__ __forceinline__ double exact_partial(const uint4* __restrict__ row,
     em[w] = ((uint32_t)(__popc(blo & (2 * w)) & 1) << 15) |
             ((uint32_t)(__popc(blo & (2 * w + 1)) & 1) << 31);
   double acc[4] = {0.0, 0.0, 0.0, 0.0};
-#pragma unroll 1
+#pragma unroll 2
   for (int k = 0; k < kChunks / 128; ++k) {
     const int ch = tau + 128 * k;
     const int a = ch >> 4, c16 = ch & 15;
     const uint32_t flip =
         (h96_negative(o, a) ^ (__popc(bhi & c16) & 1)) ? 0x80008000u : 0u;
-    const uint4 v = __ldg(row + ch);
-    const uint4 m = smask[ch];
-    const uint32_t ww[4] = {v.x ^ m.x, v.y ^ m.y, v.z ^ m.z, v.w ^ m.w};
+    const uint4 v = *reinterpret_cast<const uint4*>(tok + b_chunk(a, c16));
+    const uint32_t ww[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
       double lo, hi;
@@ -134,13 +139,6 @@ __device__ __forceinline__ double exact_partial(const uint4* __restrict__ row,
     }
   }
   return ((acc[0] + acc[1]) + (acc[2] + acc[3])) * kF64Unscale;
-}
-
-// Byte offset of 16-byte chunk c16 (0..15) of row a of a staged token: two
-// halves of 96 rows x 128 bytes (columns 64h .. 64h+63), 128-byte swizzle
-// (chunk c of row a at chunk position c ^ (a & 7)).
-__device__ __forceinline__ uint32_t b_chunk(int a, int c16) {
-  return (uint32_t)((c16 >> 3) * kHalfBytes + a * 128 + (((c16 & 7) ^ (a & 7)) << 4));
 }
 
 // Seven butterfly stages (H_128, natural order) on f[0..63] (f[p] holds
@@ -189,19 +187,51 @@ k_tc12288(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ s
   uint64_t* bars = reinterpret_cast<uint64_t*>(gs + 2);
   uint64_t* full = bars;                                 // TMA landed
   uint64_t* ready = bars + kStages;                      // signs applied
-  uint64_t* empty = bars + 2 * kStages;                  // MMAs done reading the stage
+  uint64_t* empty = bars + 2 * kStages;                  // MMAs and fix-ups done with the stage
   uint64_t* tfull = bars + 3 * kStages;                  // accumulator written (kAcc)
   uint64_t* tempty = tfull + kAcc;                       // accumulator read (kAcc)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + kAcc);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // ---- set-up: A operand, sign masks, barriers, TMEM
-  for (int idx = threadIdx.x; idx < 128 * 128; idx += blockDim.x) {
-    const int m = idx >> 7, k = idx & 127;
-    uint16_t v = 0;                                       // zero padding
-    if (m < kRows && k < kRows) v = h96_negative(m, k) ? 0xBF80 : 0x3F80;   // -1 / +1
-    *reinterpret_cast<uint16_t*>(sA + a_off(m, k)) = v;
+  const int64_t my_tiles = (P.tokens - blockIdx.x + gridDim.x - 1) / gridDim.x;
+
+  // ---- set-up.  The producer thread initialises the barriers and starts the
+  // first copies before the rest of the set-up, so they overlap it.
+  int64_t prefilled = 0;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&ready[s], 32 * kSignWarps);
+      mbar_init(&empty[s], kMode == kInt4 ? 2 : 1);   // MMA commit [+ epilogue]
+    }
+    for (int d = 0; d < kAcc; ++d) {
+      mbar_init(&tfull[d], 1);
+      mbar_init(&tempty[d], 128);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    prefilled = my_tiles < kStages ? my_tiles : kStages;
+    for (int64_t k = 0; k < prefilled; ++k) {
+      const int64_t token = blockIdx.x + k * gridDim.x;
+      mbar_expect_tx(&full[k], kStageBytes);
+      tma_load_2d(sB + k * kStageBytes, &tmap, 0, (int)(token * kRows), &full[k]);
+      tma_load_2d(sB + k * kStageBytes + kHalfBytes, &tmap, 64, (int)(token * kRows), &full[k]);
+    }
+  }
+  // A = H_96 zero-padded, one 16-byte chunk (8 columns) per step
+  for (int idx = threadIdx.x; idx < 128 * 16; idx += blockDim.x) {
+    const int m = idx >> 4, k0 = (idx & 15) * 8;
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      uint32_t lo = 0, hi = 0;                        // zero padding
+      if (m < kRows && k0 + 2 * e < kRows) {
+        lo = h96_negative(m, k0 + 2 * e) ? 0xBF80u : 0x3F80u;       // -1 / +1
+        hi = h96_negative(m, k0 + 2 * e + 1) ? 0xBF80u : 0x3F80u;
+      }
+      w[e] = lo | (hi << 16);
+    }
+    *reinterpret_cast<uint4*>(sA + a_off(m, k0)) = make_uint4(w[0], w[1], w[2], w[3]);
   }
   for (int i = threadIdx.x; i < kChunks; i += blockDim.x) {
     uint4 m4 = make_uint4(0, 0, 0, 0);
@@ -214,18 +244,6 @@ k_tc12288(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ s
     }
     smask[i] = m4;
   }
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&ready[s], 32 * kSignWarps);
-      mbar_init(&empty[s], 1);
-    }
-    for (int d = 0; d < kAcc; ++d) {
-      mbar_init(&tfull[d], 1);
-      mbar_init(&tempty[d], 128);
-    }
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                  :: "r"(smem_u32(tmem_slot)), "n"(kTmemCols));
@@ -237,13 +255,12 @@ k_tc12288(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ s
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int64_t my_tiles = (P.tokens - blockIdx.x + gridDim.x - 1) / gridDim.x;
 
   if (warp == 0) {
     // ================= TMA producer: two 96-row boxes per token
     if (lane == 0) {
-      int64_t issued = 0;
-      for (int64_t k = 0; k < my_tiles; ++k) {
+      int64_t issued = prefilled;
+      for (int64_t k = prefilled; k < my_tiles; ++k) {
         const int s = (int)(k % kStages);
         if (k >= kStages && !wait(&empty[s], (uint32_t)(k / kStages - 1) & 1)) break;
         const int64_t token = blockIdx.x + k * gridDim.x;
@@ -288,26 +305,33 @@ k_tc12288(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ s
     }
   } else if (warp < 2 + kSignWarps) {
     // ================= sign flip: lane l of sign warp w takes the physical
-    // chunks l + 32 w + 64 i (conflict-free), whatever logical chunk they hold
+    // chunks t0 + 64 i (conflict-free), i = 0..23: half i / 12, row a = t0 / 8 +
+    // 8 (i % 12), slot t0 % 8, which holds logical chunk (t0 % 8) ^ (a % 8) of
+    // the half.  The lane's 24 sign masks stay in registers.
     const int t0 = (warp - 2) * 32 + lane;
+    constexpr int kPer = kChunks / 64;
+    uint4 msk[kPer];
+    {
+      const int cl = (t0 & 7) ^ ((t0 >> 3) & 7);
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) {
+        const int a = (t0 >> 3) + 8 * (i % 12);
+        msk[i] = smask[a * 16 + (i / 12) * 8 + cl];
+      }
+    }
     for (int64_t k = 0; k < my_tiles; ++k) {
       const int s = (int)(k % kStages);
       if (!wait(&full[s], (uint32_t)(k / kStages) & 1)) break;
       if (signs) {
-        uint8_t* st = sB + s * kStageBytes;
-#pragma unroll 4
-        for (int i = 0; i < kChunks / 64; ++i) {
-          const int pc = t0 + 64 * i;                 // physical chunk
-          const int h = pc / (kRows * 8), r = pc % (kRows * 8);
-          const int a = r >> 3, c16 = h * 8 + ((r & 7) ^ (a & 7));
-          uint4* p = reinterpret_cast<uint4*>(st) + pc;
-          uint4 w = *p;
-          const uint4 m = smask[a * 16 + c16];
-          w.x ^= m.x;
-          w.y ^= m.y;
-          w.z ^= m.z;
-          w.w ^= m.w;
-          *p = w;
+        uint4* st = reinterpret_cast<uint4*>(sB + s * kStageBytes) + t0;
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+          uint4 w = st[64 * i];
+          w.x ^= msk[i].x;
+          w.y ^= msk[i].y;
+          w.z ^= msk[i].z;
+          w.w ^= msk[i].w;
+          st[64 * i] = w;
         }
         fence_async_smem();
       }
@@ -323,6 +347,7 @@ k_tc12288(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ s
     GroupScratch& S = gs[g];
     for (int64_t k = g; k < my_tiles; k += 2) {
       const int d = (int)(k % kAcc);
+      const int st = (int)(k % kStages);
       const int64_t token = blockIdx.x + k * gridDim.x;
       // A timed-out wait does not leave the loop: the failure is recorded and
       // the token's outputs are not written.
@@ -412,7 +437,8 @@ k_tc12288(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ s
 
       // ---- exact maximum over the candidates, kMaxCand at a time
       double best = 0.0;
-      const uint16_t* xrow = P.x + token * N;
+      const uint8_t* tok = sB + st * kStageBytes;   // held until the fix-ups are done
+      if (total > 0) wait(&ready[st], (uint32_t)(k / kStages) & 1);   // sign flips visible
       for (int r0 = 0; r0 < total; r0 += kMaxCand) {
         if (myc > 0 && rank0 < r0 + kMaxCand && rank0 + myc > r0) {
           int rk = rank0;
@@ -431,7 +457,7 @@ k_tc12288(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ s
         const int nc = min(kMaxCand, total - r0);
         for (int c = 0; c < nc; ++c) {
           const int i = S.cand[c];
-          double part = exact_partial(reinterpret_cast<const uint4*>(xrow), smask, i, o);
+          double part = exact_partial(tok, i, o);
           part = warp_sum_d(part);
           if (lane == 0) S.part[q] = part;
           group_sync(g);
@@ -439,6 +465,8 @@ k_tc12288(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ s
           group_sync(g);
         }
       }
+
+      if (o == 0) mbar_arrive(&empty[st]);   // every read of the stage is behind a group sync
 
       // ---- scale and codes: 64 bytes per row thread.  A row holding an
       // infinity or NaN gets the scale of its computed maximum (not exact).
@@ -506,7 +534,6 @@ bool tcp_supported(const Geometry& g, int dtype, const void* x, int64_t tokens) 
 cudaError_t launch_tcp_int4(const void* x, int64_t tokens, const Geometry& g,
                             const int8_t* signs, uint8_t* codes, float* scales, cudaStream_t s) {
   tcp::Params P{};
-  P.x = static_cast<const uint16_t*>(x);
   P.codes = codes;
   P.scales = scales;
   P.tokens = tokens;
@@ -516,7 +543,6 @@ cudaError_t launch_tcp_int4(const void* x, int64_t tokens, const Geometry& g,
 cudaError_t launch_tcp_rot(const void* x, int64_t tokens, const Geometry& g,
                            const int8_t* signs, float* out, cudaStream_t s) {
   tcp::Params P{};
-  P.x = static_cast<const uint16_t*>(x);
   P.out = out;
   P.tokens = tokens;
   return launch_tcp<tcp::kRot>(x, signs, P, g, s);
