@@ -83,8 +83,9 @@ struct Params {
 struct GroupScratch {
   float wmax[4];
   float wsq[4];
-  double part[4];
+  double part[2][4];     // per candidate parity
   int wcnt[4];
+  int ncand;
   int cand[kMaxCand];
 };
 
@@ -183,8 +184,8 @@ k_tc12288(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ s
   uint8_t* sA = smem;                                    // 32 KB: A = H_96, zero-padded
   uint8_t* sB = smem + 32768;                            // kStages x 24 KB
   uint4* smask = reinterpret_cast<uint4*>(sB + kStages * kStageBytes);   // kChunks
-  GroupScratch* gs = reinterpret_cast<GroupScratch*>(smask + kChunks);   // 2 groups
-  uint64_t* bars = reinterpret_cast<uint64_t*>(gs + 2);
+  GroupScratch* gs = reinterpret_cast<GroupScratch*>(smask + kChunks);   // 2 groups x 2
+  uint64_t* bars = reinterpret_cast<uint64_t*>(gs + 4);
   uint64_t* full = bars;                                 // TMA landed
   uint64_t* ready = bars + kStages;                      // signs applied
   uint64_t* empty = bars + 2 * kStages;                  // MMAs and fix-ups done with the stage
@@ -344,128 +345,158 @@ k_tc12288(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ s
     const int q = warp & 3;                   // TMEM lane quarter
     const int o = q * 32 + lane;              // accumulator row = thread within group
     const bool rowv = o < kRows;
-    GroupScratch& S = gs[g];
     for (int64_t k = g; k < my_tiles; k += 2) {
       const int d = (int)(k % kAcc);
       const int st = (int)(k % kStages);
       const int64_t token = blockIdx.x + k * gridDim.x;
+      // scratch alternates between the group's consecutive tokens, so a token
+      // never overwrites one that a slower warp may still be reading
+      GroupScratch& S = gs[2 * g + ((k >> 1) & 1)];
       // A timed-out wait does not leave the loop: the failure is recorded and
       // the token's outputs are not written.
       const bool ok = wait(&tfull[d], (uint32_t)(k / kAcc) & 1);
       tc_fence_after();
-      float2 f[64];
-      if (rowv) {
-        const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(d * kCols);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tmem_ld32(taddr + c * 32, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 16; ++e)
-            f[16 * c + e] = make_float2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
-        }
-      } else {
-#pragma unroll
-        for (int p = 0; p < 64; ++p) f[p] = make_float2(0.0f, 0.0f);
-      }
-      tc_fence_before();
-      mbar_arrive(&tempty[d]);
-      h128(f);
-
-      if (kMode == kRot) {
-        if (ok && rowv) {
-          const float inv = (float)(1.0 / P.sqrt_n);
-          float4* dst = reinterpret_cast<float4*>(P.out + token * N + o * 128);
-#pragma unroll
-          for (int p = 0; p < 32; ++p)
-            dst[p] = make_float4(f[2 * p].x * inv, f[2 * p].y * inv, f[2 * p + 1].x * inv,
-                                 f[2 * p + 1].y * inv);
-        }
-        continue;
-      }
-
-      // ---- token maximum and ||S_hat||_2^2 over the group
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(d * kCols);
       float mx = 0.0f, sq = 0.0f;
+      uint32_t cm[4] = {0u, 0u, 0u, 0u};   // candidate bits (kInt4)
+      {
+        float2 f[64];
+        if (rowv) {
 #pragma unroll
-      for (int p = 0; p < 64; ++p) {
-        mx = fmax3(mx, fabsf(f[p].x), fabsf(f[p].y));
-        sq = fmaf(f[p].x, f[p].x, fmaf(f[p].y, f[p].y, sq));
-      }
-      const float own_mx = mx;
-      mx = warp_max(mx);
+          for (int c = 0; c < 4; ++c)
+            tmem_ld32(taddr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(
+                                          reinterpret_cast<uint32_t*>(f) + 32 * c));
+          tmem_wait_ld();
+        } else {
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
-      group_sync(g);                           // the previous token's scratch reads are done
-      if (lane == 0) {
-        S.wmax[q] = mx;
-        S.wsq[q] = sq;
-      }
-      group_sync(g);
-      const float M = fmaxf(fmaxf(S.wmax[0], S.wmax[1]), fmaxf(S.wmax[2], S.wmax[3]));
-      const float Q = (S.wsq[0] + S.wsq[1]) + (S.wsq[2] + S.wsq[3]);
-      const bool finite = isfinite(M) && isfinite(Q);
-      // fp32 sums of 12288 squares err by far less than 2^-10 relative
-      const double E = kBoundC * sqrt((double)Q * (1.0 + 0x1p-10));
-      const float thr = __double2float_rd((double)M - 2.0 * E);
+          for (int p = 0; p < 64; ++p) f[p] = make_float2(0.0f, 0.0f);
+        }
+        h128(f);
 
-      // ---- candidates: every output within 2E of the maximum, ranked
-      uint32_t cm[4] = {0u, 0u, 0u, 0u};
-      if (rowv && finite && M > 0.0f && own_mx >= thr) {
+        if (kMode == kRot) {
+          tc_fence_before();
+          mbar_arrive(&tempty[d]);
+          if (ok && rowv) {
+            const float inv = (float)(1.0 / P.sqrt_n);
+            float4* dst = reinterpret_cast<float4*>(P.out + token * N + o * 128);
+#pragma unroll
+            for (int p = 0; p < 32; ++p)
+              dst[p] = make_float4(f[2 * p].x * inv, f[2 * p].y * inv, f[2 * p + 1].x * inv,
+                                   f[2 * p + 1].y * inv);
+          }
+          continue;
+        }
+
+        // ---- token maximum and ||S_hat||_2^2 over the group
 #pragma unroll
         for (int p = 0; p < 64; ++p) {
-          if (fabsf(f[p].x) >= thr) cm[p >> 4] |= 1u << (2 * (p & 15));
-          if (fabsf(f[p].y) >= thr) cm[p >> 4] |= 1u << (2 * (p & 15) + 1);
+          mx = fmax3(mx, fabsf(f[p].x), fabsf(f[p].y));
+          sq = fmaf(f[p].x, f[p].x, fmaf(f[p].y, f[p].y, sq));
+        }
+        const float own_mx = mx;
+        mx = warp_max(mx);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
+        if (lane == 0) {
+          S.wmax[q] = mx;
+          S.wsq[q] = sq;
+        }
+        if (o == 0) S.ncand = 0;
+        group_sync(g);
+        const float M = fmaxf(fmaxf(S.wmax[0], S.wmax[1]), fmaxf(S.wmax[2], S.wmax[3]));
+        const float Q = (S.wsq[0] + S.wsq[1]) + (S.wsq[2] + S.wsq[3]);
+        mx = M;
+        sq = Q;
+        // E rounded up (fp32 sums of 12288 squares err by far less than 2^-10)
+        const float E = __fmul_ru((float)kBoundC, __fsqrt_ru(__fmul_ru(Q, 1.0f + 0x1p-10f)));
+        const float thr = __fsub_rd(M, __fmul_ru(2.0f, E));
+        // ---- candidates: every output within 2E of the maximum
+        if (rowv && isfinite(M) && isfinite(Q) && M > 0.0f && own_mx >= thr) {
+#pragma unroll
+          for (int p = 0; p < 64; ++p) {
+            if (fabsf(f[p].x) >= thr) cm[p >> 4] |= 1u << (2 * (p & 15));
+            if (fabsf(f[p].y) >= thr) cm[p >> 4] |= 1u << (2 * (p & 15) + 1);
+          }
+        }
+        // park S_hat in the accumulator while the registers serve the fix-ups
+        if (rowv) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            tmem_st32(taddr + c * 32, *reinterpret_cast<const uint32_t(*)[32]>(
+                                          reinterpret_cast<const uint32_t*>(f) + 32 * c));
         }
       }
+      const float M = mx, Q = sq;
+      const bool finite = isfinite(M) && isfinite(Q);
       const int myc = __popc(cm[0]) + __popc(cm[1]) + __popc(cm[2]) + __popc(cm[3]);
-      int incl = myc;
+      if (myc > 0) {
+        int slot = atomicAdd(&S.ncand, myc);
 #pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += v;
+        for (int w = 0; w < 4; ++w) {
+          uint32_t bits = cm[w];
+          while (bits) {
+            const int b = __ffs(bits) - 1;
+            bits &= bits - 1;
+            if (slot < kMaxCand) S.cand[slot] = o * 128 + w * 32 + b;
+            ++slot;
+          }
+        }
       }
-      if (lane == 31) S.wcnt[q] = incl;
       group_sync(g);
-      int base = 0, total = 0;
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        base += (w < q) ? S.wcnt[w] : 0;
-        total += S.wcnt[w];
-      }
-      const int rank0 = base + incl - myc;
+      const int total = S.ncand;
 
-      // ---- exact maximum over the candidates, kMaxCand at a time
+      // ---- exact maximum over the candidates
       double best = 0.0;
       const uint8_t* tok = sB + st * kStageBytes;   // held until the fix-ups are done
       if (total > 0) wait(&ready[st], (uint32_t)(k / kStages) & 1);   // sign flips visible
-      for (int r0 = 0; r0 < total; r0 += kMaxCand) {
-        if (myc > 0 && rank0 < r0 + kMaxCand && rank0 + myc > r0) {
-          int rk = rank0;
+      if (total <= kMaxCand) {
+        for (int c = 0; c < total; ++c) {
+          double part = warp_sum_d(exact_partial(tok, S.cand[c], o));
+          if (lane == 0) S.part[c & 1][q] = part;
+          group_sync(g);
+          best = fmax(best, fabs((S.part[c & 1][0] + S.part[c & 1][1]) +
+                                 (S.part[c & 1][2] + S.part[c & 1][3])));
+        }
+      } else {
+        // many candidates (degenerate rows): rank them and take kMaxCand at a time
+        int incl = myc;
 #pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            uint32_t bits = cm[w];
-            while (bits) {
-              const int b = __ffs(bits) - 1;
-              bits &= bits - 1;
-              if (rk >= r0 && rk < r0 + kMaxCand) S.cand[rk - r0] = o * 128 + w * 32 + b;
-              ++rk;
+        for (int off = 1; off < 32; off <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, off);
+          if (lane >= off) incl += v;
+        }
+        if (lane == 31) S.wcnt[q] = incl;
+        group_sync(g);
+        int base = 0;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) base += (w < q) ? S.wcnt[w] : 0;
+        const int rank0 = base + incl - myc;
+        for (int r0 = 0; r0 < total; r0 += kMaxCand) {
+          group_sync(g);                        // the previous round's reads are done
+          if (myc > 0 && rank0 < r0 + kMaxCand && rank0 + myc > r0) {
+            int rk = rank0;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              uint32_t bits = cm[w];
+              while (bits) {
+                const int b = __ffs(bits) - 1;
+                bits &= bits - 1;
+                if (rk >= r0 && rk < r0 + kMaxCand) S.cand[rk - r0] = o * 128 + w * 32 + b;
+                ++rk;
+              }
             }
           }
-        }
-        group_sync(g);
-        const int nc = min(kMaxCand, total - r0);
-        for (int c = 0; c < nc; ++c) {
-          const int i = S.cand[c];
-          double part = exact_partial(tok, i, o);
-          part = warp_sum_d(part);
-          if (lane == 0) S.part[q] = part;
           group_sync(g);
-          best = fmax(best, fabs((S.part[0] + S.part[1]) + (S.part[2] + S.part[3])));
-          group_sync(g);
+          const int nc = min(kMaxCand, total - r0);
+          for (int c = 0; c < nc; ++c) {
+            double part = warp_sum_d(exact_partial(tok, S.cand[c], o));
+            if (lane == 0) S.part[c & 1][q] = part;
+            group_sync(g);
+            best = fmax(best, fabs((S.part[c & 1][0] + S.part[c & 1][1]) +
+                                   (S.part[c & 1][2] + S.part[c & 1][3])));
+          }
         }
       }
-
       if (o == 0) mbar_arrive(&empty[st]);   // every read of the stage is behind a group sync
 
       // ---- scale and codes: 64 bytes per row thread.  A row holding an
@@ -473,15 +504,24 @@ k_tc12288(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ s
       if (!finite) best = (double)M;
       const float scale = (M > 0.0f || !finite) ? __double2float_rn((best / P.sqrt_n) / 7.0)
                                                 : 0.0f;
-      if (ok && rowv) {
+      if (rowv) {
+        tmem_wait_st();
         const float cq = scale > 0.0f ? __double2float_rn(1.0 / (P.sqrt_n * (double)scale)) : 0.0f;
         const float2 c2 = make_float2(cq, cq);
         uint4* dst = reinterpret_cast<uint4*>(P.codes + token * (N / 2) + o * 64);
 #pragma unroll
-        for (int w = 0; w < 4; ++w)
-          dst[w] = make_uint4(int4x8(f + 16 * w, c2), int4x8(f + 16 * w + 4, c2),
-                              int4x8(f + 16 * w + 8, c2), int4x8(f + 16 * w + 12, c2));
+        for (int c = 0; c < 4; ++c) {
+          float2 f[16];
+          tmem_ld32(taddr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(
+                                        reinterpret_cast<uint32_t*>(f)));
+          tmem_wait_ld();
+          if (ok)
+            dst[c] = make_uint4(int4x8(f, c2), int4x8(f + 4, c2), int4x8(f + 8, c2),
+                                int4x8(f + 12, c2));
+        }
       }
+      tc_fence_before();
+      mbar_arrive(&tempty[d]);
       if (ok && o == 0) P.scales[token] = scale;
     }
   }
@@ -501,7 +541,7 @@ k_tc12288(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ s
 namespace {
 
 constexpr size_t kTcpSmem = 1024 + 32768 + tcp::kStages * tcp::kStageBytes +
-                            tcp::kChunks * 16 + 2 * sizeof(tcp::GroupScratch) + 256;
+                            tcp::kChunks * 16 + 4 * sizeof(tcp::GroupScratch) + 256;
 
 template <int kMode>
 cudaError_t launch_tcp(const void* x, const int8_t* signs, tcp::Params& P, const Geometry& g,
