@@ -37,11 +37,11 @@
 // bounds by a 2^-4 relative margin).  Block scales that E leaves undecided are
 // recomputed exactly (fp64) from the input row in global memory.
 //
-// Warp roles (19 warps): 0 TMA producer, 1 MMA issuer + TMEM owner, 2-9 sign
+// Warp roles (20 warps): 0 TMA producer, 1 MMA issuer + TMEM owner, 2-9 sign
 // flip and error bound (two per token of a tile), 10-17 epilogue (two groups
-// of four warps; warp w reads TMEM lane quarter w % 4), 18 fix-up: blocks
+// of four warps; warp w reads TMEM lane quarter w % 4), 18-19 fix-up: blocks
 // whose scale the bound leaves undecided are stored provisionally by the
-// epilogue and queued (shared memory); the fix-up warp decides them exactly
+// epilogue and queued (shared memory); the fix-up warps decide them exactly
 // and rewrites their scale and codes.  A shared-memory stage
 // is recycled as soon as the MMAs have read it (tcgen05.commit); the tile's
 // error bounds travel with its accumulator.  Every wait on an mbarrier is
@@ -71,8 +71,9 @@ constexpr int kAccCols = 32 * kTok;            // fp32 columns per accumulator
 constexpr int kTmemCols = kAcc * kAccCols;     // power of two >= 32
 constexpr int kSignWarps = 2 * kTok;           // two per token
 constexpr int kEpiWarps = 4 * kGroups;
-constexpr int kFixWarp = 2 + kSignWarps + kEpiWarps;   // finishes undecided blocks
-constexpr int kThreads = 32 * (kFixWarp + 1);
+constexpr int kFixWarp = 2 + kSignWarps + kEpiWarps;   // first of the fix-up warps
+constexpr int kFixWarps = 2;                   // finish undecided blocks
+constexpr int kThreads = 32 * (kFixWarp + kFixWarps);
 constexpr int kQ = 32;                         // fix-up queue entries
 static_assert(kAcc % kGroups == 0 && (kTmemCols & (kTmemCols - 1)) == 0 && kTmemCols <= 512,
               "accumulators: a multiple of the groups, a power-of-two column count <= 512");
@@ -133,7 +134,7 @@ __device__ __noinline__ double warp_exact_S(const uint4* __restrict__ row,
     em[w] = ((uint32_t)(__popc(ilo & (2 * w)) & 1) << 15) |
             ((uint32_t)(__popc(ilo & (2 * w + 1)) & 1) << 31);
   double acc[4] = {0.0, 0.0, 0.0, 0.0};
-#pragma unroll 8
+#pragma unroll
   for (int k = 0; k < 16; ++k) {
     const int idx = lane + 32 * k;            // chunk (a, c)
     const int a = idx >> 2, c = idx & 3;
@@ -179,8 +180,8 @@ struct FixEntry {
 struct FixQueue {
   FixEntry e[kQ];
   unsigned int seq[kQ];   // slot k holds entry h when seq[k] == h + 1
+  unsigned int cons[kQ];  // slot k's entry h is finished when cons[k] == h + 1
   unsigned int tail;      // entries reserved by the epilogue
-  unsigned int head;      // entries finished by the fix-up warp
   unsigned int done;      // epilogue warps that will enqueue nothing more
 };
 
@@ -255,7 +256,6 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
       mbar_init(&tempty[d], 128);
     }
     fq->tail = 0;
-    fq->head = 0;
     fq->done = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     prefilled = my_tiles < kStages ? my_tiles : kStages;
@@ -292,7 +292,10 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
     }
     smask[i] = m4;
   }
-  for (int i = threadIdx.x; i < kQ; i += blockDim.x) fq->seq[i] = 0;
+  for (int i = threadIdx.x; i < kQ; i += blockDim.x) {
+    fq->seq[i] = 0;
+    fq->cons[i] = 0;
+  }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                  :: "r"(smem_u32(tmem_slot)), "n"(kTmemCols));
@@ -593,8 +596,8 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
           if (!((undecided >> j) & 1u)) continue;
           const unsigned int slot = atomicAdd(&fq->tail, 1u);
           const long long t0 = clock64();
-          bool room = true;
-          while (slot - ld_acquire(&fq->head) >= (unsigned int)kQ) {
+          bool room = true;   // the slot's previous entry (slot - kQ) is finished
+          while (slot >= (unsigned int)kQ && ld_acquire(&fq->cons[slot % kQ]) != slot - kQ + 1) {
             if (clock64() - t0 > kWaitCycles) { room = false; break; }
             __nanosleep(64);
           }
@@ -620,8 +623,9 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
     __syncwarp();
     __threadfence_block();
     if (lane == 0) atomicAdd(&fq->done, 1u);
-  } else if (warp == kFixWarp) {
-    // ================= fix-up warp: exact scales of the queued blocks
+  } else {
+    // ================= fix-up warps: exact scales of the queued blocks; fix-up
+    // warp f takes entries f, f + kFixWarps, ...
     if (kMode == kNvfp4) {
       float ts = 0.0f, inv_bt = 0.0f;
       if (P.ws) {
@@ -631,7 +635,7 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
         ts = *P.tensor_scale;
       }
       inv_bt = (ts > 0.0f) ? (float)(1.0 / (kSqrtN * (double)ts)) : 0.0f;
-      unsigned int h = 0;
+      unsigned int h = (unsigned int)(warp - kFixWarp);
       long long idle0 = clock64();
       for (;;) {
         if (ld_acquire(&fq->seq[h % kQ]) == h + 1) {
@@ -659,12 +663,12 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
             P.scales8[token * (N / 16) + blk] = (uint8_t)code;
           }
           __syncwarp();
-          if (lane == 0) st_release(&fq->head, h + 1);
-          ++h;
+          if (lane == 0) st_release(&fq->cons[h % kQ], h + 1);
+          h += kFixWarps;
           idle0 = clock64();
           continue;
         }
-        if (ld_acquire(&fq->done) == (unsigned int)kEpiWarps && ld_acquire(&fq->tail) == h) break;
+        if (ld_acquire(&fq->done) == (unsigned int)kEpiWarps && ld_acquire(&fq->tail) <= h) break;
         if (clock64() - idle0 > kWaitCycles) {
           atomicOr(&g_tc_error, 4u);
           break;
