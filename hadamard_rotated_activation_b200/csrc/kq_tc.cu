@@ -186,12 +186,14 @@ struct FixQueue {
 };
 
 // E2M1 codes of one 16-element block (v: 8 pairs) for the E4M3 scale `code`:
-// two words, element k in bits 4k..4k+3.  A zero scale (or tensor scale)
-// leaves only the signs.
+// two words, element k in bits 4k..4k+3.  rcp[c] = 1 / value of E4M3 code c
+// (a shared-memory table).  A zero scale (or tensor scale) leaves only the
+// signs.
 __device__ __forceinline__ void nvfp4_block_words(const float2* v, uint32_t code, float inv_bt,
-                                                  float ts, uint32_t& w0, uint32_t& w1) {
+                                                  float ts, const float* rcp, uint32_t& w0,
+                                                  uint32_t& w1) {
   if (code != 0 && ts > 0.0f) {
-    const float cs = inv_bt * e4m3_recip(code);
+    const float cs = inv_bt * rcp[code];
     const float2 c2 = make_float2(cs, cs), zero2 = make_float2(0.0f, 0.0f);
     float qv[16];
 #pragma unroll
@@ -237,6 +239,7 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
   uint64_t* tempty = tfull + kAcc;                      // accumulator read (kAcc)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + kAcc);
   FixQueue* fq = reinterpret_cast<FixQueue*>(bars + 64);   // after the 512-byte barrier area
+  float* srcp = reinterpret_cast<float*>(fq + 1);          // 1 / E4M3 value, 128 codes
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -296,6 +299,9 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
     fq->seq[i] = 0;
     fq->cons[i] = 0;
   }
+  // codes 1..126 (0 takes the sign-only path; 127 is NaN and never produced)
+  for (int i = threadIdx.x; i < 128; i += blockDim.x)
+    srcp[i] = (i >= 1 && i <= 126) ? 1.0f / e4m3_decode((uint32_t)i) : 0.0f;
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                  :: "r"(smem_u32(tmem_slot)), "n"(kTmemCols));
@@ -584,8 +590,8 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
 
         // ---- codes: 16 bytes per lane, contiguous across the warp
         uint32_t words[4];
-        nvfp4_block_words(v, sc & 0xffu, inv_bt, ts, words[0], words[1]);
-        nvfp4_block_words(v + 8, sc >> 8, inv_bt, ts, words[2], words[3]);
+        nvfp4_block_words(v, sc & 0xffu, inv_bt, ts, srcp, words[0], words[1]);
+        nvfp4_block_words(v + 8, sc >> 8, inv_bt, ts, srcp, words[2], words[3]);
         if (valid) {
           *reinterpret_cast<uint4*>(P.codes + token * (N / 2) + o * 16) =
               make_uint4(words[0], words[1], words[2], words[3]);
@@ -658,7 +664,8 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
           const uint32_t code = e4m3_pair(rr, rr) & 0xffu;
           if (lane == 0) {
             uint32_t w0, w1;
-            nvfp4_block_words(reinterpret_cast<const float2*>(fe.v), code, inv_bt, ts, w0, w1);
+            nvfp4_block_words(reinterpret_cast<const float2*>(fe.v), code, inv_bt, ts, srcp, w0,
+                              w1);
             *reinterpret_cast<uint2*>(P.codes + token * (N / 2) + blk * 8) = make_uint2(w0, w1);
             P.scales8[token * (N / 16) + blk] = (uint8_t)code;
           }
@@ -783,7 +790,7 @@ bool make_tmap(CUtensorMap* map, const void* x, int64_t rows) {
 }
 
 constexpr size_t kSmemBytes = 1024 + 32768 + tc::kStages * tc::kStageBytes + 512 * 16 +
-                              tc::kBoundFloats * 4 + 512 + sizeof(tc::FixQueue);
+                              tc::kBoundFloats * 4 + 512 + sizeof(tc::FixQueue) + 128 * 4;
 
 template <int kMode>
 cudaError_t launch_tc(const void* x, const int8_t* signs, tc::Params& P, cudaStream_t s) {
