@@ -502,6 +502,7 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
       c6 = (ts > 0.0f) ? (float)(1.0 / (kSqrtN * 6.0 * (double)ts)) : 0.0f;
       inv_bt = (ts > 0.0f) ? (float)(1.0 / (kSqrtN * (double)ts)) : 0.0f;
     }
+    float lower = 0.0f;                       // kNvStats: max over tokens of (max - E)
     for (int64_t k = g; k < my_tiles; k += kGroups) {
       const int d = (int)(k % kAcc);
       const int64_t tile = blockIdx.x + k * gridDim.x;
@@ -570,7 +571,7 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
           if (valid && lane == 0) {   // four warps per token: max through atomics
             atomicMax(reinterpret_cast<unsigned int*>(&P.ws->rows[token].x), __float_as_uint(mh));
             atomicMax(reinterpret_cast<unsigned int*>(&P.ws->rows[token].y), __float_as_uint(E));
-            atomicMax(&P.ws->lower_bits, __float_as_uint(fmaxf(__fsub_rd(mh, E), 0.0f)));
+            lower = fmaxf(lower, __fsub_rd(mh, E));   // one global atomic per warp, at the end
           }
           continue;
         }
@@ -626,6 +627,8 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
         }
       }
     }
+    if (kMode == kNvStats && lane == 0 && lower > 0.0f)
+      atomicMax(&P.ws->lower_bits, __float_as_uint(lower));
     __syncwarp();
     __threadfence_block();
     if (lane == 0) atomicAdd(&fq->done, 1u);
