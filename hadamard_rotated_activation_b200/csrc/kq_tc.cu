@@ -43,8 +43,9 @@
 // whose scale the bound leaves undecided are stored provisionally by the
 // epilogue and queued (shared memory); the fix-up warps decide them exactly
 // and rewrites their scale and codes.  A shared-memory stage
-// is recycled as soon as the MMAs have read it (tcgen05.commit); the tile's
-// error bounds travel with its accumulator.  Every wait on an mbarrier is
+// is recycled as soon as the MMAs have read it (tcgen05.commit); the sign warps
+// release a tile to the MMA right after flipping it and pass its error bounds
+// to the epilogue through a ring of slots.  Every wait on an mbarrier is
 // bounded; on timeout the kernel records an error code and returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -77,8 +78,14 @@ constexpr int kThreads = 32 * (kFixWarp + kFixWarps);
 constexpr int kQ = 32;                         // fix-up queue entries
 static_assert(kAcc % kGroups == 0 && (kTmemCols & (kTmemCols - 1)) == 0 && kTmemCols <= 512,
               "accumulators: a multiple of the groups, a power-of-two column count <= 512");
-static_assert((3 * kStages + 2 * kAcc) * 8 + 4 <= 512, "barrier area");
-constexpr int kBoundFloats = (kStages + kAcc) * kTok * 2;   // sE + sEacc
+static_assert((3 * kStages + 2 * kAcc + 16) * 8 + 4 <= 512, "barrier area");
+// Error bounds of tile k live in ring slot k % kBRing until its epilogue has
+// read them: the sign warps can reach tile k + kBRing only after the MMA of
+// tile k + kBRing - kStages, which follows the MMA of tile k + kAcc, which
+// waits for tile k's accumulator (and bounds) to be consumed.
+constexpr int kBRing = 16;
+static_assert(kBRing >= kStages + kAcc, "bound ring too short");
+constexpr int kBoundFloats = kBRing * kTok * 2;
 
 __device__ unsigned int g_tc_error = 0;        // nonzero: a wait timed out
 
@@ -229,15 +236,15 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
   uint8_t* sA = smem;                                   // 32 KB: A = H_128
   uint8_t* sB = smem + 32768;                           // kStages x 32 KB
   uint4* smask = reinterpret_cast<uint4*>(sB + kStages * kStageBytes);   // 512 chunks
-  float* sE = reinterpret_cast<float*>(smask + 512);   // error bound halves per (stage, token)
-  float* sEacc = sE + kStages * kTok * 2;              // the same, handed to the epilogue per accumulator
+  float* sE = reinterpret_cast<float*>(smask + 512);   // bound halves per (ring slot, token)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sE + kBoundFloats);
   uint64_t* full = bars;                                // TMA landed
-  uint64_t* ready = bars + kStages;                     // signs applied, bounds written
+  uint64_t* ready = bars + kStages;                     // signs applied
   uint64_t* empty = bars + 2 * kStages;                 // MMAs done reading the stage
-  uint64_t* tfull = bars + 3 * kStages;                 // accumulator written + bounds (kAcc)
+  uint64_t* tfull = bars + 3 * kStages;                 // accumulator written (kAcc)
   uint64_t* tempty = tfull + kAcc;                      // accumulator read (kAcc)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + kAcc);
+  uint64_t* bready = tempty + kAcc;                     // bounds written (kBRing)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bready + kBRing);
   FixQueue* fq = reinterpret_cast<FixQueue*>(bars + 64);   // after the 512-byte barrier area
   float* srcp = reinterpret_cast<float*>(fq + 1);          // 1 / E4M3 value, 128 codes
 
@@ -255,9 +262,10 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
       mbar_init(&empty[s], 1);
     }
     for (int d = 0; d < kAcc; ++d) {
-      mbar_init(&tfull[d], 2);
+      mbar_init(&tfull[d], 1);
       mbar_init(&tempty[d], 128);
     }
+    for (int j = 0; j < kBRing; ++j) mbar_init(&bready[j], kSignWarps);
     fq->tail = 0;
     fq->done = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -345,10 +353,6 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
         if (!mbar_wait(&ready[s], (uint32_t)(k / kStages) & 1)) break;
         if (k >= kAcc && !mbar_wait(&tempty[d], (uint32_t)(k / kAcc - 1) & 1)) break;
         tc_fence_after();
-        // the tile's error bounds move to the accumulator's slot: the stage
-        // is recycled as soon as the MMAs below have read it
-#pragma unroll
-        for (int e = 0; e < kTok * 2; ++e) sEacc[d * kTok * 2 + e] = sE[s * kTok * 2 + e];
         const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB + s * kStageBytes);
         const uint32_t tmem_d = tmem_base + (uint32_t)(d * kAccCols);
 #pragma unroll
@@ -362,7 +366,6 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
         }
         mma_commit(&empty[s]);
         mma_commit(&tfull[d]);
-        mbar_arrive(&tfull[d]);          // publishes sEacc[d] (release)
         issued = k + 1;
       }
       // the accumulators must not be released with MMAs still running
@@ -422,6 +425,10 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
           }
         }
       }
+      // the flipped tile goes to the tensor cores now; the bound follows
+      if (signs) fence_async_smem();
+      __syncwarp();
+      mbar_arrive(&ready[s]);
       // Each bf16 sum of 8 non-negative terms is at least (1 - 2^-8)^7 of the
       // exact sum (round to nearest), so x (1 + 2^-4) bounds it from above,
       // with room for the fp32 additions below.
@@ -478,11 +485,9 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
         const float e1 = __fmul_ru(__fadd_ru(__fmul_ru(2.5f, W), __fmul_ru(5.000002f, S)),
                                    0x1p-24f);
         const float e = __fmul_ru(__fadd_ru(e1, __fmul_ru(R, 0x1.0001p-21f)), 1.0f + 0x1p-10f);
-        sE[(s * kTok + t) * 2 + hc] = e;
+        sE[((int)(k % kBRing) * kTok + t) * 2 + hc] = e;
+        mbar_arrive(&bready[k % kBRing]);
       }
-      if (signs) fence_async_smem();
-      __syncwarp();
-      mbar_arrive(&ready[s]);
     }
   } else if (warp < kFixWarp) {
     // ================= epilogue: group g of warps 10+4g .. 13+4g
@@ -508,14 +513,16 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
       const int64_t tile = blockIdx.x + k * gridDim.x;
       // A timed-out wait does not leave the loop: the failure is recorded
       // (g_tc_error) and the tile's outputs are not written.
-      const bool ok = mbar_wait(&tfull[d], (uint32_t)(k / kAcc) & 1);
+      bool ok = mbar_wait(&tfull[d], (uint32_t)(k / kAcc) & 1);
       tc_fence_after();
+      const int rb = (int)(k % kBRing);
+      ok = mbar_wait(&bready[rb], (uint32_t)(k / kBRing) & 1) && ok;
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(d * kAccCols);
 #pragma unroll 1
       for (int t = 0; t < kTok; ++t) {
         // |S_hat - S| <= E for every output of the token; read before the
         // accumulator (and with it the bound slot) is handed back below
-        const float E = __fadd_ru(sEacc[(d * kTok + t) * 2], sEacc[(d * kTok + t) * 2 + 1]);
+        const float E = __fadd_ru(sE[(rb * kTok + t) * 2], sE[(rb * kTok + t) * 2 + 1]);
         float2 v[16];
         {
           uint32_t r[32];
