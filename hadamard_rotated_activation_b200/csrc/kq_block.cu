@@ -238,7 +238,13 @@ k_blk128_nvfp4(Params P) {
   extern __shared__ __align__(16) uint4 smem4[];
   uint4* stages = smem4 + (threadIdx.x >> 5) * 1024;      // two 8 KB stages per warp
   uint4* smask = P.signs ? smem4 + (blockDim.x >> 5) * 1024 : nullptr;
+  // 1 / value of E4M3 codes 1..126 (0 takes the sign-only path, 127 is NaN)
+  float* rcp = reinterpret_cast<float*>(smem4 + (blockDim.x >> 5) * 1024 +
+                                        (P.signs ? P.n / 8 : 0));
   if (smask) stage_signs(P.signs, P.n, smask);
+  if (kMode == 0)
+    for (int i = threadIdx.x; i < 128; i += blockDim.x)
+      rcp[i] = (i >= 1 && i <= 126) ? e4m3_recip((uint32_t)i) : 0.0f;
   __syncthreads();
   const int kpr = P.n / B;                  // column blocks per row (power of two)
   const int kpr_log2 = __ffs(kpr) - 1;
@@ -355,7 +361,7 @@ k_blk128_nvfp4(Params P) {
         const int j = 2 * k + jj;
         const uint32_t code = (sc[j >> 2] >> (8 * (j & 3))) & 0xffu;
         if (code != 0 && t > 0.0f) {
-          const float c = inv_bt * e4m3_recip(code);
+          const float c = inv_bt * rcp[code];
           const float2 c2 = make_float2(c, c);
           float q[16];
 #pragma unroll
@@ -527,7 +533,7 @@ k_blk128_asym(Params P) {
 // ------------------------------------------------------------- launchers
 namespace {
 size_t blk_smem(int n, bool signs) {
-  return (size_t)(blk::kThreads / 32) * 1024 * 16 + (signs ? (size_t)n / 8 * 16 : 0);
+  return (size_t)(blk::kThreads / 32) * 1024 * 16 + (signs ? (size_t)n / 8 * 16 : 0) + 128 * 4;
 }
 
 int blk_grid(const void* kernel, int64_t units, size_t smem) {
