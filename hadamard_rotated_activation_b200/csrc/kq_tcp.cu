@@ -13,9 +13,10 @@
 //       128 (bf16 +-1, K-major, built in shared memory once) and B = the
 //       sign-flipped token (K = a, N = beta; MN-major, 128-byte swizzle, two
 //       TMA boxes of 64 columns);
-//   (2) the H_128 over beta, run by the epilogue thread that owns TMEM lane o
-//       (o < 96): 128 columns in registers, seven butterfly stages in fp32.
-// That thread then holds the 128 contiguous outputs o*128 .. o*128+127.
+//   (2) the H_128 over beta, run by the two epilogue threads of TMEM lane o
+//       (o < 96): each reads all 128 columns, does the beta6 stage for its
+//       output half, then six butterfly stages in fp32 on 64 values; it then
+//       holds 64 contiguous outputs o*128 + oh*64 .. +63.
 //
 // Exact scale.  The per-token scale fp32(max|y| / 7), y = S / sqrt(n), needs
 // max|S| exactly.  With the accumulation model of tcgen05.mma (see the
@@ -29,11 +30,12 @@
 // the whole epilogue group from the staged token, which the epilogue holds
 // until then.
 //
-// Warp roles (12 warps, three per scheduler, so a thread may hold 168
-// registers): 0 TMA producer, 1 MMA issuer + TMEM owner, 2-3 sign flip, 4-7
-// and 8-11 two epilogue groups taking alternate tokens (warp w reads TMEM
-// lane quarter w % 4; quarter 3 holds the zero padding of A and only helps
-// with reductions and fix-ups).  Every wait is bounded; on timeout the kernel
+// Warp roles (20 warps): 0 TMA producer, 1 MMA issuer + TMEM owner, 2-3 sign
+// flip, 4-11 and 12-19 two epilogue groups taking alternate tokens.  In a
+// group, warp w reads TMEM lane quarter w % 4 (quarter 3 holds the zero
+// padding of A and only helps with reductions and fix-ups), and the two warps
+// of a quarter split the row's outputs into halves (beta6 = 0, 1), so a thread
+// holds 64 values.  Every wait is bounded; on timeout the kernel
 // records an error code and returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -59,13 +61,21 @@ constexpr uint32_t kStageBytes = 2 * kHalfBytes;   // one token, 24 KB
 constexpr int kStages = 5;
 constexpr int kAcc = 4;                            // TMEM accumulators (128 columns each)
 constexpr int kTmemCols = kAcc * kCols;
-constexpr int kSignWarps = 2;
-constexpr int kThreads = 32 * 12;
+// 20 warps: 0 TMA, 1 MMA; epilogue group g owns warps 4 + 8g .. 11 + 8g
+// except those in lane quarter 3 (A's zero padding), which flip signs with
+// warps 2 and 3.
+constexpr int kSignWarps = 6;
+constexpr int kGroupWarps = 6;                     // per epilogue group: 3 lane quarters x 2 halves
+constexpr int kGroupThreads = 32 * kGroupWarps;
+constexpr int kThreads = 32 * 20;
+__device__ __forceinline__ bool is_sign_warp(int w) { return w == 2 || w == 3 || (w >= 4 && (w & 3) == 3); }
+__device__ __forceinline__ int sign_index(int w) { return w < 4 ? w - 2 : 2 + (w - 7) / 4; }
 constexpr int kChunks = N / 8;                     // 16-byte chunks per token
 constexpr int kMaxCand = 32;                       // fix-up candidates handled per token
 constexpr double kBoundC = 72.0 * 0x1p-24;         // E = kBoundC ||S_hat||_2
-static_assert(kChunks % (32 * kSignWarps) == 0, "sign warps split the chunks evenly");
-static_assert(kChunks % 128 == 0, "an epilogue group splits the chunks evenly");
+static_assert(kChunks % (32 * kSignWarps) == 0 && (kChunks / 2) % (32 * kSignWarps) == 0,
+              "sign warps split the chunks (and each half) evenly");
+static_assert(kChunks % kGroupThreads == 0, "an epilogue group splits the chunks evenly");
 
 __device__ unsigned int g_tcp_error = 0;           // nonzero: a wait timed out
 
@@ -81,10 +91,10 @@ struct Params {
 
 // Per-group scratch for the token reductions.
 struct GroupScratch {
-  float wmax[4];
-  float wsq[4];
-  double part[2][4];     // per candidate parity
-  int wcnt[4];
+  float wmax[kGroupWarps];
+  float wsq[kGroupWarps];
+  double part[2][kGroupWarps];   // per candidate parity
+  int wcnt[kGroupWarps];
   int ncand;
   int cand[kMaxCand];
 };
@@ -93,7 +103,7 @@ __device__ __forceinline__ bool wait(uint64_t* bar, uint32_t parity) {
   return sm100::mbar_wait(bar, parity, &g_tcp_error);
 }
 __device__ __forceinline__ void group_sync(int g) {
-  asm volatile("bar.sync %0, 128;" :: "r"(1 + g) : "memory");
+  asm volatile("bar.sync %0, %1;" :: "r"(1 + g), "n"(kGroupThreads) : "memory");
 }
 
 // H_96[m][k] = H_12[m/8][k/8] (-1)^popc((m%8) & (k%8)), negative?
@@ -108,9 +118,9 @@ __device__ __forceinline__ uint32_t b_chunk(int a, int c16) {
   return (uint32_t)((c16 >> 3) * kHalfBytes + a * 128 + (((c16 & 7) ^ (a & 7)) << 4));
 }
 
-// Exact S_i (fp64) of a staged, sign-flipped token, computed by the 128
-// threads of an epilogue group: thread tau takes the 16-byte chunks tau,
-// tau + 128, ...; chunk ch holds x'[a*128 + c16*8 .. +7] (a = ch / 16, c16 =
+// Exact S_i (fp64) of a staged, sign-flipped token, computed by the
+// kGroupThreads threads of an epilogue group: thread tau takes the 16-byte
+// chunks tau, tau + kGroupThreads, ...; chunk ch holds x'[a*128 + c16*8 .. +7] (a = ch / 16, c16 =
 // ch % 16).  H[i][j] for i = o*128 + b, j = a*128 + c16*8 + e is H_96[o][a]
 // (-1)^(popc(b_hi & c16) + popc(b_lo & e)), b_hi = b / 8, b_lo = b % 8.
 // Values enter fp64 exactly through bf16x2_to_f64_scaled.  Returns this
@@ -124,8 +134,8 @@ __device__ __forceinline__ double exact_partial(const uint8_t* tok, int i, int t
             ((uint32_t)(__popc(blo & (2 * w + 1)) & 1) << 31);
   double acc[4] = {0.0, 0.0, 0.0, 0.0};
 #pragma unroll 2
-  for (int k = 0; k < kChunks / 128; ++k) {
-    const int ch = tau + 128 * k;
+  for (int k = 0; k < kChunks / kGroupThreads; ++k) {
+    const int ch = tau + kGroupThreads * k;
     const int a = ch >> 4, c16 = ch & 15;
     const uint32_t flip =
         (h96_negative(o, a) ^ (__popc(bhi & c16) & 1)) ? 0x80008000u : 0u;
@@ -142,18 +152,18 @@ __device__ __forceinline__ double exact_partial(const uint8_t* tok, int i, int t
   return ((acc[0] + acc[1]) + (acc[2] + acc[3])) * kF64Unscale;
 }
 
-// Seven butterfly stages (H_128, natural order) on f[0..63] (f[p] holds
+// Six butterfly stages (H_64, natural order) on f[0..31] (f[p] holds
 // elements 2p, 2p + 1) in place.
-__device__ __forceinline__ void h128(float2 (&f)[64]) {
+__device__ __forceinline__ void h64(float2 (&f)[32]) {
 #pragma unroll
-  for (int p = 0; p < 64; ++p) {
+  for (int p = 0; p < 32; ++p) {
     const float a = f[p].x, b = f[p].y;
     f[p] = make_float2(a + b, a - b);
   }
 #pragma unroll
-  for (int hh = 1; hh < 64; hh <<= 1)
+  for (int hh = 1; hh < 32; hh <<= 1)
 #pragma unroll
-    for (int p = 0; p < 64; ++p)
+    for (int p = 0; p < 32; ++p)
       if (!(p & hh)) bfly2(f[p], f[p | hh]);
 }
 
@@ -208,7 +218,7 @@ k_tc12288(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ s
     }
     for (int d = 0; d < kAcc; ++d) {
       mbar_init(&tfull[d], 1);
-      mbar_init(&tempty[d], 128);
+      mbar_init(&tempty[d], kGroupThreads);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     prefilled = my_tiles < kStages ? my_tiles : kStages;
@@ -304,20 +314,21 @@ k_tc12288(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ s
       for (int64_t k = issued > kAcc ? issued - kAcc : 0; k < issued; ++k)
         wait(&tfull[k % kAcc], (uint32_t)(k / kAcc) & 1);
     }
-  } else if (warp < 2 + kSignWarps) {
-    // ================= sign flip: lane l of sign warp w takes the physical
-    // chunks t0 + 64 i (conflict-free), i = 0..23: half i / 12, row a = t0 / 8 +
-    // 8 (i % 12), slot t0 % 8, which holds logical chunk (t0 % 8) ^ (a % 8) of
-    // the half.  The lane's 24 sign masks stay in registers.
-    const int t0 = (warp - 2) * 32 + lane;
-    constexpr int kPer = kChunks / 64;
+  } else if (is_sign_warp(warp)) {
+    // ================= sign flip: lane t0 of the sign warps takes the physical
+    // chunks t0 + 192 i (conflict-free), i = 0..7: half i / 4, row a = t0 / 8 +
+    // 24 (i % 4), slot t0 % 8, which holds logical chunk (t0 % 8) ^ (a % 8) of
+    // the half.  The lane's 8 sign masks stay in registers.
+    constexpr int kLanes = 32 * kSignWarps;
+    constexpr int kPer = kChunks / kLanes;
+    const int t0 = sign_index(warp) * 32 + lane;
     uint4 msk[kPer];
     {
       const int cl = (t0 & 7) ^ ((t0 >> 3) & 7);
 #pragma unroll
       for (int i = 0; i < kPer; ++i) {
-        const int a = (t0 >> 3) + 8 * (i % 12);
-        msk[i] = smask[a * 16 + (i / 12) * 8 + cl];
+        const int a = (t0 >> 3) + (kLanes / 8) * (i % (kPer / 2));
+        msk[i] = smask[a * 16 + (i / (kPer / 2)) * 8 + cl];
       }
     }
     for (int64_t k = 0; k < my_tiles; ++k) {
@@ -327,12 +338,12 @@ k_tc12288(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ s
         uint4* st = reinterpret_cast<uint4*>(sB + s * kStageBytes) + t0;
 #pragma unroll
         for (int i = 0; i < kPer; ++i) {
-          uint4 w = st[64 * i];
+          uint4 w = st[kLanes * i];
           w.x ^= msk[i].x;
           w.y ^= msk[i].y;
           w.z ^= msk[i].z;
           w.w ^= msk[i].w;
-          st[64 * i] = w;
+          st[kLanes * i] = w;
         }
         fence_async_smem();
       }
@@ -340,11 +351,19 @@ k_tc12288(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ s
       mbar_arrive(&ready[s]);
     }
   } else {
-    // ================= epilogue: group g of warps 4+4g .. 7+4g
-    const int g = (warp - 4) >> 2;
-    const int q = warp & 3;                   // TMEM lane quarter
-    const int o = q * 32 + lane;              // accumulator row = thread within group
-    const bool rowv = o < kRows;
+    // ================= epilogue: group g of warps 4+8g .. 11+8g.  Warp w
+    // reads TMEM lane quarter q = w % 4 (rows o = 32 q + lane); the first four
+    // warps of a group take output half oh = 0, the other four oh = 1.  The
+    // accumulator row o holds D0 (columns 0-63, beta6 = 0) and D1 (64-127);
+    // the beta6 stage gives S[o][oh][.] = D0 + D1 (oh = 0) or D0 - D1, then
+    // H_64 over the 64 low columns: outputs o*128 + oh*64 .. +63.
+    const int g = (warp - 4) >> 3;
+    const int q = warp & 3;                   // TMEM lane quarter (0..2)
+    const int oh = (warp >> 2) & 1 ? 0 : 1;   // output half (beta6 of the output)
+    const int o = q * 32 + lane;              // accumulator row
+    const int wg = oh * 3 + q;                // warp within the group
+    const int tau = wg * 32 + lane;           // thread within the group
+    const bool rowv = true;
     for (int64_t k = g; k < my_tiles; k += 2) {
       const int d = (int)(k % kAcc);
       const int st = (int)(k % kStages);
@@ -357,87 +376,95 @@ k_tc12288(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ s
       const bool ok = wait(&tfull[d], (uint32_t)(k / kAcc) & 1);
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(d * kCols);
-      float mx = 0.0f, sq = 0.0f;
-      uint32_t cm[4] = {0u, 0u, 0u, 0u};   // candidate bits (kInt4)
-      {
-        float2 f[64];
-        if (rowv) {
+      float2 f[32];
+      if (rowv) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
-            tmem_ld32(taddr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(
-                                          reinterpret_cast<uint32_t*>(f) + 32 * c));
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r0[16], r1[16];
+          tmem_ld16(taddr + c * 16, r0);
+          tmem_ld16(taddr + 64 + c * 16, r1);
           tmem_wait_ld();
-        } else {
 #pragma unroll
-          for (int p = 0; p < 64; ++p) f[p] = make_float2(0.0f, 0.0f);
-        }
-        h128(f);
-
-        if (kMode == kRot) {
-          tc_fence_before();
-          mbar_arrive(&tempty[d]);
-          if (ok && rowv) {
-            const float inv = (float)(1.0 / P.sqrt_n);
-            float4* dst = reinterpret_cast<float4*>(P.out + token * N + o * 128);
-#pragma unroll
-            for (int p = 0; p < 32; ++p)
-              dst[p] = make_float4(f[2 * p].x * inv, f[2 * p].y * inv, f[2 * p + 1].x * inv,
-                                   f[2 * p + 1].y * inv);
-          }
-          continue;
-        }
-
-        // ---- token maximum and ||S_hat||_2^2 over the group
-#pragma unroll
-        for (int p = 0; p < 64; ++p) {
-          mx = fmax3(mx, fabsf(f[p].x), fabsf(f[p].y));
-          sq = fmaf(f[p].x, f[p].x, fmaf(f[p].y, f[p].y, sq));
-        }
-        const float own_mx = mx;
-        mx = warp_max(mx);
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
-        if (lane == 0) {
-          S.wmax[q] = mx;
-          S.wsq[q] = sq;
-        }
-        if (o == 0) S.ncand = 0;
-        group_sync(g);
-        const float M = fmaxf(fmaxf(S.wmax[0], S.wmax[1]), fmaxf(S.wmax[2], S.wmax[3]));
-        const float Q = (S.wsq[0] + S.wsq[1]) + (S.wsq[2] + S.wsq[3]);
-        mx = M;
-        sq = Q;
-        // E rounded up (fp32 sums of 12288 squares err by far less than 2^-10)
-        const float E = __fmul_ru((float)kBoundC, __fsqrt_ru(__fmul_ru(Q, 1.0f + 0x1p-10f)));
-        const float thr = __fsub_rd(M, __fmul_ru(2.0f, E));
-        // ---- candidates: every output within 2E of the maximum
-        if (rowv && isfinite(M) && isfinite(Q) && M > 0.0f && own_mx >= thr) {
-#pragma unroll
-          for (int p = 0; p < 64; ++p) {
-            if (fabsf(f[p].x) >= thr) cm[p >> 4] |= 1u << (2 * (p & 15));
-            if (fabsf(f[p].y) >= thr) cm[p >> 4] |= 1u << (2 * (p & 15) + 1);
+          for (int e = 0; e < 8; ++e) {
+            const float a0 = __uint_as_float(r0[2 * e]), a1 = __uint_as_float(r0[2 * e + 1]);
+            const float b0 = __uint_as_float(r1[2 * e]), b1 = __uint_as_float(r1[2 * e + 1]);
+            f[8 * c + e] = oh ? make_float2(a0 - b0, a1 - b1) : make_float2(a0 + b0, a1 + b1);
           }
         }
-        // park S_hat in the accumulator while the registers serve the fix-ups
-        if (rowv) {
+      } else {
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
-            tmem_st32(taddr + c * 32, *reinterpret_cast<const uint32_t(*)[32]>(
-                                          reinterpret_cast<const uint32_t*>(f) + 32 * c));
+        for (int p = 0; p < 32; ++p) f[p] = make_float2(0.0f, 0.0f);
+      }
+      h64(f);
+
+      if (kMode == kRot) {
+        tc_fence_before();
+        mbar_arrive(&tempty[d]);
+        if (ok && rowv) {
+          const float inv = (float)(1.0 / P.sqrt_n);
+          float4* dst = reinterpret_cast<float4*>(P.out + token * N + o * 128 + oh * 64);
+#pragma unroll
+          for (int p = 0; p < 16; ++p)
+            dst[p] = make_float4(f[2 * p].x * inv, f[2 * p].y * inv, f[2 * p + 1].x * inv,
+                                 f[2 * p + 1].y * inv);
+        }
+        continue;
+      }
+
+      // ---- token maximum and ||S_hat||_2^2 over the group
+      float mx = 0.0f, sq = 0.0f;
+#pragma unroll
+      for (int p = 0; p < 32; ++p) {
+        mx = fmax3(mx, fabsf(f[p].x), fabsf(f[p].y));
+        sq = fmaf(f[p].x, f[p].x, fmaf(f[p].y, f[p].y, sq));
+      }
+      const float own_mx = mx;
+      mx = warp_max(mx);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
+      if (lane == 0) {
+        S.wmax[wg] = mx;
+        S.wsq[wg] = sq;
+      }
+      if (tau == 0) S.ncand = 0;
+      group_sync(g);                           // also: every thread has read D0 and D1
+      float M = 0.0f, Q = 0.0f;
+#pragma unroll
+      for (int w = 0; w < kGroupWarps; ++w) {
+        M = fmaxf(M, S.wmax[w]);
+        Q += S.wsq[w];
+      }
+      const bool finite = isfinite(M) && isfinite(Q);
+      // E rounded up (fp32 sums of 12288 squares err by far less than 2^-10)
+      const float E = __fmul_ru((float)kBoundC, __fsqrt_ru(__fmul_ru(Q, 1.0f + 0x1p-10f)));
+      const float thr = __fsub_rd(M, __fmul_ru(2.0f, E));
+      // ---- candidates: every output within 2E of the maximum
+      uint32_t cm[2] = {0u, 0u};
+      if (rowv && finite && M > 0.0f && own_mx >= thr) {
+#pragma unroll
+        for (int p = 0; p < 32; ++p) {
+          if (fabsf(f[p].x) >= thr) cm[p >> 4] |= 1u << (2 * (p & 15));
+          if (fabsf(f[p].y) >= thr) cm[p >> 4] |= 1u << (2 * (p & 15) + 1);
         }
       }
-      const float M = mx, Q = sq;
-      const bool finite = isfinite(M) && isfinite(Q);
-      const int myc = __popc(cm[0]) + __popc(cm[1]) + __popc(cm[2]) + __popc(cm[3]);
+      // park S_hat in this thread's half of the accumulator row while the
+      // registers serve the fix-ups (both halves were read before the sync)
+      if (rowv) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+          tmem_st32(taddr + oh * 64 + c * 32, *reinterpret_cast<const uint32_t(*)[32]>(
+                                                  reinterpret_cast<const uint32_t*>(f) + 32 * c));
+      }
+      const int myc = __popc(cm[0]) + __popc(cm[1]);
       if (myc > 0) {
         int slot = atomicAdd(&S.ncand, myc);
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
+        for (int w = 0; w < 2; ++w) {
           uint32_t bits = cm[w];
           while (bits) {
             const int b = __ffs(bits) - 1;
             bits &= bits - 1;
-            if (slot < kMaxCand) S.cand[slot] = o * 128 + w * 32 + b;
+            if (slot < kMaxCand) S.cand[slot] = o * 128 + oh * 64 + w * 32 + b;
             ++slot;
           }
         }
@@ -451,11 +478,13 @@ k_tc12288(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ s
       if (total > 0) wait(&ready[st], (uint32_t)(k / kStages) & 1);   // sign flips visible
       if (total <= kMaxCand) {
         for (int c = 0; c < total; ++c) {
-          double part = warp_sum_d(exact_partial(tok, S.cand[c], o));
-          if (lane == 0) S.part[c & 1][q] = part;
+          double part = warp_sum_d(exact_partial(tok, S.cand[c], tau));
+          if (lane == 0) S.part[c & 1][wg] = part;
           group_sync(g);
-          best = fmax(best, fabs((S.part[c & 1][0] + S.part[c & 1][1]) +
-                                 (S.part[c & 1][2] + S.part[c & 1][3])));
+          double sum = 0.0;
+#pragma unroll
+          for (int w = 0; w < kGroupWarps; ++w) sum += S.part[c & 1][w];
+          best = fmax(best, fabs(sum));
         }
       } else {
         // many candidates (degenerate rows): rank them and take kMaxCand at a time
@@ -465,23 +494,24 @@ k_tc12288(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ s
           const int v = __shfl_up_sync(0xffffffffu, incl, off);
           if (lane >= off) incl += v;
         }
-        if (lane == 31) S.wcnt[q] = incl;
+        if (lane == 31) S.wcnt[wg] = incl;
         group_sync(g);
         int base = 0;
 #pragma unroll
-        for (int w = 0; w < 4; ++w) base += (w < q) ? S.wcnt[w] : 0;
+        for (int w = 0; w < kGroupWarps; ++w) base += (w < wg) ? S.wcnt[w] : 0;
         const int rank0 = base + incl - myc;
         for (int r0 = 0; r0 < total; r0 += kMaxCand) {
           group_sync(g);                        // the previous round's reads are done
           if (myc > 0 && rank0 < r0 + kMaxCand && rank0 + myc > r0) {
             int rk = rank0;
 #pragma unroll
-            for (int w = 0; w < 4; ++w) {
+            for (int w = 0; w < 2; ++w) {
               uint32_t bits = cm[w];
               while (bits) {
                 const int b = __ffs(bits) - 1;
                 bits &= bits - 1;
-                if (rk >= r0 && rk < r0 + kMaxCand) S.cand[rk - r0] = o * 128 + w * 32 + b;
+                if (rk >= r0 && rk < r0 + kMaxCand)
+                  S.cand[rk - r0] = o * 128 + oh * 64 + w * 32 + b;
                 ++rk;
               }
             }
@@ -489,17 +519,19 @@ k_tc12288(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ s
           group_sync(g);
           const int nc = min(kMaxCand, total - r0);
           for (int c = 0; c < nc; ++c) {
-            double part = warp_sum_d(exact_partial(tok, S.cand[c], o));
-            if (lane == 0) S.part[c & 1][q] = part;
+            double part = warp_sum_d(exact_partial(tok, S.cand[c], tau));
+            if (lane == 0) S.part[c & 1][wg] = part;
             group_sync(g);
-            best = fmax(best, fabs((S.part[c & 1][0] + S.part[c & 1][1]) +
-                                   (S.part[c & 1][2] + S.part[c & 1][3])));
+            double sum = 0.0;
+#pragma unroll
+            for (int w = 0; w < kGroupWarps; ++w) sum += S.part[c & 1][w];
+            best = fmax(best, fabs(sum));
           }
         }
       }
-      if (o == 0) mbar_arrive(&empty[st]);   // every read of the stage is behind a group sync
+      if (tau == 0) mbar_arrive(&empty[st]);   // every read of the stage is behind a group sync
 
-      // ---- scale and codes: 64 bytes per row thread.  A row holding an
+      // ---- scale and codes: 32 bytes per row thread.  A row holding an
       // infinity or NaN gets the scale of its computed maximum (not exact).
       if (!finite) best = (double)M;
       const float scale = (M > 0.0f || !finite) ? __double2float_rn((best / P.sqrt_n) / 7.0)
@@ -508,21 +540,21 @@ k_tc12288(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ s
         tmem_wait_st();
         const float cq = scale > 0.0f ? __double2float_rn(1.0 / (P.sqrt_n * (double)scale)) : 0.0f;
         const float2 c2 = make_float2(cq, cq);
-        uint4* dst = reinterpret_cast<uint4*>(P.codes + token * (N / 2) + o * 64);
+        uint4* dst = reinterpret_cast<uint4*>(P.codes + token * (N / 2) + o * 64 + oh * 32);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float2 f[16];
-          tmem_ld32(taddr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(
-                                        reinterpret_cast<uint32_t*>(f)));
+        for (int c = 0; c < 2; ++c) {
+          float2 h[16];
+          tmem_ld32(taddr + oh * 64 + c * 32,
+                    *reinterpret_cast<uint32_t(*)[32]>(reinterpret_cast<uint32_t*>(h)));
           tmem_wait_ld();
           if (ok)
-            dst[c] = make_uint4(int4x8(f, c2), int4x8(f + 4, c2), int4x8(f + 8, c2),
-                                int4x8(f + 12, c2));
+            dst[c] = make_uint4(int4x8(h, c2), int4x8(h + 4, c2), int4x8(h + 8, c2),
+                                int4x8(h + 12, c2));
         }
       }
       tc_fence_before();
       mbar_arrive(&tempty[d]);
-      if (ok && o == 0) P.scales[token] = scale;
+      if (ok && tau == 0) P.scales[token] = scale;
     }
   }
 
