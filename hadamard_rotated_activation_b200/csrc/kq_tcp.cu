@@ -123,8 +123,8 @@ __device__ __forceinline__ uint32_t b_chunk(int a, int c16) {
 // chunks tau, tau + kGroupThreads, ...; chunk ch holds x'[a*128 + c16*8 .. +7] (a = ch / 16, c16 =
 // ch % 16).  H[i][j] for i = o*128 + b, j = a*128 + c16*8 + e is H_96[o][a]
 // (-1)^(popc(b_hi & c16) + popc(b_lo & e)), b_hi = b / 8, b_lo = b % 8.
-// Values enter fp64 exactly through bf16x2_to_f64_scaled.  Returns this
-// thread's partial sum.
+// Values enter fp64 exactly (bf16 -> fp32 -> fp64 conversions).  Returns
+// this thread's partial sum.
 __device__ __forceinline__ double exact_partial(const uint8_t* tok, int i, int tau) {
   const int o = i >> 7, bhi = (i >> 3) & 15, blo = i & 7;
   uint32_t em[4];
@@ -132,24 +132,23 @@ __device__ __forceinline__ double exact_partial(const uint8_t* tok, int i, int t
   for (int w = 0; w < 4; ++w)
     em[w] = ((uint32_t)(__popc(blo & (2 * w)) & 1) << 15) |
             ((uint32_t)(__popc(blo & (2 * w + 1)) & 1) << 31);
+  const uint32_t fc = (__popc(bhi & (tau & 15)) & 1) ? 0x80008000u : 0u;   // c16 = tau % 16
   double acc[4] = {0.0, 0.0, 0.0, 0.0};
-#pragma unroll 2
+#pragma unroll
   for (int k = 0; k < kChunks / kGroupThreads; ++k) {
     const int ch = tau + kGroupThreads * k;
     const int a = ch >> 4, c16 = ch & 15;
-    const uint32_t flip =
-        (h96_negative(o, a) ^ (__popc(bhi & c16) & 1)) ? 0x80008000u : 0u;
+    const uint32_t flip = (h96_negative(o, a) ? 0x80008000u : 0u) ^ fc;
     const uint4 v = *reinterpret_cast<const uint4*>(tok + b_chunk(a, c16));
     const uint32_t ww[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
-      double lo, hi;
-      bf16x2_to_f64_scaled(ww[w] ^ em[w] ^ flip, lo, hi);
-      acc[w] += lo;
-      acc[(w + 2) & 3] += hi;
+      const uint32_t x2 = ww[w] ^ em[w] ^ flip;   // the two terms' signed bf16 bits
+      acc[w] += (double)__uint_as_float(x2 << 16);           // exact: bf16 -> fp32 -> fp64
+      acc[(w + 2) & 3] += (double)__uint_as_float(x2 & 0xffff0000u);
     }
   }
-  return ((acc[0] + acc[1]) + (acc[2] + acc[3])) * kF64Unscale;
+  return (acc[0] + acc[1]) + (acc[2] + acc[3]);
 }
 
 // Six butterfly stages (H_64, natural order) on f[0..31] (f[p] holds
