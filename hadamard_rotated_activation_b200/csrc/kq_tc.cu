@@ -128,8 +128,8 @@ __device__ __forceinline__ uint32_t tok_chunk(int a, int c) {
 // (a, c) holds x[a*32 + c*8 .. +7] and its sign-flip masks are smask[a*4 + c];
 // H[i][j] for those j is (-1)^(popc(i_hi & a) + popc(i_mid & c) + popc(i_lo &
 // e)) with i = i_hi*32 + i_mid*8 + i_lo, so the Hadamard signs are two bit
-// masks per word selected per chunk.  Values enter fp64 exactly through
-// bf16x2_to_f64_scaled, into four independent accumulators.  Every lane gets
+// masks per word selected per chunk.  Values enter fp64 exactly (bf16 -> fp32
+// -> fp64 conversions), into four independent accumulators.  Every lane gets
 // the result.  Finite inputs.
 __device__ __noinline__ double warp_exact_S(const uint4* __restrict__ row,
                                             const uint4* __restrict__ smask, int i) {
@@ -151,13 +151,12 @@ __device__ __noinline__ double warp_exact_S(const uint4* __restrict__ row,
     const uint32_t ww[4] = {v.x ^ m.x, v.y ^ m.y, v.z ^ m.z, v.w ^ m.w};
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
-      double lo, hi;
-      bf16x2_to_f64_scaled(ww[w] ^ em[w] ^ flip, lo, hi);
-      acc[w] += lo;
-      acc[(w + 2) & 3] += hi;
+      const uint32_t x2 = ww[w] ^ em[w] ^ flip;   // the two terms' signed bf16 bits
+      acc[w] += (double)__uint_as_float(x2 << 16);           // exact: bf16 -> fp32 -> fp64
+      acc[(w + 2) & 3] += (double)__uint_as_float(x2 & 0xffff0000u);
     }
   }
-  return warp_sum_d((acc[0] + acc[1]) + (acc[2] + acc[3])) * kF64Unscale;
+  return warp_sum_d((acc[0] + acc[1]) + (acc[2] + acc[3]));
 }
 
 // The same for rows that hold an infinity or NaN (IEEE conversions, slow).
