@@ -65,6 +65,16 @@ __device__ __forceinline__ float fmin3(float a, float b, float c) {
   return d;
 }
 
+// Eight integers -> eight nibbles (element k in bits 4k .. 4k+3), each
+// saturated to 0..15 by the packing conversion.
+__device__ __forceinline__ uint32_t pack_u4x8(const int (&q)[8]) {
+  uint32_t d = 0;
+#pragma unroll
+  for (int k = 3; k >= 0; --k)
+    asm("cvt.pack.sat.u4.s32.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(q[2 * k + 1]), "r"(q[2 * k]), "r"(d));
+  return d;
+}
+
 __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
   uint64_t ua = *reinterpret_cast<uint64_t*>(&a), ub = *reinterpret_cast<uint64_t*>(&b),
            uc = *reinterpret_cast<uint64_t*>(&c), r;
@@ -399,7 +409,7 @@ __device__ __forceinline__ uint32_t f16x2_pair(float lo, float hi) {
   return out;   // bits 0-15: fp16(lo), bits 16-31: fp16(hi)
 }
 
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 3)
 k_blk128_asym(Params P) {
   const int lane = threadIdx.x & 31;
   const float k15 = (float)(1.0 / (15.0 * 11.313708498984761));
@@ -488,37 +498,31 @@ k_blk128_asym(Params P) {
         decided = true;
       }
     }
-    uint32_t words[16];
-    if (s16 != 0) {
-      const float c = 1.0f / (11.313708498984761f * f16_bits_to_f32((uint16_t)s16));
-      const float2 c2 = make_float2(c, c);
-      // (S c) + (1.5 2^23 + z) rounds S c + z to an integer in the low bits
-      const float magic = 12582912.0f + zf;
-      const float2 m2 = make_float2(magic, magic);
+    // codes, 16 bytes (32 elements) at a time, straight to global memory
+    const float c = (s16 != 0) ? 1.0f / (11.313708498984761f * f16_bits_to_f32((uint16_t)s16))
+                               : 0.0f;
+    if (s16 == 0) zf = 0.0f;
+    const float2 c2 = make_float2(c, c);
+    // (S c) + (1.5 2^23 + z) rounds S c + z to an integer in the low bits
+    const float magic = 12582912.0f + zf;
+    const float2 m2 = make_float2(magic, magic);
+    uint4* dst = reinterpret_cast<uint4*>(P.codes + u * (B / 2));
 #pragma unroll
-      for (int w = 0; w < 16; ++w) {
-        uint32_t word = 0;
+    for (int k = 0; k < 4; ++k) {
+      uint32_t words[4];
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        int q[8];
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
-          const float2 a = fma2(v[4 * w + p], c2, m2);
-          int qx = __float_as_int(a.x) - 0x4B400000;
-          int qy = __float_as_int(a.y) - 0x4B400000;
-          qx = min(max(qx, 0), 15);
-          qy = min(max(qy, 0), 15);
-          word |= ((uint32_t)qx << (8 * p)) | ((uint32_t)qy << (8 * p + 4));
+          const float2 a = fma2(v[16 * k + 4 * w + p], c2, m2);
+          q[2 * p] = __float_as_int(a.x) - 0x4B400000;
+          q[2 * p + 1] = __float_as_int(a.y) - 0x4B400000;
         }
-        words[w] = word;
+        words[w] = pack_u4x8(q);
       }
-    } else {
-#pragma unroll
-      for (int w = 0; w < 16; ++w) words[w] = 0;
-      zf = 0.0f;
+      if (active) dst[k] = make_uint4(words[0], words[1], words[2], words[3]);
     }
-    uint4 cw[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k)
-      cw[k] = make_uint4(words[4 * k], words[4 * k + 1], words[4 * k + 2], words[4 * k + 3]);
-    store_codes(stage, cw, P.codes, ub, P.units);
     if (active) {
       uint16_t zh;
       asm("cvt.rn.f16.f32 %0, %1;" : "=h"(zh) : "f"(zf));
