@@ -162,24 +162,6 @@ __device__ __forceinline__ void load_transform(const uint4* stage, int t, const 
       if (!(p & h)) bfly2(v[p], v[p | h]);
 }
 
-// Writes each thread's 64 code bytes (4 chunks) through the stage so that the
-// warp stores 2 KB with coalesced 16-byte stores.
-__device__ __forceinline__ void store_codes(uint4* stage, const uint4 (&cw)[4], uint8_t* codes,
-                                            int64_t ub, int64_t units) {
-  const int lane = threadIdx.x & 31;
-  __syncwarp();
-#pragma unroll
-  for (int k = 0; k < 4; ++k) stage[lane * 4 + (k ^ (lane & 3))] = cw[k];
-  __syncwarp();
-  uint4* dst = reinterpret_cast<uint4*>(codes + ub * (B / 2));
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int idx = lane + 32 * j;       // chunk idx = unit * 4 + k
-    const int t = idx >> 2, k = idx & 3;
-    if (ub + t < units) dst[idx] = stage[t * 4 + (k ^ (t & 3))];
-  }
-}
-
 // Exact S of element `e` (0..127) of the warp's unit `t`, computed by the
 // whole warp in fp64 from the staged input (lane l sums inputs 4l..4l+3) and
 // the staged sign masks of column block k; every lane gets the result.
@@ -227,7 +209,7 @@ __device__ __forceinline__ float e4m3_recip(uint32_t c) {
 // kMode 0: quantize with the static/dynamic tensor scale.
 // kMode 1: dynamic-scale statistics (row max and bound), no outputs.
 template <int kMode>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 3)
 k_blk128_nvfp4(Params P) {
   const int lane = threadIdx.x & 31;
   float t = 0.0f, c6 = 0.0f, inv_bt = 0.0f;
@@ -360,8 +342,8 @@ k_blk128_nvfp4(Params P) {
         }
       }
     }
-    // codes, two 16-blocks (one 16-byte chunk) at a time
-    uint4 cw[4];
+    // codes, two 16-blocks (one 16-byte chunk) at a time, straight to global
+    uint4* dst = reinterpret_cast<uint4*>(P.codes + u * (B / 2));
     const float2 zero2 = make_float2(0.0f, 0.0f);
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -395,9 +377,8 @@ k_blk128_nvfp4(Params P) {
           words[2 * jj + 1] = w1;
         }
       }
-      cw[k] = make_uint4(words[0], words[1], words[2], words[3]);
+      if (active) dst[k] = make_uint4(words[0], words[1], words[2], words[3]);
     }
-    store_codes(stage, cw, P.codes, ub, P.units);
     if (active) *reinterpret_cast<uint2*>(P.scales8 + u * (B / 16)) = make_uint2(sc[0], sc[1]);
   }
 }
