@@ -37,6 +37,7 @@ KQ_FMT_NVFP4 = 2
 
 C_SYMBOLS = (
     "kq_rht", "kq_rht_quant_int4", "kq_rht_quant_nvfp4", "kq_dequant",
+    "kq_dequant_rht_inverse",
     "kq_workspace_size", "kq_status_str", "kq_last_cuda_error", "kq_version",
     "kq_rht_quant_nvfp4_dynamic_noalloc", "kq_diag_tc_steps",
 )
@@ -76,6 +77,8 @@ def lib() -> ctypes.CDLL:
     L.kq_rht_quant_nvfp4.restype = i32
     L.kq_dequant.argtypes = [i32, vp, vp, vp, vp, i64, i32, i32, vp, vp]
     L.kq_dequant.restype = i32
+    L.kq_dequant_rht_inverse.argtypes = [i32, vp, vp, vp, vp, i64, i32, i32, i32, vp, vp, vp]
+    L.kq_dequant_rht_inverse.restype = i32
     L.kq_rht_quant_nvfp4_dynamic_noalloc.argtypes = [vp, i32, i64, i32, i32, vp, vp, vp,
                                                      vp, vp]
     L.kq_rht_quant_nvfp4_dynamic_noalloc.restype = i32
@@ -182,6 +185,15 @@ def kq_dequant(fmt: int, codes, scales, zeros, tensor_scale, tokens: int, dim: i
     _check(lib().kq_dequant(fmt, _ptr(codes), _ptr(scales), _ptr(zeros),
                             _ptr(tensor_scale), tokens, dim, group, _ptr(out),
                             _stream(stream)), "kq_dequant")
+
+
+def kq_dequant_rht_inverse(fmt: int, codes, scales, zeros, tensor_scale, tokens: int,
+                           dim: int, block: int, group: int, signs, out, stream=None) -> None:
+    """Dequantize and undo the rotation in one call (fp32 out)."""
+    _check(lib().kq_dequant_rht_inverse(fmt, _ptr(codes), _ptr(scales), _ptr(zeros),
+                                        _ptr(tensor_scale), tokens, dim, block, group,
+                                        _ptr(signs), _ptr(out), _stream(stream)),
+           "kq_dequant_rht_inverse")
 
 
 def kq_diag_tc_steps(a, b, d1, d2, status, stream=None) -> None:

@@ -64,6 +64,31 @@ kq_status finish(cudaError_t e) {
   return KQ_OK;
 }
 
+// Format-specific argument checks shared by kq_dequant and
+// kq_dequant_rht_inverse.
+kq_status check_dequant(int fmt, const uint8_t* codes, const void* scales, const void* zeros,
+                        const float* tensor_scale, int64_t tokens, int dim, int group,
+                        const float* out) {
+  if (!aligned(codes, 16) || !aligned(out, 16)) return KQ_ERR_MISALIGNED;
+  switch (fmt) {
+    case KQ_FMT_INT4_SYM:
+      if (!aligned(scales, 4)) return KQ_ERR_MISALIGNED;
+      break;
+    case KQ_FMT_INT4_ASYM:
+      if (group != 128 || dim % group != 0) return KQ_ERR_UNSUPPORTED;
+      if (tokens > 0 && !zeros) return KQ_ERR_INVALID_ARG;
+      if (!aligned(scales, 2) || !aligned(zeros, 2)) return KQ_ERR_MISALIGNED;
+      break;
+    case KQ_FMT_NVFP4:
+      if (tokens > 0 && !tensor_scale) return KQ_ERR_INVALID_ARG;
+      if (!aligned(tensor_scale, 4)) return KQ_ERR_MISALIGNED;
+      break;
+    default:
+      return KQ_ERR_INVALID_ARG;
+  }
+  return KQ_OK;
+}
+
 size_t nv_workspace_bytes(int64_t tokens) {
   return kq::kNvWorkspaceHeader + (size_t)tokens * sizeof(float2);
 }
@@ -175,26 +200,33 @@ KQ_API kq_status kq_dequant(int fmt, const uint8_t* codes, const void* scales,
                             int dim, int group, float* out, kq_stream_t stream) {
   if (tokens < 0 || (tokens > 0 && (!codes || !scales || !out))) return KQ_ERR_INVALID_ARG;
   if (dim <= 0 || dim % 32 != 0) return KQ_ERR_UNSUPPORTED;
-  if (!aligned(codes, 16) || !aligned(out, 16)) return KQ_ERR_MISALIGNED;
-  switch (fmt) {
-    case KQ_FMT_INT4_SYM:
-      if (!aligned(scales, 4)) return KQ_ERR_MISALIGNED;
-      break;
-    case KQ_FMT_INT4_ASYM:
-      if (group != 128 || dim % group != 0) return KQ_ERR_UNSUPPORTED;
-      if (tokens > 0 && !zeros) return KQ_ERR_INVALID_ARG;
-      if (!aligned(scales, 2) || !aligned(zeros, 2)) return KQ_ERR_MISALIGNED;
-      break;
-    case KQ_FMT_NVFP4:
-      if (tokens > 0 && !tensor_scale) return KQ_ERR_INVALID_ARG;
-      if (!aligned(tensor_scale, 4)) return KQ_ERR_MISALIGNED;
-      break;
-    default:
-      return KQ_ERR_INVALID_ARG;
-  }
+  const kq_status st = check_dequant(fmt, codes, scales, zeros, tensor_scale, tokens, dim,
+                                     group, out);
+  if (st != KQ_OK) return st;
   if (tokens == 0) return KQ_OK;
   return finish(kq::launch_dequant(fmt, codes, scales, zeros, tensor_scale, tokens, dim,
                                    group, out, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+KQ_API kq_status kq_dequant_rht_inverse(int fmt, const uint8_t* codes, const void* scales,
+                                        const void* zeros, const float* tensor_scale,
+                                        int64_t tokens, int dim, int block, int group,
+                                        const int8_t* signs, float* out, kq_stream_t stream) {
+  if (tokens < 0 || (tokens > 0 && (!codes || !scales || !out))) return KQ_ERR_INVALID_ARG;
+  kq::Geometry g;
+  kq_status st = make_geometry(dim, block, &g);
+  if (st != KQ_OK) return st;
+  if (signs && !aligned(signs, 8)) return KQ_ERR_MISALIGNED;
+  st = check_dequant(fmt, codes, scales, zeros, tensor_scale, tokens, dim, group, out);
+  if (st != KQ_OK) return st;
+  if (tokens == 0) return KQ_OK;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (fmt == KQ_FMT_NVFP4 &&
+      kq::tci_supported(g, codes, static_cast<const uint8_t*>(scales), signs, out))
+    return finish(kq::launch_tcinv_nvfp4(codes, static_cast<const uint8_t*>(scales),
+                                         tensor_scale, tokens, g, signs, out, s));
+  return finish(kq::launch_dequant_rht_inv(fmt, codes, scales, zeros, tensor_scale, tokens, g,
+                                           group, signs, out, s));
 }
 
 KQ_API size_t kq_workspace_size(int64_t tokens, int dim, int block) {

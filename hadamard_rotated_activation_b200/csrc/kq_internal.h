@@ -83,5 +83,15 @@ cudaError_t launch_diag_tc_steps(const uint16_t* a, const uint16_t* b, float* d1
 cudaError_t launch_dequant(int fmt, const uint8_t* codes, const void* scales,
                            const void* zeros, const float* tensor_scale, int64_t tokens,
                            int n, int group, float* out, cudaStream_t s);
+cudaError_t launch_dequant_rht_inv(int fmt, const uint8_t* codes, const void* scales,
+                                  const void* zeros, const float* tensor_scale,
+                                  int64_t tokens, const Geometry& g, int group,
+                                  const int8_t* signs, float* out, cudaStream_t s);
+// NVFP4 dequant + inverse rotation of 4096-wide rows on the tensor cores.
+bool tci_supported(const Geometry& g, const uint8_t* codes, const uint8_t* scales,
+                   const int8_t* signs, const float* out);
+cudaError_t launch_tcinv_nvfp4(const uint8_t* codes, const uint8_t* scales,
+                               const float* tensor_scale, int64_t tokens, const Geometry& g,
+                               const int8_t* signs, float* out, cudaStream_t s);
 
 }  // namespace kq

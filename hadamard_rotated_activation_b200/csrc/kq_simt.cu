@@ -614,6 +614,72 @@ __global__ void k_dequant_nvfp4(const uint8_t* __restrict__ codes,
   }
 }
 
+// ================================================ dequant + inverse rotation
+// One row per CTA (grid-stride): the row's codes are dequantized into shared
+// memory exactly as kq_dequant writes them (each value the product of code
+// and scale(s), rounded once to fp32), then rotated back as kq_rht with
+// KQ_INVERSE does: FWHT, the transposed Paley factor, 1/sqrt(b), signs.
+__global__ void __launch_bounds__(kThreads)
+k_dequant_rht_inv(int fmt, const uint8_t* __restrict__ codes, const void* __restrict__ scales,
+                  const uint16_t* __restrict__ zeros, const float* __restrict__ tensor_scale,
+                  const int8_t* __restrict__ signs, float* __restrict__ out, int64_t tokens,
+                  Geometry g, int group) {
+  extern __shared__ __align__(16) float smem[];
+  float* buf = smem;
+  const int words = g.n / 8;
+  const float t = fmt == 2 ? *tensor_scale : 0.0f;
+  for (int64_t row = blockIdx.x; row < tokens; row += gridDim.x) {
+    const uint32_t* cw = reinterpret_cast<const uint32_t*>(codes + row * (g.n / 2));
+    for (int c = threadIdx.x; c < words; c += blockDim.x) {
+      const uint32_t w = cw[c];
+      float v[8];
+      if (fmt == 0) {
+        const float s = static_cast<const float*>(scales)[row];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          int q = (w >> (4 * k)) & 15;
+          q = q >= 8 ? q - 16 : q;
+          v[k] = (float)q * s;
+        }
+      } else if (fmt == 1) {
+        const int64_t gi = row * (g.n / group) + (8 * c) / group;
+        const float s = f16_bits_to_f32(static_cast<const uint16_t*>(scales)[gi]);
+        const float z = f16_bits_to_f32(zeros[gi]);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[k] = s * ((float)((w >> (4 * k)) & 15) - z);
+      } else {
+        const float sb =
+            e4m3_decode(static_cast<const uint8_t*>(scales)[row * (g.n / 16) + (c >> 1)]);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[k] = (e2m1_decode((w >> (4 * k)) & 15u) * sb) * t;
+      }
+      float4* b4 = reinterpret_cast<float4*>(buf + 8 * c);
+      b4[0] = make_float4(v[0], v[1], v[2], v[3]);
+      b4[1] = make_float4(v[4], v[5], v[6], v[7]);
+    }
+    __syncthreads();
+    fwht_smem(buf, g.n, g.m);
+    if (g.paley) paley_smem<true>(buf, g.m);
+    float* orow = out + row * g.n;
+    for (int c = threadIdx.x; c < g.n / 4; c += blockDim.x) {
+      float4 v = reinterpret_cast<const float4*>(buf)[c];
+      v.x *= g.inv_sqrt_b;
+      v.y *= g.inv_sqrt_b;
+      v.z *= g.inv_sqrt_b;
+      v.w *= g.inv_sqrt_b;
+      if (signs) {
+        const uint32_t sw = __ldg(reinterpret_cast<const uint32_t*>(signs) + c);
+        v.x = __uint_as_float(__float_as_uint(v.x) ^ (((sw >> 7) & 1u) << 31));
+        v.y = __uint_as_float(__float_as_uint(v.y) ^ (((sw >> 15) & 1u) << 31));
+        v.z = __uint_as_float(__float_as_uint(v.z) ^ (((sw >> 23) & 1u) << 31));
+        v.w = __uint_as_float(__float_as_uint(v.w) ^ (((sw >> 31) & 1u) << 31));
+      }
+      reinterpret_cast<float4*>(orow)[c] = v;
+    }
+    __syncthreads();
+  }
+}
+
 // ============================================================= launchers
 namespace {
 
@@ -755,6 +821,18 @@ cudaError_t launch_dequant(int fmt, const uint8_t* codes, const void* scales,
   else
     k_dequant_nvfp4<<<(int)blocks, 256, 0, s>>>(
         codes, static_cast<const uint8_t*>(scales), tensor_scale, out, tokens, n);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dequant_rht_inv(int fmt, const uint8_t* codes, const void* scales,
+                                  const void* zeros, const float* tensor_scale,
+                                  int64_t tokens, const Geometry& g, int group,
+                                  const int8_t* signs, float* out, cudaStream_t s) {
+  const size_t smem = (size_t)g.n * sizeof(float);
+  auto k = k_dequant_rht_inv;
+  k<<<grid_for((const void*)k, smem, tokens), kThreads, smem, s>>>(
+      fmt, codes, scales, static_cast<const uint16_t*>(zeros), tensor_scale, signs, out,
+      tokens, g, group);
   return cudaGetLastError();
 }
 

@@ -226,3 +226,52 @@ def edge_rows(dim: int, dtype: str, rng_seed: int = 7) -> np.ndarray:
     if dtype == BF16:
         return round_to_bf16(x)
     return x.astype(np.float32).astype(np.float64)
+
+
+@dataclass
+class CodedInputs:
+    """Host-side input of a dequantizing call: packed codes and their scales.
+
+    codes:  uint8 [tokens, dim/2], two 4-bit codes per byte (low nibble first).
+    scales: fp32 [tokens] (INT4 symmetric), fp16 [tokens, dim/group]
+            (asymmetric) or E4M3 bytes [tokens, dim/16] (NVFP4).
+    zeros:  fp16 [tokens, dim/group] (asymmetric) or None.
+    tensor_scale: fp32 (NVFP4) or None.
+    signs:  int8 [dim] of +-1, or None.
+    """
+
+    workload: Workload
+    codes: np.ndarray
+    scales: np.ndarray
+    zeros: Optional[np.ndarray]
+    tensor_scale: Optional[np.float32]
+    signs: Optional[np.ndarray]
+
+
+def make_coded_inputs(w: Workload, tokens: Optional[int] = None,
+                      seed: Optional[int] = None) -> CodedInputs:
+    """Uniformly random codes and scales in the format of workload `w`.
+
+    Every 4-bit code value is equally likely.  NVFP4 block scales are uniform
+    over the finite E4M3 codes 0x00..0x7E (zero and subnormal scales
+    included); the tensor scale is fixed at 2^-8 * 1.37.  INT4 scales are
+    lognormal; asymmetric zeros are uniform on [0, 15] in fp16.  The signs are
+    those `make_inputs` draws for the same workload.
+    """
+    if tokens is not None:
+        w = w.with_tokens(tokens)
+    t, n = w.tokens, w.dim
+    signs = make_inputs(w, tokens=1).signs
+    rng = np.random.default_rng(1000 + (w.seed if seed is None else int(seed)))
+    codes = rng.integers(0, 256, size=(t, n // 2), dtype=np.uint8)
+    zeros = None
+    tscale = None
+    if w.fmt == NVFP4:
+        scales = rng.integers(0, 0x7F, size=(t, n // 16), dtype=np.uint8)
+        tscale = np.float32(1.37 * 2.0 ** -8)
+    elif w.fmt == INT4_SYM:
+        scales = rng.lognormal(-2.0, 1.0, size=t).astype(np.float32)
+    else:
+        scales = rng.lognormal(-3.0, 1.0, size=(t, n // w.group)).astype(np.float16)
+        zeros = rng.uniform(0.0, 15.0, size=(t, n // w.group)).astype(np.float16)
+    return CodedInputs(w, codes, scales, zeros, tscale, signs)

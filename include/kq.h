@@ -181,6 +181,27 @@ KQ_API kq_status kq_dequant(int fmt, const uint8_t* codes, const void* scales,
                             kq_stream_t stream);
 
 /*
+ * kq_dequant_rht_inverse -- the receiving end of the round trip in one call:
+ * out = the inverse rotation (as kq_rht with KQ_INVERSE) of the values that
+ * kq_dequant would write, x_j = s_j sum_i H[i][j] yq_i / sqrt(b) (QuaRot
+ * reviews, review 2 Summary: the rotation is undone exactly by its transpose,
+ * H^T = H for the Sylvester factor).  No intermediate tensor is written.
+ * fmt, codes, scales, zeros, tensor_scale, group: as for kq_dequant.
+ * dim, block, signs: the geometry and signs the codes were produced with (as
+ * for kq_rht).  out: fp32 [tokens, dim], 16-byte aligned; may not alias the
+ * inputs.  Errors: as kq_dequant and kq_rht (KQ_ERR_UNSUPPORTED for a geometry
+ * kq_rht rejects, KQ_ERR_MISALIGNED, KQ_ERR_INVALID_ARG); nothing is launched
+ * on an error.  Results agree with kq_dequant followed by kq_rht(KQ_INVERSE)
+ * to fp32 rounding (the order of the sums may differ).
+ */
+KQ_API kq_status kq_dequant_rht_inverse(int fmt, const uint8_t* codes,
+                                        const void* scales, const void* zeros,
+                                        const float* tensor_scale, int64_t tokens,
+                                        int dim, int block, int group,
+                                        const int8_t* signs, float* out,
+                                        kq_stream_t stream);
+
+/*
  * kq_rht_quant_nvfp4_dynamic_noalloc -- kq_rht_quant_nvfp4 with
  * KQ_SCALE_DYNAMIC, for callers that cannot allocate device memory.  The
  * pages have no counterpart to this entry point; it exists for integration.

@@ -115,6 +115,51 @@ def gpu_dequant(fmt, codes, scales, zeros, tensor_scale, tokens, dim, group=0):
     return out.cpu().numpy()
 
 
+def gpu_dequant_rht_inverse(ci: wl.CodedInputs, signs_mode: str = "aligned"):
+    """kq_dequant_rht_inverse on coded inputs.  signs_mode: "aligned" (the
+    signs at a 16-byte boundary), "offset8" (8 bytes past one: a call the
+    tensor-core kernel declines), or "none" (no signs)."""
+    w = ci.workload
+    dev = "cuda"
+    c = torch.from_numpy(np.ascontiguousarray(ci.codes)).to(dev)
+    s = torch.from_numpy(np.ascontiguousarray(ci.scales)).to(dev)
+    z = None if ci.zeros is None else torch.from_numpy(np.ascontiguousarray(ci.zeros)).to(dev)
+    t = None
+    if ci.tensor_scale is not None:
+        t = torch.tensor([float(ci.tensor_scale)], dtype=torch.float32, device=dev)
+    sg = None
+    if ci.signs is not None and signs_mode != "none":
+        if signs_mode == "aligned":
+            sg = torch.from_numpy(ci.signs).to(dev)
+        else:
+            buf = torch.zeros(w.dim + 16, dtype=torch.int8, device=dev)
+            buf[8:8 + w.dim] = torch.from_numpy(ci.signs).to(dev)
+            sg = buf[8:8 + w.dim]
+            assert sg.data_ptr() % 16 == 8
+    fmt = {wl.INT4_SYM: kq.KQ_FMT_INT4_SYM, wl.INT4_ASYM: kq.KQ_FMT_INT4_ASYM,
+           wl.NVFP4: kq.KQ_FMT_NVFP4}[w.fmt]
+    out = torch.empty((w.tokens, w.dim), dtype=torch.float32, device=dev)
+    kq.kq_dequant_rht_inverse(fmt, c, s, z, t, w.tokens, w.dim, w.block, w.group, sg, out)
+    torch.cuda.synchronize()
+    return out.cpu().numpy()
+
+
+def oracle_dequant_rht_inverse(ci: wl.CodedInputs, rows=None, use_signs=True):
+    """The oracle's dequantized values (fp32, as kq_dequant defines them),
+    rotated back in float64."""
+    w = ci.workload
+    sel = slice(None) if rows is None else rows
+    codes = oracle.unpack_nibbles(ci.codes[sel])
+    if w.fmt == wl.NVFP4:
+        deq = oracle.dequant_nvfp4(codes, ci.scales[sel], ci.tensor_scale)
+    elif w.fmt == wl.INT4_SYM:
+        deq = oracle.dequant_int4_sym(int4_from_nibble(codes), ci.scales[sel])
+    else:
+        deq = oracle.dequant_int4_asym(codes, ci.scales[sel], ci.zeros[sel], w.group)
+    signs = ci.signs if use_signs else None
+    return oracle.rht_inverse(deq.astype(np.float64), signs, w.block)
+
+
 # ------------------------------------------------------------ comparisons
 def check_rotation(got: np.ndarray, want: np.ndarray) -> float:
     """Max relative L2 error per row; asserts the contract."""

@@ -214,3 +214,72 @@ def test_full_size_nvfp4(key):
                          inverse=True)
         want = oracle.rht_inverse(deq[rows].astype(np.float64), inp.signs, w.block)
         P.check_rotation(back[rows], want)
+
+
+# ------------------------------------------------ dequant + inverse rotation
+def _rows_with_tail(t, k, seed):
+    rows = _sample_rows(t, k, seed)
+    return np.unique(np.concatenate([rows, np.arange(max(0, t - 5), t)]))
+
+
+@pytest.mark.parametrize("key,tokens,signs_mode", [
+    ("c4", 37, "aligned"),       # tensor-core kernel, ragged last tile
+    ("c4", 37, "none"),
+    ("c4", 37, "offset8"),       # general kernel
+    ("c4", 4 * 148 * 6 + 3, "aligned"),   # several tiles per CTA: every stage wraps
+    ("c2", 37, "aligned"),       # NVFP4 on block-128 rotation
+    ("c1", 37, "aligned"),       # INT4 symmetric, full 4096
+    ("c3", 13, "aligned"),       # INT4 symmetric, H12 x H1024
+    ("c5", 37, "none"),          # asymmetric INT4 g128, per-head H128
+])
+def test_dequant_rht_inverse_random_codes(key, tokens, signs_mode):
+    ci = wl.make_coded_inputs(wl.WORKLOADS[key], tokens=tokens)
+    got = P.gpu_dequant_rht_inverse(ci, signs_mode)
+    rows = _rows_with_tail(tokens, 40, 3) if tokens > 64 else np.arange(tokens)
+    use = signs_mode != "none" and ci.signs is not None
+    P.check_rotation(got[rows], P.oracle_dequant_rht_inverse(ci, rows, use_signs=use))
+
+
+def test_dequant_rht_inverse_round_trip_c4():
+    """Codes and scales from the oracle's NVFP4 of real rows (edge rows
+    included); the fused call must give the oracle's inverse of them, and x'
+    must lie within the quantization error of x."""
+    inp = small_inputs("c4", 37)
+    w = inp.workload
+    y = oracle.rht(inp.values, inp.signs, w.block)
+    codes, bs, ts = oracle.nvfp4(y)
+    ci = wl.CodedInputs(w.with_tokens(inp.values.shape[0]), oracle.pack_nibbles(codes), bs,
+                        None, ts, inp.signs)
+    got = P.gpu_dequant_rht_inverse(ci)
+    want = P.oracle_dequant_rht_inverse(ci)
+    P.check_rotation(got, want)
+    err = np.linalg.norm(got - inp.values, axis=1)
+    unit = np.repeat(oracle.e4m3_decode(bs), 16, axis=1) * np.float64(ts)
+    unit = np.where(unit > 0, unit, 6.0 * np.float64(ts) * 2.0 ** -10)
+    assert np.all(err <= np.sqrt(np.sum(unit ** 2, axis=1)) * 1.0001 + 1e-6)
+
+
+def test_dequant_rht_inverse_zero_tokens():
+    ci = wl.make_coded_inputs(wl.WORKLOADS["c4"], tokens=1)
+    out = torch.empty((0, 4096), dtype=torch.float32, device="cuda")
+    c = torch.empty((0, 2048), dtype=torch.uint8, device="cuda")
+    s = torch.empty((0, 256), dtype=torch.uint8, device="cuda")
+    t = torch.ones(1, dtype=torch.float32, device="cuda")
+    kq.kq_dequant_rht_inverse(kq.KQ_FMT_NVFP4, c, s, None, t, 0, 4096, 0, 0,
+                              torch.from_numpy(ci.signs).cuda(), out)
+
+
+def test_full_size_dequant_rht_inverse_c4():
+    """The benchmark's round-trip launch (16384 x 4096 NVFP4 -> fp32) on random
+    codes; sampled rows against the oracle, and every row against the
+    two-call path (dequant, then the inverse rotation) within fp32 rounding."""
+    w = wl.WORKLOADS["c4"]
+    ci = wl.make_coded_inputs(w)
+    got = P.gpu_dequant_rht_inverse(ci)
+    rows = _rows_with_tail(w.tokens, 64, 5)
+    P.check_rotation(got[rows], P.oracle_dequant_rht_inverse(ci, rows))
+    deq = P.gpu_dequant(kq.KQ_FMT_NVFP4, ci.codes, ci.scales, None, ci.tensor_scale,
+                        w.tokens, w.dim)
+    winv = wl.Workload("inv", w.tokens, w.dim, wl.F32, w.block, True, w.fmt, 0)
+    two = P.gpu_rht(wl.Inputs(winv, deq.astype(np.float64), deq, ci.signs), inverse=True)
+    P.check_rotation(got, two.astype(np.float64))
