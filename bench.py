@@ -2,7 +2,7 @@
 """Benchmark: rotated + quantized GB/s and tokens/s on B200, fraction of HBM peak.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c4]
-                    [--impl kq|reference] [--no-extras]
+                    [--impl kq|reference] [--no-extras] [--roundtrip-only]
 
 A step is one pass of the hot path over one batch of the workload: load +
 sign, Hadamard butterflies, normalisation folded into the scales, extrema,
@@ -55,6 +55,8 @@ def parse_args():
     p.add_argument("--no-extras", action="store_true",
                    help="skip the per-workload table, dynamic and round-trip timings")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--roundtrip-only", action="store_true",
+                   help="time only the c4 dequant + inverse round trip (one JSON line)")
     p.add_argument("--cpu-seconds", type=float, default=12.0,
                    help="target CPU time of the oracle baseline sample")
     return p.parse_args()
@@ -345,6 +347,13 @@ def main():
     if args.tokens:
         w = w.with_tokens(args.tokens)
     peak, peak_kind = measured_peaks()
+    if args.roundtrip_only:
+        if rank == 0:
+            print(json.dumps(roundtrip(torch, kq, wl, dev, peak, args.steps, args.warmup,
+                                       args.tokens)), flush=True)
+        if dist is not None:
+            dist.destroy_process_group()
+        return
     # every rank draws its own batch (weak scaling)
     inp = wl.make_inputs(w, seed=w.seed + 1000 * rank)
     x0 = device_input(torch, inp, wl, dev)
@@ -477,35 +486,47 @@ def extras(torch, kq, wl, dev, peak, args):
                          "bytes": alg}
             del sets
         if key == "c4":
-            # round trip: dequantize and undo the rotation, fused (one launch),
-            # and as two calls for comparison; rotating code sets of 3x L2
-            c, bs, ts, ws = kq.empty_nvfp4(w.tokens, w.dim, w.block)
-            kq.kq_rht_quant_nvfp4(x0, w.block, signs, c, bs, ts, ws, dynamic=True)
-            in_bytes = w.tokens * w.dim // 2 + w.tokens * w.dim // 16
-            code_sets = [(c, bs)] + [(c.clone(), bs.clone())
-                                     for _ in range(n_sets(in_bytes) - 1)]
-            back = torch.empty((w.tokens, w.dim), dtype=torch.float32, device=dev)
-
-            def rt(cs):
-                kq.kq_dequant_rht_inverse(kq.KQ_FMT_NVFP4, cs[0], cs[1], None, ts, w.tokens,
-                                          w.dim, w.block, 0, signs, back)
-            ms = time_steps(torch, rt, code_sets, k, 5) / k
-            rbytes = in_bytes + 4 * w.tokens * w.dim
-            gbs = rbytes / (ms * 1e-3) / 1e9
-            out["c4_roundtrip"] = {"ms": round(ms, 5), "GB/s": round(gbs, 2),
-                                   "frac": round(gbs / peak, 4), "bytes": rbytes,
-                                   "tokens_per_s": round(w.tokens / (ms * 1e-3), 1),
-                                   "launches_per_step": 1}
-            deq = torch.empty_like(back)
-
-            def rt2(cs):
-                kq.kq_dequant(kq.KQ_FMT_NVFP4, cs[0], cs[1], None, ts, w.tokens, w.dim, 0, deq)
-                kq.kq_rht(deq, w.block, signs, back, inverse=True)
-            ms2 = time_steps(torch, rt2, code_sets, 20, 3) / 20
-            out["c4_roundtrip_two_calls"] = {"ms": round(ms2, 5), "launches_per_step": 2}
-            del code_sets, deq, back
+            out.update(roundtrip(torch, kq, wl, dev, peak, k, 5, 0, x0, signs))
         del x0
         torch.cuda.empty_cache()
+    return out
+
+
+def roundtrip(torch, kq, wl, dev, peak, k, warmup, tokens=0, x0=None, signs=None):
+    """The c4 round trip: NVFP4 codes of the batch, dequantized and rotated back
+    to fp32 by the fused call (one launch), and by the two calls (dequant, then
+    inverse rotation) for comparison; code sets rotate over 3x the L2."""
+    w = wl.WORKLOADS["c4"]
+    if tokens:
+        w = w.with_tokens(tokens)
+    if x0 is None:
+        inp = wl.make_inputs(w)
+        x0 = device_input(torch, inp, wl, dev)
+        signs = None if inp.signs is None else torch.from_numpy(inp.signs).to(dev)
+    c, bs, ts, ws = kq.empty_nvfp4(w.tokens, w.dim, w.block)
+    kq.kq_rht_quant_nvfp4(x0, w.block, signs, c, bs, ts, ws, dynamic=True)
+    in_bytes = w.tokens * w.dim // 2 + w.tokens * w.dim // 16
+    code_sets = [(c, bs)] + [(c.clone(), bs.clone()) for _ in range(n_sets(in_bytes) - 1)]
+    back = torch.empty((w.tokens, w.dim), dtype=torch.float32, device=dev)
+
+    def rt(cs):
+        kq.kq_dequant_rht_inverse(kq.KQ_FMT_NVFP4, cs[0], cs[1], None, ts, w.tokens,
+                                  w.dim, w.block, 0, signs, back)
+    ms = time_steps(torch, rt, code_sets, k, warmup) / k
+    rbytes = in_bytes + 4 * w.tokens * w.dim
+    gbs = rbytes / (ms * 1e-3) / 1e9
+    out = {"c4_roundtrip": {"ms": round(ms, 5), "GB/s": round(gbs, 2),
+                            "frac": round(gbs / peak, 4), "bytes": rbytes,
+                            "tokens_per_s": round(w.tokens / (ms * 1e-3), 1),
+                            "launches_per_step": 1}}
+    deq = torch.empty_like(back)
+
+    def rt2(cs):
+        kq.kq_dequant(kq.KQ_FMT_NVFP4, cs[0], cs[1], None, ts, w.tokens, w.dim, 0, deq)
+        kq.kq_rht(deq, w.block, signs, back, inverse=True)
+    k2 = max(3, min(k, 20))
+    ms2 = time_steps(torch, rt2, code_sets, k2, min(warmup, 3)) / k2
+    out["c4_roundtrip_two_calls"] = {"ms": round(ms2, 5), "launches_per_step": 2}
     return out
 
 
