@@ -141,6 +141,10 @@ KQ_API kq_status kq_rht_quant_int4(const void* x, int dtype, int64_t tokens, int
   if (!aligned(codes, 16)) return KQ_ERR_MISALIGNED;
   if (tokens == 0) return KQ_OK;
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (asym == 1 && kq::tcb_supported(g, dtype, x, tokens))
+    return finish(kq::launch_tcb_asym(x, tokens, g, signs, codes,
+                                      static_cast<uint16_t*>(scales),
+                                      static_cast<uint16_t*>(zeros), s));
   if (asym == 1 && kq::blk128_supported(g, dtype) && aligned(signs, 16))
     return finish(kq::launch_blk128_asym(x, tokens, g, signs, codes,
                                          static_cast<uint16_t*>(scales),

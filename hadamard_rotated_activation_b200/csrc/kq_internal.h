@@ -87,6 +87,11 @@ cudaError_t launch_dequant_rht_inv(int fmt, const uint8_t* codes, const void* sc
                                   const void* zeros, const float* tensor_scale,
                                   int64_t tokens, const Geometry& g, int group,
                                   const int8_t* signs, float* out, cudaStream_t s);
+// Block-128 rotation + asymmetric INT4 g128 on the tensor cores.
+bool tcb_supported(const Geometry& g, int dtype, const void* x, int64_t tokens);
+cudaError_t launch_tcb_asym(const void* x, int64_t tokens, const Geometry& g,
+                            const int8_t* signs, uint8_t* codes, uint16_t* scales,
+                            uint16_t* zeros, cudaStream_t s);
 // NVFP4 dequant + inverse rotation of 4096-wide rows on the tensor cores.
 bool tci_supported(const Geometry& g, const uint8_t* codes, const uint8_t* scales,
                    const int8_t* signs, const float* out);

@@ -107,6 +107,26 @@ def test_int4_asym_other_rotations():
         P.check_int4_asym(c, sc, z, oracle.rht(x, s, block))
 
 
+@pytest.mark.parametrize("dim,tokens,signs", [
+    (4096, 43, True),             # tensor-core block kernel with sign flips
+    (12288, 11, True),            # 96 column blocks per row
+    (4096, 4 * 148 * 6 + 3, False),   # several tiles per CTA, overlapped last tile
+    (4096, 3, True),              # 96 units: below one tile, general kernel
+    (1024, 129, True),            # ragged: 1032 units
+])
+def test_int4_asym_block128_shapes(dim, tokens, signs):
+    rng = np.random.default_rng(dim + tokens)
+    x = rng.standard_normal((tokens, dim)) * np.exp(rng.standard_normal(dim))[None, :]
+    x[:, rng.choice(dim, 4, replace=False)] *= 30
+    edges = wl.edge_rows(dim, wl.BF16)[: max(0, min(6, tokens - 1))]
+    x = wl.round_to_bf16(np.concatenate([x[: tokens - len(edges)], edges]))
+    sg = (1 - 2 * rng.integers(0, 2, dim)).astype(np.int8) if signs else None
+    w = wl.Workload("x", tokens, dim, wl.BF16, 128, signs, wl.INT4_ASYM, 0, group=128)
+    inp = P.inputs_from_values(w, x, sg)
+    c, sc, z = P.gpu_int4_asym(inp)
+    P.check_int4_asym(c, sc, z, oracle.rht(x, sg, 128))
+
+
 # --------------------------------------------------------------- NVFP4
 @pytest.mark.parametrize("key,tokens", [("c2", 37), ("c4", 37)])
 def test_nvfp4_small_dynamic_and_static(key, tokens):
