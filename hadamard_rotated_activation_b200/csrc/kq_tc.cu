@@ -191,6 +191,36 @@ struct FixQueue {
   unsigned int done;      // epilogue warps that will enqueue nothing more
 };
 
+// Queues one undecided block for the fix-up warps (its 16 S_hat values, max,
+// bound and position); kept out of line so that the epilogue's hot path
+// carries none of it.  If no slot frees up within the wait limit the block
+// keeps its provisional scale and the error word records it.
+__device__ __noinline__ void enqueue_fix(FixQueue* fq, long long token, int block, float bm,
+                                         float E, float a0, float a1, float a2, float a3,
+                                         float a4, float a5, float a6, float a7, float a8,
+                                         float a9, float a10, float a11, float a12, float a13,
+                                         float a14, float a15) {
+  const unsigned int slot = atomicAdd(&fq->tail, 1u);
+  const long long t0 = clock64();
+  while (slot >= (unsigned int)kQ && ld_acquire(&fq->cons[slot % kQ]) != slot - kQ + 1) {
+    if (clock64() - t0 > kWaitCycles) {
+      atomicOr(&g_tc_error, 2u);
+      return;
+    }
+    __nanosleep(64);
+  }
+  FixEntry& fe = fq->e[slot % kQ];
+  const float a[16] = {a0, a1, a2, a3, a4, a5, a6, a7, a8, a9, a10, a11, a12, a13, a14, a15};
+#pragma unroll
+  for (int i = 0; i < 16; ++i) fe.v[i] = a[i];
+  fe.bm = bm;
+  fe.E = E;
+  fe.token = token;
+  fe.block = block;
+  __threadfence_block();       // the provisional stores come first
+  st_release(&fq->seq[slot % kQ], slot + 1);
+}
+
 // E2M1 codes of one 16-element block (v: 8 pairs) for the E4M3 scale `code`:
 // two words, element k in bits 4k..4k+3.  rcp[c] = 1 / value of E4M3 code c
 // (a shared-memory table).  A zero scale (or tensor scale) leaves only the
@@ -607,29 +637,10 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
           if (!((undecided >> j) & 1u)) continue;
-          const unsigned int slot = atomicAdd(&fq->tail, 1u);
-          const long long t0 = clock64();
-          bool room = true;   // the slot's previous entry (slot - kQ) is finished
-          while (slot >= (unsigned int)kQ && ld_acquire(&fq->cons[slot % kQ]) != slot - kQ + 1) {
-            if (clock64() - t0 > kWaitCycles) { room = false; break; }
-            __nanosleep(64);
-          }
-          if (!room) {                 // the block keeps its provisional scale
-            atomicOr(&g_tc_error, 2u);
-            continue;
-          }
-          FixEntry& fe = fq->e[slot % kQ];
-#pragma unroll
-          for (int p = 0; p < 8; ++p) {
-            fe.v[2 * p] = v[8 * j + p].x;
-            fe.v[2 * p + 1] = v[8 * j + p].y;
-          }
-          fe.bm = bm[j];
-          fe.E = E;
-          fe.token = token;
-          fe.block = o * 2 + j;
-          __threadfence_block();       // the provisional stores above come first
-          st_release(&fq->seq[slot % kQ], slot + 1);
+          const float2* vb = v + 8 * j;
+          enqueue_fix(fq, token, o * 2 + j, bm[j], E, vb[0].x, vb[0].y, vb[1].x, vb[1].y, vb[2].x,
+                      vb[2].y, vb[3].x, vb[3].y, vb[4].x, vb[4].y, vb[5].x, vb[5].y, vb[6].x,
+                      vb[6].y, vb[7].x, vb[7].y);
         }
       }
     }
