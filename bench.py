@@ -73,24 +73,29 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def source_digest():
+KERNEL_HEADERS = ("kq_sm100.cuh", "kq_device.cuh", "kq_internal.h")
+
+
+def source_digest(files):
+    """Digest of the named csrc files (name and contents), in order."""
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "hadamard_rotated_activation_b200", "csrc", "*"))):
-        with open(f, "rb") as fh:
-            h.update(os.path.basename(f).encode())
+    for name in files:
+        with open(os.path.join(ROOT, "hadamard_rotated_activation_b200", "csrc", name), "rb") as fh:
+            h.update(name.encode())
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
 def ncu_traffic(kernel_key):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel sources; else None."""
+    the kernel's current sources (its .cu file and the shared headers); else
+    None."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             d = json.load(f)
         e = d[kernel_key]
-        if e.get("source_digest") != source_digest():
+        if e.get("source_digest") != source_digest(e["sources"]):
             return None
         return float(e["dram_bytes_per_launch"])
     except Exception:
@@ -484,6 +489,9 @@ def extras(torch, kq, wl, dev, peak, args):
                          "tokens_per_s": round(w.tokens / (ms * 1e-3), 1),
                          "launches_per_step": launches,
                          "bytes": alg}
+            tkey = f"{key}_{w.fmt}" + ("_static" if mode == "static" else "")
+            if mode != "dynamic" and ncu_traffic(tkey) is not None:
+                out[name]["traffic"] = round(ncu_traffic(tkey))
             del sets
         if key == "c4":
             out.update(roundtrip(torch, kq, wl, dev, peak, k, 5, 0, x0, signs))
@@ -519,6 +527,8 @@ def roundtrip(torch, kq, wl, dev, peak, k, warmup, tokens=0, x0=None, signs=None
                             "frac": round(gbs / peak, 4), "bytes": rbytes,
                             "tokens_per_s": round(w.tokens / (ms * 1e-3), 1),
                             "launches_per_step": 1}}
+    if ncu_traffic("c4_roundtrip") is not None and not tokens:
+        out["c4_roundtrip"]["traffic"] = round(ncu_traffic("c4_roundtrip"))
     deq = torch.empty_like(back)
 
     def rt2(cs):
