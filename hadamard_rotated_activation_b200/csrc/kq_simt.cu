@@ -524,7 +524,9 @@ k_nvfp4_rowstats(const T* __restrict__ x, const int8_t* __restrict__ signs,
 }
 
 // Dynamic tensor scale, step 2: exact max|S| over the elements of the rows
-// that can hold the global maximum.
+// that can hold the global maximum.  Each CTA screens a contiguous range of
+// rows with all its threads at once (one row's statistics per thread) and
+// then transforms only the candidates.
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
 k_nvfp4_global(const T* __restrict__ x, const int8_t* __restrict__ signs,
@@ -532,19 +534,34 @@ k_nvfp4_global(const T* __restrict__ x, const int8_t* __restrict__ signs,
   extern __shared__ __align__(16) float smem[];
   float* buf = smem;
   double* red = reinterpret_cast<double*>(buf + g.n);
+  __shared__ int64_t cand[kThreads];
+  __shared__ int ncand;
   const float L = __uint_as_float(ws->lower_bits);
-  for (int64_t row = blockIdx.x; row < tokens; row += gridDim.x) {
-    const float2 st = ws->rows[row];
-    if ((double)st.x + (double)st.y < (double)L) continue;   // uniform per CTA
-    const T* xr = x + row * g.n;
-    transform_row(xr, signs, buf, g, false);
-    // candidates from this kernel's own fp32 values and their own bound
-    const double Eg = error_bound(g, row_absmax(buf, g.n, red));
-    const double best = exact_max_abs(xr, signs, g, buf, 0, g.n,
-                                      thr_down((double)L - Eg), red);
-    if (threadIdx.x == 0)
-      atomicMax(&ws->gmax_bits, (unsigned long long)__double_as_longlong(best));
+  const int64_t per = (tokens + gridDim.x - 1) / gridDim.x;
+  const int64_t r0 = (int64_t)blockIdx.x * per;
+  const int64_t r1 = r0 + per < tokens ? r0 + per : tokens;
+  for (int64_t base = r0; base < r1; base += blockDim.x) {
+    if (threadIdx.x == 0) ncand = 0;
     __syncthreads();
+    const int64_t row = base + threadIdx.x;
+    if (row < r1) {
+      const float2 st = ws->rows[row];
+      if ((double)st.x + (double)st.y >= (double)L) cand[atomicAdd(&ncand, 1)] = row;
+    }
+    __syncthreads();
+    const int nc = ncand;
+    for (int c = 0; c < nc; ++c) {
+      const T* xr = x + cand[c] * g.n;
+      transform_row(xr, signs, buf, g, false);
+      // candidates from this kernel's own fp32 values and their own bound
+      const double Eg = error_bound(g, row_absmax(buf, g.n, red));
+      const double best = exact_max_abs(xr, signs, g, buf, 0, g.n,
+                                        thr_down((double)L - Eg), red);
+      if (threadIdx.x == 0)
+        atomicMax(&ws->gmax_bits, (unsigned long long)__double_as_longlong(best));
+      __syncthreads();
+    }
+    __syncthreads();   // every thread has read ncand before the next reset
   }
 }
 
