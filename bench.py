@@ -529,6 +529,19 @@ def roundtrip(torch, kq, wl, dev, peak, k, warmup, tokens=0, x0=None, signs=None
                             "launches_per_step": 1}}
     if ncu_traffic("c4_roundtrip") is not None and not tokens:
         out["c4_roundtrip"]["traffic"] = round(ncu_traffic("c4_roundtrip"))
+    back16 = torch.empty((w.tokens, w.dim), dtype=torch.bfloat16, device=dev)
+
+    def rt16(cs):
+        kq.kq_dequant_rht_inverse(kq.KQ_FMT_NVFP4, cs[0], cs[1], None, ts, w.tokens,
+                                  w.dim, w.block, 0, signs, back16)
+    ms16 = time_steps(torch, rt16, code_sets, k, warmup) / k
+    b16 = in_bytes + 2 * w.tokens * w.dim
+    g16 = b16 / (ms16 * 1e-3) / 1e9
+    out["c4_roundtrip_bf16"] = {"ms": round(ms16, 5), "GB/s": round(g16, 2),
+                                "frac": round(g16 / peak, 4), "bytes": b16,
+                                "tokens_per_s": round(w.tokens / (ms16 * 1e-3), 1),
+                                "launches_per_step": 1}
+    del back16
     deq = torch.empty_like(back)
 
     def rt2(cs):

@@ -77,7 +77,8 @@ def lib() -> ctypes.CDLL:
     L.kq_rht_quant_nvfp4.restype = i32
     L.kq_dequant.argtypes = [i32, vp, vp, vp, vp, i64, i32, i32, vp, vp]
     L.kq_dequant.restype = i32
-    L.kq_dequant_rht_inverse.argtypes = [i32, vp, vp, vp, vp, i64, i32, i32, i32, vp, vp, vp]
+    L.kq_dequant_rht_inverse.argtypes = [i32, vp, vp, vp, vp, i64, i32, i32, i32, vp, vp, i32,
+                                         vp]
     L.kq_dequant_rht_inverse.restype = i32
     L.kq_rht_quant_nvfp4_dynamic_noalloc.argtypes = [vp, i32, i64, i32, i32, vp, vp, vp,
                                                      vp, vp]
@@ -189,10 +190,11 @@ def kq_dequant(fmt: int, codes, scales, zeros, tensor_scale, tokens: int, dim: i
 
 def kq_dequant_rht_inverse(fmt: int, codes, scales, zeros, tensor_scale, tokens: int,
                            dim: int, block: int, group: int, signs, out, stream=None) -> None:
-    """Dequantize and undo the rotation in one call (fp32 out)."""
+    """Dequantize and undo the rotation in one call; `out` is fp32 or bf16."""
     _check(lib().kq_dequant_rht_inverse(fmt, _ptr(codes), _ptr(scales), _ptr(zeros),
                                         _ptr(tensor_scale), tokens, dim, block, group,
-                                        _ptr(signs), _ptr(out), _stream(stream)),
+                                        _ptr(signs), _ptr(out), _dtype_code(out),
+                                        _stream(stream)),
            "kq_dequant_rht_inverse")
 
 

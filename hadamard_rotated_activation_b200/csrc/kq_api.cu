@@ -68,7 +68,7 @@ kq_status finish(cudaError_t e) {
 // kq_dequant_rht_inverse.
 kq_status check_dequant(int fmt, const uint8_t* codes, const void* scales, const void* zeros,
                         const float* tensor_scale, int64_t tokens, int dim, int group,
-                        const float* out) {
+                        const void* out) {
   if (!aligned(codes, 16) || !aligned(out, 16)) return KQ_ERR_MISALIGNED;
   switch (fmt) {
     case KQ_FMT_INT4_SYM:
@@ -215,8 +215,10 @@ KQ_API kq_status kq_dequant(int fmt, const uint8_t* codes, const void* scales,
 KQ_API kq_status kq_dequant_rht_inverse(int fmt, const uint8_t* codes, const void* scales,
                                         const void* zeros, const float* tensor_scale,
                                         int64_t tokens, int dim, int block, int group,
-                                        const int8_t* signs, float* out, kq_stream_t stream) {
+                                        const int8_t* signs, void* out, int out_dtype,
+                                        kq_stream_t stream) {
   if (tokens < 0 || (tokens > 0 && (!codes || !scales || !out))) return KQ_ERR_INVALID_ARG;
+  if (out_dtype != KQ_F32 && out_dtype != KQ_BF16) return KQ_ERR_UNSUPPORTED;
   kq::Geometry g;
   kq_status st = make_geometry(dim, block, &g);
   if (st != KQ_OK) return st;
@@ -225,12 +227,13 @@ KQ_API kq_status kq_dequant_rht_inverse(int fmt, const uint8_t* codes, const voi
   if (st != KQ_OK) return st;
   if (tokens == 0) return KQ_OK;
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int bf16 = out_dtype == KQ_BF16 ? 1 : 0;
   if (fmt == KQ_FMT_NVFP4 &&
       kq::tci_supported(g, codes, static_cast<const uint8_t*>(scales), signs, out))
     return finish(kq::launch_tcinv_nvfp4(codes, static_cast<const uint8_t*>(scales),
-                                         tensor_scale, tokens, g, signs, out, s));
+                                         tensor_scale, tokens, g, signs, out, bf16, s));
   return finish(kq::launch_dequant_rht_inv(fmt, codes, scales, zeros, tensor_scale, tokens, g,
-                                           group, signs, out, s));
+                                           group, signs, out, bf16, s));
 }
 
 KQ_API size_t kq_workspace_size(int64_t tokens, int dim, int block) {

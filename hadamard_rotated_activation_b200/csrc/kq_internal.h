@@ -86,7 +86,7 @@ cudaError_t launch_dequant(int fmt, const uint8_t* codes, const void* scales,
 cudaError_t launch_dequant_rht_inv(int fmt, const uint8_t* codes, const void* scales,
                                   const void* zeros, const float* tensor_scale,
                                   int64_t tokens, const Geometry& g, int group,
-                                  const int8_t* signs, float* out, cudaStream_t s);
+                                  const int8_t* signs, void* out, int out_bf16, cudaStream_t s);
 // Block-128 rotation + asymmetric INT4 g128 on the tensor cores.
 bool tcb_supported(const Geometry& g, int dtype, const void* x, int64_t tokens);
 cudaError_t launch_tcb_asym(const void* x, int64_t tokens, const Geometry& g,
@@ -94,9 +94,9 @@ cudaError_t launch_tcb_asym(const void* x, int64_t tokens, const Geometry& g,
                             uint16_t* zeros, cudaStream_t s);
 // NVFP4 dequant + inverse rotation of 4096-wide rows on the tensor cores.
 bool tci_supported(const Geometry& g, const uint8_t* codes, const uint8_t* scales,
-                   const int8_t* signs, const float* out);
+                   const int8_t* signs, const void* out);
 cudaError_t launch_tcinv_nvfp4(const uint8_t* codes, const uint8_t* scales,
                                const float* tensor_scale, int64_t tokens, const Geometry& g,
-                               const int8_t* signs, float* out, cudaStream_t s);
+                               const int8_t* signs, void* out, int out_bf16, cudaStream_t s);
 
 }  // namespace kq

@@ -636,10 +636,11 @@ __global__ void k_dequant_nvfp4(const uint8_t* __restrict__ codes,
 // memory exactly as kq_dequant writes them (each value the product of code
 // and scale(s), rounded once to fp32), then rotated back as kq_rht with
 // KQ_INVERSE does: FWHT, the transposed Paley factor, 1/sqrt(b), signs.
+template <bool kBf16Out>
 __global__ void __launch_bounds__(kThreads)
 k_dequant_rht_inv(int fmt, const uint8_t* __restrict__ codes, const void* __restrict__ scales,
                   const uint16_t* __restrict__ zeros, const float* __restrict__ tensor_scale,
-                  const int8_t* __restrict__ signs, float* __restrict__ out, int64_t tokens,
+                  const int8_t* __restrict__ signs, void* __restrict__ out, int64_t tokens,
                   Geometry g, int group) {
   extern __shared__ __align__(16) float smem[];
   float* buf = smem;
@@ -677,7 +678,6 @@ k_dequant_rht_inv(int fmt, const uint8_t* __restrict__ codes, const void* __rest
     __syncthreads();
     fwht_smem(buf, g.n, g.m);
     if (g.paley) paley_smem<true>(buf, g.m);
-    float* orow = out + row * g.n;
     for (int c = threadIdx.x; c < g.n / 4; c += blockDim.x) {
       float4 v = reinterpret_cast<const float4*>(buf)[c];
       v.x *= g.inv_sqrt_b;
@@ -691,7 +691,14 @@ k_dequant_rht_inv(int fmt, const uint8_t* __restrict__ codes, const void* __rest
         v.z = __uint_as_float(__float_as_uint(v.z) ^ (((sw >> 23) & 1u) << 31));
         v.w = __uint_as_float(__float_as_uint(v.w) ^ (((sw >> 31) & 1u) << 31));
       }
-      reinterpret_cast<float4*>(orow)[c] = v;
+      if (kBf16Out) {
+        uint32_t lo, hi;
+        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(lo) : "f"(v.y), "f"(v.x));
+        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(hi) : "f"(v.w), "f"(v.z));
+        reinterpret_cast<uint2*>(static_cast<uint16_t*>(out) + row * g.n)[c] = make_uint2(lo, hi);
+      } else {
+        reinterpret_cast<float4*>(static_cast<float*>(out) + row * g.n)[c] = v;
+      }
     }
     __syncthreads();
   }
@@ -844,9 +851,9 @@ cudaError_t launch_dequant(int fmt, const uint8_t* codes, const void* scales,
 cudaError_t launch_dequant_rht_inv(int fmt, const uint8_t* codes, const void* scales,
                                   const void* zeros, const float* tensor_scale,
                                   int64_t tokens, const Geometry& g, int group,
-                                  const int8_t* signs, float* out, cudaStream_t s) {
+                                  const int8_t* signs, void* out, int out_bf16, cudaStream_t s) {
   const size_t smem = (size_t)g.n * sizeof(float);
-  auto k = k_dequant_rht_inv;
+  auto k = out_bf16 ? k_dequant_rht_inv<true> : k_dequant_rht_inv<false>;
   k<<<grid_for((const void*)k, smem, tokens), kThreads, smem, s>>>(
       fmt, codes, scales, static_cast<const uint16_t*>(zeros), tensor_scale, signs, out,
       tokens, g, group);

@@ -11,7 +11,7 @@
 // H_128 z' over a on the tensor cores (A = H_128, B = z of four tokens,
 // MN-major, 64-byte swizzle), then H_32 over beta in the epilogue thread that
 // owns TMEM lane o; it holds outputs o*32 .. o*32+31, multiplies by
-// t / sqrt(n), applies the signs and stores fp32.
+// t / sqrt(n), applies the signs and stores fp32 or bf16 (rounded to nearest).
 //
 // Warp roles (14 warps, up to 128 registers a thread): 0 copies (1-D bulk
 // copies of the codes and block scales of four tokens), 1 MMA issuer + TMEM
@@ -58,7 +58,7 @@ struct Params {
   const uint8_t* scales8;       // [T, n/16] E4M3
   const float* tensor_scale;    // device
   const int8_t* signs;          // [n] or null
-  float* out;                   // [T, n]
+  void* out;                    // [T, n] fp32 or bf16
   int64_t tokens;
   int64_t tiles;
 };
@@ -90,6 +90,12 @@ __device__ __forceinline__ uint32_t e4m3_to_f16x2_dup(uint32_t code) {
   asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(d) : "h"(two));
   return d;
 }
+// bf16x2 of (lo, hi), each rounded to nearest even.
+__device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
 __device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
   uint32_t d;
   asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
@@ -100,6 +106,7 @@ __device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
 constexpr uint32_t kIdesc = (1u << 4) | (0u << 7) | (0u << 10) | (1u << 16) |
                             ((uint32_t)(kAccCols >> 3) << 17) | ((128u >> 4) << 24);
 
+template <bool kBf16Out>
 __global__ void __launch_bounds__(kThreads, 1) k_tcinv4096(Params P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -297,27 +304,49 @@ __global__ void __launch_bounds__(kThreads, 1) k_tcinv4096(Params P) {
           for (int p = 0; p < 16; ++p)
             if (!(p & hh)) bfly2(v[p], v[p | hh]);
         // The warp's 32 lanes hold outputs q*1024 .. q*1024+1023 of the token,
-        // 128 contiguous bytes per lane: staged through shared memory (16-byte
-        // chunk p of lane l at position p ^ (l & 7)), they leave as 512-byte
-        // coalesced stores.
+        // 128 (fp32) or 64 (bf16) contiguous bytes per lane: staged through
+        // shared memory (16-byte chunk p of lane l at position p ^ (l & 7),
+        // or p ^ ((l >> 1) & 3) for bf16), they leave as 512-byte coalesced
+        // stores.
+        const int64_t token = tile * kTok + t;
+        float4 r[8];
 #pragma unroll
         for (int p = 0; p < 8; ++p) {
-          float4 r = make_float4(v[2 * p].x * scale, v[2 * p].y * scale,
-                                 v[2 * p + 1].x * scale, v[2 * p + 1].y * scale);
-          r.x = __uint_as_float(__float_as_uint(r.x) ^ (((sbits >> (4 * p)) & 1u) << 31));
-          r.y = __uint_as_float(__float_as_uint(r.y) ^ (((sbits >> (4 * p + 1)) & 1u) << 31));
-          r.z = __uint_as_float(__float_as_uint(r.z) ^ (((sbits >> (4 * p + 2)) & 1u) << 31));
-          r.w = __uint_as_float(__float_as_uint(r.w) ^ (((sbits >> (4 * p + 3)) & 1u) << 31));
-          *reinterpret_cast<float4*>(wbuf + lane * 128 + ((p ^ (lane & 7)) << 4)) = r;
+          r[p] = make_float4(v[2 * p].x * scale, v[2 * p].y * scale, v[2 * p + 1].x * scale,
+                             v[2 * p + 1].y * scale);
+          r[p].x = __uint_as_float(__float_as_uint(r[p].x) ^ (((sbits >> (4 * p)) & 1u) << 31));
+          r[p].y = __uint_as_float(__float_as_uint(r[p].y) ^ (((sbits >> (4 * p + 1)) & 1u) << 31));
+          r[p].z = __uint_as_float(__float_as_uint(r[p].z) ^ (((sbits >> (4 * p + 2)) & 1u) << 31));
+          r[p].w = __uint_as_float(__float_as_uint(r[p].w) ^ (((sbits >> (4 * p + 3)) & 1u) << 31));
         }
-        __syncwarp();
-        const int64_t token = tile * kTok + t;
-        if (token < P.tokens) {
-          float4* dst = reinterpret_cast<float4*>(P.out + token * N + q * 1024);
+        if (kBf16Out) {
 #pragma unroll
-          for (int r8 = 0; r8 < 8; ++r8) {
-            const int kc = r8 * 32 + lane, l2 = kc >> 3, p2 = kc & 7;
-            dst[kc] = *reinterpret_cast<const float4*>(wbuf + l2 * 128 + ((p2 ^ (l2 & 7)) << 4));
+          for (int c = 0; c < 4; ++c)
+            *reinterpret_cast<uint4*>(wbuf + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4)) =
+                make_uint4(bf16x2_rn(r[2 * c].x, r[2 * c].y), bf16x2_rn(r[2 * c].z, r[2 * c].w),
+                           bf16x2_rn(r[2 * c + 1].x, r[2 * c + 1].y),
+                           bf16x2_rn(r[2 * c + 1].z, r[2 * c + 1].w));
+          __syncwarp();
+          if (token < P.tokens) {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(P.out) + token * N + q * 1024);
+#pragma unroll
+            for (int r4 = 0; r4 < 4; ++r4) {
+              const int kc = r4 * 32 + lane, l2 = kc >> 2, p2 = kc & 3;
+              dst[kc] = *reinterpret_cast<const uint4*>(wbuf + l2 * 64 + ((p2 ^ ((l2 >> 1) & 3)) << 4));
+            }
+          }
+        } else {
+#pragma unroll
+          for (int p = 0; p < 8; ++p)
+            *reinterpret_cast<float4*>(wbuf + lane * 128 + ((p ^ (lane & 7)) << 4)) = r[p];
+          __syncwarp();
+          if (token < P.tokens) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(P.out) + token * N + q * 1024);
+#pragma unroll
+            for (int r8 = 0; r8 < 8; ++r8) {
+              const int kc = r8 * 32 + lane, l2 = kc >> 3, p2 = kc & 7;
+              dst[kc] = *reinterpret_cast<const float4*>(wbuf + l2 * 128 + ((p2 ^ (l2 & 7)) << 4));
+            }
           }
         }
         __syncwarp();
@@ -337,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_tcinv4096(Params P) {
 }  // namespace tci
 
 bool tci_supported(const Geometry& g, const uint8_t* codes, const uint8_t* scales,
-                   const int8_t* signs, const float* out) {
+                   const int8_t* signs, const void* out) {
   return !g.paley && g.b == g.n && g.n == tci::N &&
          (reinterpret_cast<uintptr_t>(codes) & 15) == 0 &&
          (reinterpret_cast<uintptr_t>(scales) & 15) == 0 &&
@@ -347,7 +376,7 @@ bool tci_supported(const Geometry& g, const uint8_t* codes, const uint8_t* scale
 
 cudaError_t launch_tcinv_nvfp4(const uint8_t* codes, const uint8_t* scales,
                                const float* tensor_scale, int64_t tokens, const Geometry& g,
-                               const int8_t* signs, float* out, cudaStream_t s) {
+                               const int8_t* signs, void* out, int out_bf16, cudaStream_t s) {
   (void)g;
   tci::Params P{};
   P.codes = codes;
@@ -359,13 +388,13 @@ cudaError_t launch_tcinv_nvfp4(const uint8_t* codes, const uint8_t* scales,
   P.tiles = (tokens + tci::kTok - 1) / tci::kTok;
   constexpr size_t kSmem = 1024 + 32768 + tci::kStages * (tci::kZBytes + tci::kRawBytes) +
                            tci::kEpiWarps * 4096 + 256;
-  cudaFuncSetAttribute((const void*)tci::k_tcinv4096,
-                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
+  auto k = out_bf16 ? tci::k_tcinv4096<true> : tci::k_tcinv4096<false>;
+  cudaFuncSetAttribute((const void*)k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t grid = P.tiles < sms ? P.tiles : sms;
-  tci::k_tcinv4096<<<(int)grid, tci::kThreads, kSmem, s>>>(P);
+  k<<<(int)grid, tci::kThreads, kSmem, s>>>(P);
   return cudaGetLastError();
 }
 

@@ -188,18 +188,20 @@ KQ_API kq_status kq_dequant(int fmt, const uint8_t* codes, const void* scales,
  * H^T = H for the Sylvester factor).  No intermediate tensor is written.
  * fmt, codes, scales, zeros, tensor_scale, group: as for kq_dequant.
  * dim, block, signs: the geometry and signs the codes were produced with (as
- * for kq_rht).  out: fp32 [tokens, dim], 16-byte aligned; may not alias the
- * inputs.  Errors: as kq_dequant and kq_rht (KQ_ERR_UNSUPPORTED for a geometry
- * kq_rht rejects, KQ_ERR_MISALIGNED, KQ_ERR_INVALID_ARG); nothing is launched
- * on an error.  Results agree with kq_dequant followed by kq_rht(KQ_INVERSE)
- * to fp32 rounding (the order of the sums may differ).
+ * for kq_rht).  out: [tokens, dim], fp32 (out_dtype = KQ_F32) or bf16
+ * (KQ_BF16: the fp32 result rounded to nearest even), 16-byte aligned; may
+ * not alias the inputs.  Errors: as kq_dequant and kq_rht (KQ_ERR_UNSUPPORTED
+ * for a geometry kq_rht rejects or another out_dtype, KQ_ERR_MISALIGNED,
+ * KQ_ERR_INVALID_ARG); nothing is launched on an error.  Results agree with
+ * kq_dequant followed by kq_rht(KQ_INVERSE) to fp32 rounding (the order of
+ * the sums may differ).
  */
 KQ_API kq_status kq_dequant_rht_inverse(int fmt, const uint8_t* codes,
                                         const void* scales, const void* zeros,
                                         const float* tensor_scale, int64_t tokens,
                                         int dim, int block, int group,
-                                        const int8_t* signs, float* out,
-                                        kq_stream_t stream);
+                                        const int8_t* signs, void* out,
+                                        int out_dtype, kq_stream_t stream);
 
 /*
  * kq_rht_quant_nvfp4_dynamic_noalloc -- kq_rht_quant_nvfp4 with

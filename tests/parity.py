@@ -115,7 +115,8 @@ def gpu_dequant(fmt, codes, scales, zeros, tensor_scale, tokens, dim, group=0):
     return out.cpu().numpy()
 
 
-def gpu_dequant_rht_inverse(ci: wl.CodedInputs, signs_mode: str = "aligned"):
+def gpu_dequant_rht_inverse(ci: wl.CodedInputs, signs_mode: str = "aligned",
+                            out_dtype: str = "f32"):
     """kq_dequant_rht_inverse on coded inputs.  signs_mode: "aligned" (the
     signs at a 16-byte boundary), "offset8" (8 bytes past one: a call the
     tensor-core kernel declines), or "none" (no signs)."""
@@ -138,10 +139,25 @@ def gpu_dequant_rht_inverse(ci: wl.CodedInputs, signs_mode: str = "aligned"):
             assert sg.data_ptr() % 16 == 8
     fmt = {wl.INT4_SYM: kq.KQ_FMT_INT4_SYM, wl.INT4_ASYM: kq.KQ_FMT_INT4_ASYM,
            wl.NVFP4: kq.KQ_FMT_NVFP4}[w.fmt]
-    out = torch.empty((w.tokens, w.dim), dtype=torch.float32, device=dev)
+    tdt = torch.bfloat16 if out_dtype == "bf16" else torch.float32
+    out = torch.empty((w.tokens, w.dim), dtype=tdt, device=dev)
     kq.kq_dequant_rht_inverse(fmt, c, s, z, t, w.tokens, w.dim, w.block, w.group, sg, out)
     torch.cuda.synchronize()
-    return out.cpu().numpy()
+    return out.float().cpu().numpy()
+
+
+def check_rotation_bf16(got: np.ndarray, want: np.ndarray) -> None:
+    """bf16 outputs of an fp32 rotation: each within one bf16 ulp of the exact
+    value plus the fp32 rotation's own error (REL_L2 of the row norm), and an
+    all-zero row exactly zero."""
+    got = got.astype(np.float64)
+    norm = np.linalg.norm(want, axis=1, keepdims=True)
+    mag = np.abs(want)
+    with np.errstate(divide="ignore"):
+        ulp = np.where(mag > 0, 2.0 ** (np.floor(np.log2(np.where(mag > 0, mag, 1.0))) - 7), 0.0)
+    bad = np.abs(got - want) > ulp + 2 * REL_L2 * norm
+    assert not bad.any(), f"{int(bad.sum())} bf16 outputs off by more than one ulp"
+    assert np.all(got[norm[:, 0] == 0] == 0)
 
 
 def oracle_dequant_rht_inverse(ci: wl.CodedInputs, rows=None, use_signs=True):

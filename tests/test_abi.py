@@ -103,20 +103,21 @@ def test_argument_errors(L):
     assert L.kq_workspace_size(4, 4095, 0) == 0
     # dequant + inverse rotation: the rotation's shape checks, then dequant's
     r = L.kq_dequant_rht_inverse
-    assert r(2, Q, Q, None, P, 0, 4096, 0, 0, None, P, None) == kq.KQ_OK
-    assert r(2, None, None, None, None, 0, 4096, 0, 0, None, None, None) == kq.KQ_OK
-    assert r(2, Q, Q, None, P, -1, 4096, 0, 0, None, P, None) == kq.KQ_ERR_INVALID_ARG
-    assert r(2, Q, Q, None, P, 4, 4095, 0, 0, None, P, None) == kq.KQ_ERR_UNSUPPORTED
-    assert r(2, Q, Q, None, P, 4, 4096, 100, 0, None, P, None) == kq.KQ_ERR_UNSUPPORTED
-    assert r(2, Q, Q, None, None, 4, 4096, 0, 0, None, P, None) == kq.KQ_ERR_INVALID_ARG
-    assert r(2, Q, Q, None, P, 4, 4096, 0, 0, None, None, None) == kq.KQ_ERR_INVALID_ARG
-    assert r(2, Q, Q, None, P, 4, 4096, 0, 0, P + 4, P, None) == kq.KQ_ERR_MISALIGNED
-    assert r(2, Q, Q, None, P, 4, 4096, 0, 0, None, P + 4, None) == kq.KQ_ERR_MISALIGNED
-    assert r(2, Q + 8, Q, None, P, 4, 4096, 0, 0, None, P, None) == kq.KQ_ERR_MISALIGNED
-    assert r(1, Q, Q, None, None, 4, 4096, 0, 128, None, P, None) == kq.KQ_ERR_INVALID_ARG
-    assert r(1, Q, Q, Q, None, 4, 4096, 0, 64, None, P, None) == kq.KQ_ERR_UNSUPPORTED
-    assert r(0, Q, Q + 2, None, None, 4, 4096, 0, 0, None, P, None) == kq.KQ_ERR_MISALIGNED
-    assert r(5, Q, Q, None, None, 4, 4096, 0, 0, None, P, None) == kq.KQ_ERR_INVALID_ARG
+    assert r(2, Q, Q, None, P, 4, 4096, 0, 0, None, P, 2, None) == kq.KQ_ERR_UNSUPPORTED
+    assert r(2, Q, Q, None, P, 0, 4096, 0, 0, None, P, 0, None) == kq.KQ_OK
+    assert r(2, None, None, None, None, 0, 4096, 0, 0, None, None, 0, None) == kq.KQ_OK
+    assert r(2, Q, Q, None, P, -1, 4096, 0, 0, None, P, 0, None) == kq.KQ_ERR_INVALID_ARG
+    assert r(2, Q, Q, None, P, 4, 4095, 0, 0, None, P, 0, None) == kq.KQ_ERR_UNSUPPORTED
+    assert r(2, Q, Q, None, P, 4, 4096, 100, 0, None, P, 0, None) == kq.KQ_ERR_UNSUPPORTED
+    assert r(2, Q, Q, None, None, 4, 4096, 0, 0, None, P, 0, None) == kq.KQ_ERR_INVALID_ARG
+    assert r(2, Q, Q, None, P, 4, 4096, 0, 0, None, None, 0, None) == kq.KQ_ERR_INVALID_ARG
+    assert r(2, Q, Q, None, P, 4, 4096, 0, 0, P + 4, P, 0, None) == kq.KQ_ERR_MISALIGNED
+    assert r(2, Q, Q, None, P, 4, 4096, 0, 0, None, P + 4, 0, None) == kq.KQ_ERR_MISALIGNED
+    assert r(2, Q + 8, Q, None, P, 4, 4096, 0, 0, None, P, 0, None) == kq.KQ_ERR_MISALIGNED
+    assert r(1, Q, Q, None, None, 4, 4096, 0, 128, None, P, 0, None) == kq.KQ_ERR_INVALID_ARG
+    assert r(1, Q, Q, Q, None, 4, 4096, 0, 64, None, P, 0, None) == kq.KQ_ERR_UNSUPPORTED
+    assert r(0, Q, Q + 2, None, None, 4, 4096, 0, 0, None, P, 0, None) == kq.KQ_ERR_MISALIGNED
+    assert r(5, Q, Q, None, None, 4, 4096, 0, 0, None, P, 0, None) == kq.KQ_ERR_INVALID_ARG
     t = L.kq_diag_tc_steps
     assert t(None, P, P, P, P, None) == kq.KQ_ERR_INVALID_ARG
     assert t(P + 1, P, P, P, P, None) == kq.KQ_ERR_MISALIGNED

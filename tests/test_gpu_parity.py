@@ -260,6 +260,18 @@ def test_dequant_rht_inverse_random_codes(key, tokens, signs_mode):
     P.check_rotation(got[rows], P.oracle_dequant_rht_inverse(ci, rows, use_signs=use))
 
 
+@pytest.mark.parametrize("key,tokens,signs_mode", [
+    ("c4", 37, "aligned"), ("c4", 4 * 148 * 6 + 3, "aligned"), ("c4", 37, "offset8"),
+    ("c5", 37, "none"),
+])
+def test_dequant_rht_inverse_bf16_out(key, tokens, signs_mode):
+    ci = wl.make_coded_inputs(wl.WORKLOADS[key], tokens=tokens)
+    got = P.gpu_dequant_rht_inverse(ci, signs_mode, out_dtype="bf16")
+    rows = _rows_with_tail(tokens, 40, 4) if tokens > 64 else np.arange(tokens)
+    use = signs_mode != "none" and ci.signs is not None
+    P.check_rotation_bf16(got[rows], P.oracle_dequant_rht_inverse(ci, rows, use_signs=use))
+
+
 def test_dequant_rht_inverse_round_trip_c4():
     """Codes and scales from the oracle's NVFP4 of real rows (edge rows
     included); the fused call must give the oracle's inverse of them, and x'
