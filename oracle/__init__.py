@@ -32,5 +32,5 @@ from .formats import (  # noqa: F401
 from .quant import (  # noqa: F401
     int4_sym_per_token, int4_asym_group, nvfp4, nvfp4_tensor_scale,
     dequant_int4_sym, dequant_int4_asym, dequant_nvfp4, pack_nibbles,
-    unpack_nibbles,
+    unpack_nibbles, mxfp4, mxfp4_exponents, dequant_mxfp4,
 )

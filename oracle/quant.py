@@ -24,6 +24,13 @@ Readings where the pages are silent (each listed in the design notes):
   * INT4 asymmetric: scale16 = fp16((mx - mn) / 15) in one rounding;
     z = rint(-mn / scale16), stored as fp16; u = clamp(rint(y / scale16) + z,
     0, 15) using the stored z; a group with scale16 == 0 has z = 0, u = 0.
+  * MXFP4 (named on the same thread, discrete_descent's comparison of
+    rotations under NVFP4, MXFP4 and INT4-g128; the pages give no bit-level
+    definition): the public OCP Microscaling Formats (MX) v1.0 reading.
+    Blocks of 32 consecutive elements share an E8M0 scale X = 2^e with
+    e = floor(log2(amax64)) - 2 (2 = the largest E2M1 exponent), clamped to
+    [-127, 127], stored as the byte e + 127; an all-zero block has e = -127.
+    code = E2M1(y / X) (nearest even, saturating at 6), sign bit = (y < 0).
   * Dequantization: the exact product of code and scale(s), rounded once to
     fp32.
   * Packing: two codes per byte, element 2k in bits 0-3, 2k+1 in bits 4-7.
@@ -169,3 +176,47 @@ def dequant_nvfp4(codes: np.ndarray, block_scales: np.ndarray,
     v = e2m1_decode(c).reshape(t_rows, n // 16, 16)
     s = e4m3_decode(block_scales)[..., None] * np.float64(np.float32(tensor_scale))
     return (v * s).reshape(t_rows, n).astype(np.float32)
+
+
+# ------------------------------------------------------------------ MXFP4
+MX_BLOCK = 32
+E2M1_EMAX = 2          # largest E2M1 value 6 = 1.5 * 2^2
+
+
+def mxfp4_exponents(y: np.ndarray) -> np.ndarray:
+    """Shared exponent e per 32-block of rows y (float64 [T, n]), int64
+    [T, n/32]: floor(log2(max |y|)) - 2 clamped to [-127, 127] (frexp gives
+    floor(log2) exactly); an all-zero block gets -127."""
+    y = np.asarray(y, dtype=np.float64)
+    t_rows, n = y.shape
+    if n % MX_BLOCK:
+        raise ValueError("MXFP4 needs dim % 32 == 0")
+    amax = np.max(np.abs(y.reshape(t_rows, n // MX_BLOCK, MX_BLOCK)), axis=2)
+    _, ex = np.frexp(amax)                      # amax = m 2^ex, 0.5 <= m < 1
+    e = ex.astype(np.int64) - 1 - E2M1_EMAX
+    e = np.where(amax > 0, e, -127)
+    return np.clip(e, -127, 127)
+
+
+def mxfp4(y: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
+    """MXFP4 of rotated rows y (float64 [T, n], n % 32 == 0).
+
+    Returns (codes uint8 [T, n] E2M1 4-bit codes, scales uint8 [T, n/32]
+    E8M0 bytes e + 127).
+    """
+    y = np.asarray(y, dtype=np.float64)
+    t_rows, n = y.shape
+    e = mxfp4_exponents(y)
+    blk = y.reshape(t_rows, n // MX_BLOCK, MX_BLOCK)
+    v = blk / np.ldexp(1.0, e)[..., None]       # exact: division by a power of two
+    codes = e2m1_encode(v)
+    return codes.reshape(t_rows, n).astype(np.uint8), (e + 127).astype(np.uint8)
+
+
+def dequant_mxfp4(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    c = np.asarray(codes)
+    t_rows, n = c.shape
+    v = e2m1_decode(c).reshape(t_rows, n // MX_BLOCK, MX_BLOCK)
+    x = np.ldexp(1.0, np.asarray(scales, dtype=np.int64) - 127)[..., None]
+    with np.errstate(over="ignore"):
+        return (v * x).reshape(t_rows, n).astype(np.float32)

@@ -5,8 +5,9 @@ import numpy as np
 import pytest
 
 from oracle import (
-    dequant_int4_asym, dequant_int4_sym, dequant_nvfp4, e2m1_decode, e4m3_decode,
-    int4_asym_group, int4_sym_per_token, nvfp4, pack_nibbles, rht, unpack_nibbles,
+    dequant_int4_asym, dequant_int4_sym, dequant_mxfp4, dequant_nvfp4, e2m1_decode,
+    e4m3_decode, int4_asym_group, int4_sym_per_token, mxfp4, mxfp4_exponents, nvfp4,
+    pack_nibbles, rht, unpack_nibbles,
 )
 from oracle.quant import int4_from_nibble
 from hadamard_rotated_activation_b200 import workloads as wl
@@ -158,3 +159,70 @@ def test_int4_asym_constant_group():
     u, s16, z16 = int4_asym_group(y, 128)
     assert s16[0, 0] == 0 and z16[0, 0] == 0 and np.all(u[0, :128] == 0)
     assert u[0, 128] == 0 and u[0, 255] == 15
+
+
+# ------------------------------------------------------------------ MXFP4
+def test_mxfp4_hand_example():
+    """Worked by hand from the MX definition: X = 2^(floor(log2 amax) - 2)."""
+    y = np.zeros((2, 64))
+    y[0, 32] = 1.0
+    y[0, 33:64] = 0.5          # amax 1: e = -2, X = 1/4, v = 4 and 2
+    y[1, 0] = -6.0             # amax 6: e = 0, X = 1, v = -6
+    y[1, 1] = 0.75             # v = 0.75: tie between 0.5 and 1, even index -> 1
+    y[1, 32:64] = 3.9          # amax 3.9: e = -1, X = 1/2, v = 7.8 saturates to 6
+    codes, sc = mxfp4(y)
+    assert sc.tolist() == [[0, 125], [127, 126]]
+    assert np.all(codes[0, :32] == 0)                    # all-zero block
+    assert codes[0, 32] == 6 and np.all(codes[0, 33:64] == 4)
+    assert codes[1, 0] == 15 and codes[1, 1] == 2
+    assert np.all(codes[1, 32:] == 7)
+    deq = dequant_mxfp4(codes, sc)
+    assert deq[1, 0] == -6.0 and deq[1, 1] == 1.0 and deq[1, 32] == 3.0
+
+
+def test_mxfp4_exponent_brackets_block_max():
+    rng = np.random.default_rng(5)
+    y = rng.standard_normal((6, 256)) * np.exp(rng.uniform(-40, 40, (6, 1)))
+    y[0, :32] = 2.0 ** 7                   # amax exactly a power of two
+    y[1, :32] = -np.nextafter(2.0 ** 7, 0)  # just below one
+    e = mxfp4_exponents(y)
+    amax = np.max(np.abs(y.reshape(6, 8, 32)), axis=2)
+    lo, hi = np.ldexp(1.0, e + 2), np.ldexp(1.0, e + 3)
+    assert np.all((lo <= amax) & (amax < hi))
+    assert e[0, 0] == 5 and e[1, 0] == 4
+
+
+def test_mxfp4_half_step_bound_and_saturation():
+    y = _rotated("c4", 16)
+    codes, sc = mxfp4(y)
+    deq = dequant_mxfp4(codes, sc).astype(np.float64)
+    X = np.repeat(np.ldexp(1.0, sc.astype(np.int64) - 127), 32, axis=1)
+    v = np.abs(y) / X
+    mag = np.abs(e2m1_decode(codes))
+    half_gap = np.where(mag < 2, 0.25, np.where(mag < 4, 0.5, 1.0))
+    err = np.abs(y - deq)
+    unsat = v <= 6.0
+    assert np.all(err[unsat] <= half_gap[unsat] * X[unsat])
+    # v < 8 always (amax < 2^(e+3)); saturated values lose less than 2 X
+    assert np.all(v < 8.0)
+    assert np.all(err[~unsat] < 2.0 * X[~unsat])
+    assert np.all(mag[~unsat] == 6.0)
+
+
+def test_mxfp4_power_of_two_scaling_and_clamps():
+    rng = np.random.default_rng(6)
+    y = rng.standard_normal((3, 64))
+    c0, s0 = mxfp4(y)
+    c1, s1 = mxfp4(y * 2.0 ** 9)
+    assert np.array_equal(c0, c1) and np.all(s1.astype(int) - s0.astype(int) == 9)
+    tiny = np.full((1, 32), 2.0 ** -140)
+    c, s = mxfp4(tiny)
+    assert s[0, 0] == 0                  # e clamped to -127
+    huge = np.full((1, 32), 2.0 ** 200)
+    c, s = mxfp4(huge)
+    assert s[0, 0] == 254 and np.all(c == 7)   # e clamped to 127, v saturates
+    neg = np.zeros((1, 32))
+    neg[0, 0] = 1.0
+    neg[0, 1] = -1e-9                  # rounds to zero: sign bit kept (0x8)
+    c, s = mxfp4(neg)
+    assert c[0, 1] == 0x8 and c[0, 2] == 0
