@@ -495,6 +495,19 @@ def extras(torch, kq, wl, dev, peak, args):
             del sets
         if key == "c4":
             out.update(roundtrip(torch, kq, wl, dev, peak, k, 5, 0, x0, signs))
+            # the same batch as MXFP4 (E8M0 scale per 32 elements)
+            mx_sets = [(x0 if i == 0 else x0.clone(),) + kq.empty_mxfp4(w.tokens, w.dim)
+                       for i in range(n_sets(w.tokens * w.dim * 2))]
+
+            def mx_step(st):
+                kq.kq_rht_quant_mxfp4(st[0], w.block, signs, st[1], st[2])
+            ms = time_steps(torch, mx_step, mx_sets, k, 5) / k
+            mb = w.tokens * (w.dim * 2 + w.dim // 2 + w.dim // 32)
+            out["c4_mxfp4"] = {"ms": round(ms, 5), "GB/s": round(mb / (ms * 1e-3) / 1e9, 2),
+                               "frac": round(mb / (ms * 1e-3) / 1e9 / peak, 4), "bytes": mb,
+                               "tokens_per_s": round(w.tokens / (ms * 1e-3), 1),
+                               "launches_per_step": 1}
+            del mx_sets
         del x0
         torch.cuda.empty_cache()
     return out

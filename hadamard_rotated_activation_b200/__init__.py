@@ -34,10 +34,11 @@ KQ_SCALE_DYNAMIC = 4
 KQ_FMT_INT4_SYM = 0
 KQ_FMT_INT4_ASYM = 1
 KQ_FMT_NVFP4 = 2
+KQ_FMT_MXFP4 = 3
 
 C_SYMBOLS = (
     "kq_rht", "kq_rht_quant_int4", "kq_rht_quant_nvfp4", "kq_dequant",
-    "kq_dequant_rht_inverse",
+    "kq_dequant_rht_inverse", "kq_rht_quant_mxfp4",
     "kq_workspace_size", "kq_status_str", "kq_last_cuda_error", "kq_version",
     "kq_rht_quant_nvfp4_dynamic_noalloc", "kq_diag_tc_steps",
 )
@@ -77,6 +78,8 @@ def lib() -> ctypes.CDLL:
     L.kq_rht_quant_nvfp4.restype = i32
     L.kq_dequant.argtypes = [i32, vp, vp, vp, vp, i64, i32, i32, vp, vp]
     L.kq_dequant.restype = i32
+    L.kq_rht_quant_mxfp4.argtypes = [vp, i32, i64, i32, i32, vp, vp, vp, vp]
+    L.kq_rht_quant_mxfp4.restype = i32
     L.kq_dequant_rht_inverse.argtypes = [i32, vp, vp, vp, vp, i64, i32, i32, i32, vp, vp, i32,
                                          vp]
     L.kq_dequant_rht_inverse.restype = i32
@@ -169,6 +172,14 @@ def kq_rht_quant_nvfp4(x, block: int, signs, codes, block_scales, tensor_scale,
            "kq_rht_quant_nvfp4")
 
 
+def kq_rht_quant_mxfp4(x, block: int, signs, codes, scales, stream=None) -> None:
+    """Rotation + MXFP4 (E2M1 codes, one E8M0 scale byte per 32 elements)."""
+    t, n = x.shape
+    _check(lib().kq_rht_quant_mxfp4(_ptr(x), _dtype_code(x), t, n, block, _ptr(signs),
+                                    _ptr(codes), _ptr(scales), _stream(stream)),
+           "kq_rht_quant_mxfp4")
+
+
 def kq_rht_quant_nvfp4_dynamic_noalloc(x, block: int, signs, codes, block_scales,
                                        tensor_scale, stream=None) -> None:
     """Dynamic-scale NVFP4 for callers that cannot allocate device memory: the
@@ -227,6 +238,13 @@ def empty_int4_asym(tokens: int, dim: int, group: int = 128, device="cuda"):
     return (torch.empty((tokens, dim // 2), dtype=torch.uint8, device=device),
             torch.empty((tokens, g), dtype=torch.float16, device=device),
             torch.empty((tokens, g), dtype=torch.float16, device=device))
+
+
+def empty_mxfp4(tokens: int, dim: int, device="cuda"):
+    """(codes, scales) for kq_rht_quant_mxfp4."""
+    import torch
+    return (torch.empty((tokens, dim // 2), dtype=torch.uint8, device=device),
+            torch.empty((tokens, dim // 32), dtype=torch.uint8, device=device))
 
 
 def empty_nvfp4(tokens: int, dim: int, block: int = 0, device="cuda"):

@@ -83,6 +83,8 @@ kq_status check_dequant(int fmt, const uint8_t* codes, const void* scales, const
       if (tokens > 0 && !tensor_scale) return KQ_ERR_INVALID_ARG;
       if (!aligned(tensor_scale, 4)) return KQ_ERR_MISALIGNED;
       break;
+    case KQ_FMT_MXFP4:
+      break;
     default:
       return KQ_ERR_INVALID_ARG;
   }
@@ -197,6 +199,19 @@ KQ_API kq_status kq_rht_quant_nvfp4(const void* x, int dtype, int64_t tokens, in
                                            reinterpret_cast<cudaStream_t>(stream)));
   return finish(kq::launch_nvfp4(x, dtype, tokens, g, signs, codes, block_scales,
                                  tensor_scale, ws, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+KQ_API kq_status kq_rht_quant_mxfp4(const void* x, int dtype, int64_t tokens, int dim,
+                                    int block, const int8_t* signs, uint8_t* codes,
+                                    uint8_t* scales, kq_stream_t stream) {
+  kq::Geometry g;
+  kq_status st = check_common(x, dtype, tokens, dim, block, signs, &g);
+  if (st != KQ_OK) return st;
+  if (tokens > 0 && (!codes || !scales)) return KQ_ERR_INVALID_ARG;
+  if (!aligned(codes, 16)) return KQ_ERR_MISALIGNED;
+  if (tokens == 0) return KQ_OK;
+  return finish(kq::launch_mxfp4(x, dtype, tokens, g, signs, codes, scales,
+                                 reinterpret_cast<cudaStream_t>(stream)));
 }
 
 KQ_API kq_status kq_dequant(int fmt, const uint8_t* codes, const void* scales,

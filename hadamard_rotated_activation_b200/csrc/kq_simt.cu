@@ -502,6 +502,87 @@ k_nvfp4(const T* __restrict__ x, const int8_t* __restrict__ signs,
   }
 }
 
+// ================================================================ MXFP4
+// Shared exponent of a 32-block from the largest |S| of the block: e =
+// floor(log2(smax / sqrt(b))) - 2, clamped to [-127, 127] (OCP MX: the
+// largest E2M1 exponent is 2); an all-zero block gets -127.  Monotone in
+// smax, so equal exponents at both ends of an interval decide it.
+__device__ __forceinline__ int mx_exponent(double smax, double sqrt_b) {
+  const double y = smax / sqrt_b;
+  if (!(y > 0.0)) return -127;
+  const int e = ilogb(y) - 2;
+  return e < -127 ? -127 : (e > 127 ? 127 : e);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads)
+k_mxfp4(const T* __restrict__ x, const int8_t* __restrict__ signs,
+        uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, int64_t tokens, Geometry g) {
+  extern __shared__ __align__(16) float smem[];
+  float* buf = smem;
+  const int nb = g.n / 32;
+  float* bmax = buf + g.n;
+  uint8_t* bsc = reinterpret_cast<uint8_t*>(bmax + nb);
+  uint8_t* bflag = bsc + nb;
+  double* red = reinterpret_cast<double*>(
+      (reinterpret_cast<uintptr_t>(bflag + nb) + 15) & ~uintptr_t(15));
+  for (int64_t row = blockIdx.x; row < tokens; row += gridDim.x) {
+    const T* xr = x + row * g.n;
+    transform_row(xr, signs, buf, g, false);
+    const float mh = row_absmax(buf, g.n, red);
+    const double E = error_bound(g, mh);
+    for (int k = threadIdx.x; k < nb; k += blockDim.x) {
+      float m = 0.0f;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) m = fmaxf(m, fabsf(buf[32 * k + e]));
+      bmax[k] = m;
+      const int lo = mx_exponent(fmax((double)m - E, 0.0), g.sqrt_b);
+      const int hi = mx_exponent((double)m + E, g.sqrt_b);
+      bsc[k] = (uint8_t)(lo + 127);
+      bflag[k] = lo != hi;
+    }
+    __syncthreads();
+    for (int k = 0; k < nb; ++k) {
+      if (!bflag[k]) continue;                 // uniform: shared flag
+      const double smax = exact_max_abs(xr, signs, g, buf, 32 * k, 32 * k + 32,
+                                        thr_down((double)bmax[k] - 2.0 * E), red);
+      if (threadIdx.x == 0) bsc[k] = (uint8_t)(mx_exponent(smax, g.sqrt_b) + 127);
+    }
+    __syncthreads();
+    uint4* crow = reinterpret_cast<uint4*>(codes + row * (g.n / 2));
+    for (int k = threadIdx.x; k < nb; k += blockDim.x) {
+      const int e = (int)bsc[k] - 127;
+      const float c = (float)ldexp(1.0 / g.sqrt_b, -e);   // 1 / (sqrt(b) 2^e)
+      float v[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float a = buf[32 * k + i] * c;
+        v[i] = (a == 0.0f) ? 0.0f : a;          // -0 carries no sign bit
+      }
+      crow[k] = make_uint4(e2m1x8_hw(v), e2m1x8_hw(v + 8), e2m1x8_hw(v + 16), e2m1x8_hw(v + 24));
+      scales[row * nb + k] = bsc[k];
+    }
+    __syncthreads();
+  }
+}
+
+__global__ void k_dequant_mxfp4(const uint8_t* __restrict__ codes,
+                                const uint8_t* __restrict__ scales, float* __restrict__ out,
+                                int64_t tokens, int n) {
+  const int64_t words = tokens * (int64_t)(n / 8);
+  for (int64_t q = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; q < words;
+       q += (int64_t)gridDim.x * blockDim.x) {
+    const float sx = ldexpf(1.0f, (int)scales[q >> 2] - 127);   // exact power of two
+    const uint32_t w = reinterpret_cast<const uint32_t*>(codes)[q];
+    float v[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) v[k] = e2m1_decode((w >> (4 * k)) & 15u) * sx;
+    float4* o = reinterpret_cast<float4*>(out + 8 * q);
+    o[0] = make_float4(v[0], v[1], v[2], v[3]);
+    o[1] = make_float4(v[4], v[5], v[6], v[7]);
+  }
+}
+
 // Dynamic tensor scale, step 1: per-row computed max and error bound, and a
 // global lower bound on max|S| (atomicMax on non-negative float bits).
 template <typename T>
@@ -665,6 +746,11 @@ k_dequant_rht_inv(int fmt, const uint8_t* __restrict__ codes, const void* __rest
         const float z = f16_bits_to_f32(zeros[gi]);
 #pragma unroll
         for (int k = 0; k < 8; ++k) v[k] = s * ((float)((w >> (4 * k)) & 15) - z);
+      } else if (fmt == 3) {
+        const float sx =
+            ldexpf(1.0f, (int)static_cast<const uint8_t*>(scales)[row * (g.n / 32) + (c >> 2)] - 127);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[k] = e2m1_decode((w >> (4 * k)) & 15u) * sx;
       } else {
         const float sb =
             e4m3_decode(static_cast<const uint8_t*>(scales)[row * (g.n / 16) + (c >> 1)]);
@@ -842,6 +928,9 @@ cudaError_t launch_dequant(int fmt, const uint8_t* codes, const void* scales,
     k_dequant_int4_asym<<<(int)blocks, 256, 0, s>>>(
         codes, static_cast<const uint16_t*>(scales), static_cast<const uint16_t*>(zeros),
         out, tokens, n, group);
+  else if (fmt == 3)
+    k_dequant_mxfp4<<<(int)blocks, 256, 0, s>>>(
+        codes, static_cast<const uint8_t*>(scales), out, tokens, n);
   else
     k_dequant_nvfp4<<<(int)blocks, 256, 0, s>>>(
         codes, static_cast<const uint8_t*>(scales), tensor_scale, out, tokens, n);
@@ -857,6 +946,23 @@ cudaError_t launch_dequant_rht_inv(int fmt, const uint8_t* codes, const void* sc
   k<<<grid_for((const void*)k, smem, tokens), kThreads, smem, s>>>(
       fmt, codes, scales, static_cast<const uint16_t*>(zeros), tensor_scale, signs, out,
       tokens, g, group);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mxfp4(const void* x, int dtype, int64_t tokens, const Geometry& g,
+                         const int8_t* signs, uint8_t* codes, uint8_t* scales,
+                         cudaStream_t s) {
+  const int nb = g.n / 32;
+  const size_t smem = (size_t)g.n * 4 + (size_t)nb * 6 + 16 + 64 * 8;
+  if (dtype == 1) {
+    auto k = k_mxfp4<uint16_t>;
+    k<<<grid_for((const void*)k, smem, tokens), kThreads, smem, s>>>(
+        static_cast<const uint16_t*>(x), signs, codes, scales, tokens, g);
+  } else {
+    auto k = k_mxfp4<float>;
+    k<<<grid_for((const void*)k, smem, tokens), kThreads, smem, s>>>(
+        static_cast<const float*>(x), signs, codes, scales, tokens, g);
+  }
   return cudaGetLastError();
 }
 

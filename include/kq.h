@@ -113,7 +113,7 @@ enum {
 };
 
 /* formats for kq_dequant */
-enum { KQ_FMT_INT4_SYM = 0, KQ_FMT_INT4_ASYM = 1, KQ_FMT_NVFP4 = 2 };
+enum { KQ_FMT_INT4_SYM = 0, KQ_FMT_INT4_ASYM = 1, KQ_FMT_NVFP4 = 2, KQ_FMT_MXFP4 = 3 };
 
 /*
  * kq_rht -- rotation only, fp32 output.
@@ -167,12 +167,32 @@ KQ_API kq_status kq_rht_quant_nvfp4(const void* x, int dtype, int64_t tokens,
                                     kq_stream_t stream);
 
 /*
+ * kq_rht_quant_mxfp4 -- rotation fused with MXFP4 quantization (named in the
+ * NVFP4 thread, discrete_descent's comparison of rotations under NVFP4, MXFP4
+ * and INT4-g128; the bit-level layout is the OCP Microscaling (MX) v1.0
+ * format): E2M1 codes, one E8M0 power-of-two scale per 32 consecutive
+ * elements, no tensor scale.  A block's scale is X = 2^e with
+ * e = floor(log2(max |y|)) - 2 over the block, clamped to [-127, 127] and
+ * stored as the byte e + 127 (an all-zero block stores 0); code = E2M1(y / X),
+ * nearest even, saturating at 6.  The scale byte is exact: blocks whose
+ * exponent the fp32 transform leaves undecided are recomputed in fp64.
+ * codes: [tokens, dim/2] (16-byte aligned); scales: E8M0 bytes
+ * [tokens, dim/32].  dim, block, signs and errors as for kq_rht.
+ */
+KQ_API kq_status kq_rht_quant_mxfp4(const void* x, int dtype, int64_t tokens,
+                                    int dim, int block, const int8_t* signs,
+                                    uint8_t* codes, uint8_t* scales,
+                                    kq_stream_t stream);
+
+/*
  * kq_dequant -- codes and scales back to fp32: each output is the exact
  * product of the code value and its scale(s), rounded once to fp32.
  * fmt = KQ_FMT_INT4_SYM: scales fp32 [tokens]; zeros and tensor_scale unused.
  * fmt = KQ_FMT_INT4_ASYM: scales, zeros fp16 [tokens, dim/group]; group = 128.
  * fmt = KQ_FMT_NVFP4: scales = E4M3 bytes [tokens, dim/16]; tensor_scale =
  *   device fp32.
+ * fmt = KQ_FMT_MXFP4: scales = E8M0 bytes [tokens, dim/32]; tensor_scale and
+ *   zeros unused.
  * out: fp32 [tokens, dim].
  */
 KQ_API kq_status kq_dequant(int fmt, const uint8_t* codes, const void* scales,

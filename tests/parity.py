@@ -105,6 +105,10 @@ def gpu_dequant(fmt, codes, scales, zeros, tensor_scale, tokens, dim, group=0):
         s = torch.from_numpy(np.ascontiguousarray(scales)).to(dev)
         z = torch.from_numpy(np.ascontiguousarray(zeros)).to(dev)
         t = None
+    elif fmt == kq.KQ_FMT_MXFP4:
+        s = torch.from_numpy(np.ascontiguousarray(scales)).to(dev)
+        z = None
+        t = None
     else:
         s = torch.from_numpy(np.ascontiguousarray(scales)).to(dev)
         z = None
@@ -138,7 +142,7 @@ def gpu_dequant_rht_inverse(ci: wl.CodedInputs, signs_mode: str = "aligned",
             sg = buf[8:8 + w.dim]
             assert sg.data_ptr() % 16 == 8
     fmt = {wl.INT4_SYM: kq.KQ_FMT_INT4_SYM, wl.INT4_ASYM: kq.KQ_FMT_INT4_ASYM,
-           wl.NVFP4: kq.KQ_FMT_NVFP4}[w.fmt]
+           wl.NVFP4: kq.KQ_FMT_NVFP4, "mxfp4": kq.KQ_FMT_MXFP4}[w.fmt]
     tdt = torch.bfloat16 if out_dtype == "bf16" else torch.float32
     out = torch.empty((w.tokens, w.dim), dtype=tdt, device=dev)
     kq.kq_dequant_rht_inverse(fmt, c, s, z, t, w.tokens, w.dim, w.block, w.group, sg, out)
@@ -246,6 +250,32 @@ def check_nvfp4(codes, bscales, tscale, y64, tensor_scale=None):
     bad = diff & ~near
     assert not bad.any(), _first_diff(c, c_ref, "e2m1 code", bad)
     return int(diff.sum())
+
+
+def check_mxfp4(codes, scales, y64):
+    """MXFP4: E8M0 scale bytes bit-exact; codes bit-exact except within NEAR
+    (relative) of an E2M1 rounding boundary, or the sign of a zero."""
+    c_ref, s_ref = oracle.mxfp4(y64)
+    assert np.array_equal(scales, s_ref), _first_diff(scales, s_ref, "E8M0 scale")
+    c = oracle.unpack_nibbles(codes)
+    diff = c != c_ref
+    X = np.repeat(np.ldexp(1.0, s_ref.astype(np.int64) - 127), 32, axis=1)
+    v = np.abs(y64 / X)
+    near = np.any(np.abs(v[..., None] - E2M1_MIDPOINTS) <= NEAR * E2M1_MIDPOINTS, axis=-1)
+    zero_mag = (c_ref & 7) == 0
+    near |= diff & zero_mag & ((c & 7) == 0) & (v <= NEAR)
+    bad = diff & ~near
+    assert not bad.any(), _first_diff(c, c_ref, "e2m1 code", bad)
+    return int(diff.sum())
+
+
+def gpu_mxfp4(inp: wl.Inputs):
+    w = inp.workload
+    x, s = to_device(inp)
+    codes, scales = kq.empty_mxfp4(w.tokens, w.dim)
+    kq.kq_rht_quant_mxfp4(x, w.block, s, codes, scales)
+    torch.cuda.synchronize()
+    return codes.cpu().numpy(), scales.cpu().numpy()
 
 
 def _first_diff(a, b, what, mask=None):

@@ -91,7 +91,7 @@ def test_argument_errors(L):
     assert g(P, 1, 0, 4096, 0, None, Q, Q, Q, P, ws, kq.KQ_SCALE_DYNAMIC, None) == kq.KQ_OK
     # dequant
     d = L.kq_dequant
-    assert d(3, Q, Q, None, None, 4, 4096, 0, P, None) == kq.KQ_ERR_INVALID_ARG
+    assert d(4, Q, Q, None, None, 4, 4096, 0, P, None) == kq.KQ_ERR_INVALID_ARG
     assert d(2, Q, Q, None, None, 4, 4096, 0, P, None) == kq.KQ_ERR_INVALID_ARG
     assert d(1, Q, Q, None, None, 4, 4096, 128, P, None) == kq.KQ_ERR_INVALID_ARG
     assert d(1, Q, Q, Q, None, 4, 4096, 64, P, None) == kq.KQ_ERR_UNSUPPORTED
@@ -101,6 +101,15 @@ def test_argument_errors(L):
     assert L.kq_rht(None, 1, 0, 4096, 0, None, None, 0, None) == kq.KQ_OK
     assert d(2, None, None, None, None, 0, 4096, 0, None, None) == kq.KQ_OK
     assert L.kq_workspace_size(4, 4095, 0) == 0
+    # mxfp4: the rotation's checks, codes 16-byte aligned
+    m = L.kq_rht_quant_mxfp4
+    assert m(P, 1, 0, 4096, 0, None, Q, Q, None) == kq.KQ_OK
+    assert m(P, 1, 4, 4096, 0, None, None, Q, None) == kq.KQ_ERR_INVALID_ARG
+    assert m(P, 1, 4, 4096, 0, None, Q, None, None) == kq.KQ_ERR_INVALID_ARG
+    assert m(P, 1, 4, 4096, 0, None, Q + 8, Q, None) == kq.KQ_ERR_MISALIGNED
+    assert m(P, 1, 4, 4095, 0, None, Q, Q, None) == kq.KQ_ERR_UNSUPPORTED
+    assert m(P, 3, 4, 4096, 0, None, Q, Q, None) == kq.KQ_ERR_UNSUPPORTED
+    assert d(3, Q, Q + 1, None, None, 0, 4096, 0, P, None) == kq.KQ_OK
     # dequant + inverse rotation: the rotation's shape checks, then dequant's
     r = L.kq_dequant_rht_inverse
     assert r(2, Q, Q, None, P, 4, 4096, 0, 0, None, P, 2, None) == kq.KQ_ERR_UNSUPPORTED

@@ -315,3 +315,48 @@ def test_full_size_dequant_rht_inverse_c4():
     winv = wl.Workload("inv", w.tokens, w.dim, wl.F32, w.block, True, w.fmt, 0)
     two = P.gpu_rht(wl.Inputs(winv, deq.astype(np.float64), deq, ci.signs), inverse=True)
     P.check_rotation(got, two.astype(np.float64))
+
+
+# ------------------------------------------------------------------ MXFP4
+@pytest.mark.parametrize("key,tokens,block,dtype", [
+    ("c4", 37, 0, None),          # full 4096 rotation, bf16
+    ("c2", 37, 128, None),        # block-128 rotation
+    ("c3", 9, 0, None),           # H12 x H1024
+    ("c1", 37, 0, None),          # fp32 input
+    ("c4", 11, 32, None),         # Hadamard block = MX block
+])
+def test_mxfp4_parity(key, tokens, block, dtype):
+    inp = small_inputs(key, tokens)
+    w0 = inp.workload
+    w = wl.Workload(w0.key, w0.tokens, w0.dim, w0.dtype, block if block else w0.block,
+                    w0.use_signs, wl.NVFP4, w0.seed)
+    inp = P.inputs_from_values(w, inp.values, inp.signs)
+    y = oracle.rht(inp.values, inp.signs, w.block)
+    codes, scales = P.gpu_mxfp4(inp)
+    P.check_mxfp4(codes, scales, y)
+    deq = P.gpu_dequant(kq.KQ_FMT_MXFP4, codes, scales, None, None, w.tokens, w.dim)
+    want = oracle.dequant_mxfp4(oracle.unpack_nibbles(codes), scales)
+    assert np.array_equal(deq.view(np.uint32), want.view(np.uint32))
+
+
+def test_mxfp4_round_trip_fused():
+    inp = small_inputs("c4", 37)
+    w = inp.workload
+    y = oracle.rht(inp.values, inp.signs, w.block)
+    codes, sc = oracle.mxfp4(y)
+    ci = wl.CodedInputs(w.with_tokens(inp.values.shape[0]), oracle.pack_nibbles(codes), sc,
+                        None, None, inp.signs)
+    wmx = wl.Workload(w.key, ci.workload.tokens, w.dim, w.dtype, w.block, True, "mxfp4", 0)
+    ci = wl.CodedInputs(wmx, ci.codes, ci.scales, None, None, inp.signs)
+    got = P.gpu_dequant_rht_inverse(ci)
+    deq = oracle.dequant_mxfp4(codes, sc).astype(np.float64)
+    P.check_rotation(got, oracle.rht_inverse(deq, inp.signs, w.block))
+
+
+def test_full_size_mxfp4_c4():
+    w = wl.WORKLOADS["c4"]
+    inp = wl.make_inputs(w)
+    rows = _sample_rows(w.tokens, 96, 7)
+    codes, scales = P.gpu_mxfp4(inp)
+    y = oracle.rht(inp.values[rows], inp.signs, w.block)
+    P.check_mxfp4(codes[rows], scales[rows], y)
