@@ -210,8 +210,10 @@ KQ_API kq_status kq_rht_quant_mxfp4(const void* x, int dtype, int64_t tokens, in
   if (tokens > 0 && (!codes || !scales)) return KQ_ERR_INVALID_ARG;
   if (!aligned(codes, 16)) return KQ_ERR_MISALIGNED;
   if (tokens == 0) return KQ_OK;
-  return finish(kq::launch_mxfp4(x, dtype, tokens, g, signs, codes, scales,
-                                 reinterpret_cast<cudaStream_t>(stream)));
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (kq::tc_row_supported(g, dtype, x, tokens))
+    return finish(kq::launch_tc_mxfp4(x, tokens, g, signs, codes, scales, s));
+  return finish(kq::launch_mxfp4(x, dtype, tokens, g, signs, codes, scales, s));
 }
 
 KQ_API kq_status kq_dequant(int fmt, const uint8_t* codes, const void* scales,

@@ -89,7 +89,7 @@ constexpr int kBoundFloats = kBRing * kTok * 2;
 
 __device__ unsigned int g_tc_error = 0;        // nonzero: a wait timed out
 
-enum { kNvfp4 = 0, kNvStats = 1, kRot = 2 };
+enum { kNvfp4 = 0, kNvStats = 1, kRot = 2, kMxfp4 = 3 };
 
 struct Params {
   const uint16_t* x;            // bf16 [T, n]: read by the exact fix-ups
@@ -176,11 +176,11 @@ __device__ __noinline__ double warp_exact_S_ieee(const uint16_t* __restrict__ ro
 // stores a provisional scale and codes and hands the block to the fix-up
 // warp, which decides the scale exactly and rewrites both.
 struct FixEntry {
-  float v[16];        // the block's S_hat values
+  float v[32];        // the block's S_hat values (16 for NVFP4, 32 for MXFP4)
   float bm;           // max |S_hat| of the block
   float E;            // |S_hat - S| <= E (per output of the token)
   long long token;
-  int block;          // 16-element block index within the row
+  int block;          // block index within the row (16 or 32 elements)
   int pad_;
 };
 struct FixQueue {
@@ -195,6 +195,36 @@ struct FixQueue {
 // bound and position); kept out of line so that the epilogue's hot path
 // carries none of it.  If no slot frees up within the wait limit the block
 // keeps its provisional scale and the error word records it.
+// The same for a 32-element MXFP4 block (its 16 S_hat pairs).
+__device__ __noinline__ void enqueue_fix32(FixQueue* fq, long long token, int block, float bm,
+                                           float E, float2 a0, float2 a1, float2 a2, float2 a3,
+                                           float2 a4, float2 a5, float2 a6, float2 a7,
+                                           float2 a8, float2 a9, float2 a10, float2 a11,
+                                           float2 a12, float2 a13, float2 a14, float2 a15) {
+  const unsigned int slot = atomicAdd(&fq->tail, 1u);
+  const long long t0 = clock64();
+  while (slot >= (unsigned int)kQ && ld_acquire(&fq->cons[slot % kQ]) != slot - kQ + 1) {
+    if (clock64() - t0 > kWaitCycles) {
+      atomicOr(&g_tc_error, 2u);
+      return;
+    }
+    __nanosleep(64);
+  }
+  FixEntry& fe = fq->e[slot % kQ];
+  const float2 a[16] = {a0, a1, a2, a3, a4, a5, a6, a7, a8, a9, a10, a11, a12, a13, a14, a15};
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    fe.v[2 * i] = a[i].x;
+    fe.v[2 * i + 1] = a[i].y;
+  }
+  fe.bm = bm;
+  fe.E = E;
+  fe.token = token;
+  fe.block = block;
+  __threadfence_block();       // the provisional stores come first
+  st_release(&fq->seq[slot % kQ], slot + 1);
+}
+
 __device__ __noinline__ void enqueue_fix(FixQueue* fq, long long token, int block, float bm,
                                          float E, float a0, float a1, float a2, float a3,
                                          float a4, float a5, float a6, float a7, float a8,
@@ -219,6 +249,38 @@ __device__ __noinline__ void enqueue_fix(FixQueue* fq, long long token, int bloc
   fe.block = block;
   __threadfence_block();       // the provisional stores come first
   st_release(&fq->seq[slot % kQ], slot + 1);
+}
+
+// MXFP4 of 4096-wide rows (y = S / 64): the E8M0 exponent of a 32-block from
+// an fp32 value m on the scale of max |S|, e = floor(log2(m / 64)) - 2
+// clamped to [-127, 127] (OCP MX: 2 is the largest E2M1 exponent); m <= 0
+// or subnormal gives -127.  Monotone in m.
+__device__ __forceinline__ int mx_exp_s4096(float m) {
+  if (!(m > 0.0f)) return -127;
+  const int ex = (int)((__float_as_uint(m) >> 23) & 0xffu);
+  if (ex == 0) return -127;
+  const int e = ex - 127 - 8;
+  return e < -127 ? -127 : (e > 127 ? 127 : e);
+}
+// E2M1 codes of a 32-block (v: 16 pairs) for exponent e: v * 2^-(e+6), an
+// exact scaling, rounded by the conversion (nearest even, satfinite); -0
+// becomes +0.  Four words, element k in bits 4k..4k+3 of word k / 8.
+__device__ __forceinline__ void mx_block_words(const float2* v, int e, uint32_t (&w)[4]) {
+  int k = 121 - e;                                       // biased exponent of 2^-(e+6)
+  k = k < 1 ? 1 : (k > 254 ? 254 : k);
+  const float f = __uint_as_float((uint32_t)k << 23);
+  const float2 f2 = make_float2(f, f), zero2 = make_float2(0.0f, 0.0f);
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    float qv[8];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      const float2 a = fma2(v[4 * g + p], f2, zero2);
+      qv[2 * p] = a.x;
+      qv[2 * p + 1] = a.y;
+    }
+    w[g] = e2m1x8_hw(qv);
+  }
 }
 
 // E2M1 codes of one 16-element block (v: 8 pairs) for the E4M3 scale `code`:
@@ -612,6 +674,26 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
           continue;
         }
 
+        if (kMode == kMxfp4) {
+          // ---- MXFP4: the thread's 32 outputs are one block; its exponent
+          // is decided when both ends of [max - E, max + E] give the same,
+          // else stored provisionally and finished by the fix-up warps
+          const float bmx = fmaxf(bm[0], bm[1]);
+          const int elo = mx_exp_s4096(__fsub_rd(bmx, E));
+          const int ehi = mx_exp_s4096(__fadd_ru(bmx, E));
+          uint32_t words[4];
+          mx_block_words(v, elo, words);
+          if (valid) {
+            *reinterpret_cast<uint4*>(P.codes + token * (N / 2) + o * 16) =
+                make_uint4(words[0], words[1], words[2], words[3]);
+            P.scales8[token * (N / 32) + o] = (uint8_t)(elo + 127);
+            if (elo != ehi)
+              enqueue_fix32(fq, token, o, bmx, E, v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7],
+                            v[8], v[9], v[10], v[11], v[12], v[13], v[14], v[15]);
+          }
+          continue;
+        }
+
         // ---- NVFP4 block scales; a block whose scale the bound leaves
         // undecided is stored provisionally and finished by the fix-up warp
         uint32_t sc = 0, undecided = 0;
@@ -652,19 +734,57 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
   } else {
     // ================= fix-up warps: exact scales of the queued blocks; fix-up
     // warp f takes entries f, f + kFixWarps, ...
-    if (kMode == kNvfp4) {
+    if (kMode == kNvfp4 || kMode == kMxfp4) {
       float ts = 0.0f, inv_bt = 0.0f;
-      if (P.ws) {
-        const double gm = __longlong_as_double((long long)P.ws->gmax_bits);
-        ts = __double2float_rn((gm / kSqrtN) / 2688.0);
-      } else {
-        ts = *P.tensor_scale;
+      if (kMode == kNvfp4) {
+        if (P.ws) {
+          const double gm = __longlong_as_double((long long)P.ws->gmax_bits);
+          ts = __double2float_rn((gm / kSqrtN) / 2688.0);
+        } else {
+          ts = *P.tensor_scale;
+        }
+        inv_bt = (ts > 0.0f) ? (float)(1.0 / (kSqrtN * (double)ts)) : 0.0f;
       }
-      inv_bt = (ts > 0.0f) ? (float)(1.0 / (kSqrtN * (double)ts)) : 0.0f;
       unsigned int h = (unsigned int)(warp - kFixWarp);
       long long idle0 = clock64();
       for (;;) {
-        if (ld_acquire(&fq->seq[h % kQ]) == h + 1) {
+        if (kMode == kMxfp4 && ld_acquire(&fq->seq[h % kQ]) == h + 1) {
+          // MXFP4 block of 32: exact max |S| over the candidates, exponent
+          // floor(log2(max / 64)) - 2 (clamped), codes from the queued S_hat
+          const FixEntry& fe = fq->e[h % kQ];
+          const float thr = fe.bm - 2.0f * fe.E;
+          const bool finite = isfinite(fe.E);
+          uint32_t cand = __ballot_sync(0xffffffffu, fabsf(fe.v[lane]) >= thr);
+          const long long token = fe.token;
+          const int blk = fe.block;
+          double best = 0.0;
+          while (cand) {
+            const int e = __ffs(cand) - 1;
+            cand &= cand - 1;
+            const int ii = blk * 32 + e;
+            best = fmax(best, fabs(finite
+                ? warp_exact_S(reinterpret_cast<const uint4*>(P.x + token * N), smask, ii)
+                : warp_exact_S_ieee(P.x + token * N, signs, ii)));
+          }
+          int ex = -127;
+          if (best > 0.0) {
+            ex = ilogb(best / kSqrtN) - 2;
+            ex = ex < -127 ? -127 : (ex > 127 ? 127 : ex);
+          }
+          if (lane == 0) {
+            uint32_t w[4];
+            mx_block_words(reinterpret_cast<const float2*>(fe.v), ex, w);
+            *reinterpret_cast<uint4*>(P.codes + token * (N / 2) + blk * 16) =
+                make_uint4(w[0], w[1], w[2], w[3]);
+            P.scales8[token * (N / 32) + blk] = (uint8_t)(ex + 127);
+          }
+          __syncwarp();
+          if (lane == 0) st_release(&fq->cons[h % kQ], h + 1);
+          h += kFixWarps;
+          idle0 = clock64();
+          continue;
+        }
+        if (kMode == kNvfp4 && ld_acquire(&fq->seq[h % kQ]) == h + 1) {
           const FixEntry& fe = fq->e[h % kQ];
           const float thr = fe.bm - 2.0f * fe.E;
           const bool finite = isfinite(fe.E);   // sum|x| finite: every input finite
@@ -870,6 +990,18 @@ cudaError_t launch_tc_nvfp4(const void* x, int64_t tokens, const Geometry& g,
     if (e != cudaSuccess) return e;
   }
   return launch_tc<tc::kNvfp4>(x, signs, P, s);
+}
+
+cudaError_t launch_tc_mxfp4(const void* x, int64_t tokens, const Geometry& g,
+                            const int8_t* signs, uint8_t* codes, uint8_t* scales,
+                            cudaStream_t s) {
+  tc::Params P{};
+  P.x = static_cast<const uint16_t*>(x);
+  P.codes = codes;
+  P.scales8 = scales;
+  P.tokens = tokens;
+  (void)g;
+  return launch_tc<tc::kMxfp4>(x, signs, P, s);
 }
 
 cudaError_t launch_tc_rot(const void* x, int64_t tokens, const Geometry& g, const int8_t* signs,
