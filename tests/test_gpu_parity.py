@@ -128,7 +128,8 @@ def test_int4_asym_block128_shapes(dim, tokens, signs):
 
 
 # --------------------------------------------------------------- NVFP4
-@pytest.mark.parametrize("key,tokens", [("c2", 37), ("c4", 37)])
+@pytest.mark.parametrize("key,tokens", [("c2", 37), ("c4", 37), ("c2", 4 * 148 * 6 + 1),
+                                        ("c2", 3)])
 def test_nvfp4_small_dynamic_and_static(key, tokens):
     inp = small_inputs(key, tokens)
     w = inp.workload
@@ -166,8 +167,9 @@ def test_nvfp4_round_trip_c4_small():
     assert np.all(err <= np.sqrt(np.sum(unit ** 2, axis=1)) * 1.0001 + 1e-30)
 
 
-def test_nvfp4_all_zero_tensor():
-    w = wl.WORKLOADS["c4"].with_tokens(5)
+@pytest.mark.parametrize("key", ["c2", "c4"])
+def test_nvfp4_all_zero_tensor(key):
+    w = wl.WORKLOADS[key].with_tokens(5)
     vals = np.zeros((5, 4096))
     inp = P.inputs_from_values(w, vals, wl.make_inputs(w).signs)
     codes, bs, ts = P.gpu_nvfp4(inp)
