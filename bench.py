@@ -271,6 +271,28 @@ def run_cpu_baseline(w, seconds):
     }
 
 
+# ------------------------------------------------------------ multi-rank
+def rank_seed(w, rank):
+    """Seed of rank `rank`'s batch: every rank draws its own (weak scaling)."""
+    return w.seed + 1000 * rank
+
+
+def max_over_ranks(torch, dist, value, device):
+    """The maximum of a per-rank float over all ranks (the job's time is the
+    slowest rank's); `value` itself without a process group."""
+    if dist is None:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(bytes_per_rank, world, ms_per_step):
+    """GB/s of the whole job: every rank moves bytes_per_rank per step, and
+    the step lasts ms_per_step (the slowest rank's)."""
+    return bytes_per_rank * world / (ms_per_step * 1e-3) / 1e9
+
+
 def run_reference(args, rank, world):
     """--impl reference: the CPU oracle, timed on the host cores."""
     if rank != 0:
@@ -360,7 +382,7 @@ def main():
             dist.destroy_process_group()
         return
     # every rank draws its own batch (weak scaling)
-    inp = wl.make_inputs(w, seed=w.seed + 1000 * rank)
+    inp = wl.make_inputs(w, seed=rank_seed(w, rank))
     x0 = device_input(torch, inp, wl, dev)
     signs = None if inp.signs is None else torch.from_numpy(inp.signs).to(dev)
 
@@ -386,13 +408,11 @@ def main():
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
-        tt = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(torch, dist, ms, dev)
     ms_step = ms / max(args.steps, 1)
     alg = w.algorithmic_bytes()
     gbs_rank = alg / (ms_step * 1e-3) / 1e9
-    value = gbs_rank * world
+    value = whole_job_gbs(alg, world, ms_step)
     tokens_s = w.tokens * world / (ms_step * 1e-3)
 
     # ---- end to end through the public API: pinned host in, host out
@@ -413,11 +433,8 @@ def main():
 
     k_e2e = max(3, min(args.steps, 50))
     ms_e2e = time_steps(torch, e2e_step, [None], k_e2e, max(3, min(args.warmup, 5)))
-    if dist is not None:
-        tt = torch.tensor([ms_e2e], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_e2e = float(tt.item())
-    e2e_gbs = alg * world / (ms_e2e / k_e2e * 1e-3) / 1e9
+    ms_e2e = max_over_ranks(torch, dist, ms_e2e, dev)
+    e2e_gbs = whole_job_gbs(alg, world, ms_e2e / k_e2e)
 
     kernel_key = f"{w.key}_{w.fmt}_static" if w.fmt == wl.NVFP4 else f"{w.key}_{w.fmt}"
     traffic = ncu_traffic(kernel_key)
