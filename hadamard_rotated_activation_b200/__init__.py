@@ -38,7 +38,7 @@ KQ_FMT_MXFP4 = 3
 
 C_SYMBOLS = (
     "kq_rht", "kq_rht_quant_int4", "kq_rht_quant_nvfp4", "kq_dequant",
-    "kq_dequant_rht_inverse", "kq_rht_quant_mxfp4",
+    "kq_dequant_rht_inverse", "kq_rht_quant_mxfp4", "kq_rht_quant_int4_kv",
     "kq_workspace_size", "kq_status_str", "kq_last_cuda_error", "kq_version",
     "kq_rht_quant_nvfp4_dynamic_noalloc", "kq_diag_tc_steps",
 )
@@ -80,6 +80,8 @@ def lib() -> ctypes.CDLL:
     L.kq_dequant.restype = i32
     L.kq_rht_quant_mxfp4.argtypes = [vp, i32, i64, i32, i32, vp, vp, vp, vp]
     L.kq_rht_quant_mxfp4.restype = i32
+    L.kq_rht_quant_int4_kv.argtypes = [vp, i32, i64, i32, i32, vp, i32, vp, i64, vp, vp, vp, vp]
+    L.kq_rht_quant_int4_kv.restype = i32
     L.kq_dequant_rht_inverse.argtypes = [i32, vp, vp, vp, vp, i64, i32, i32, i32, vp, vp, i32,
                                          vp]
     L.kq_dequant_rht_inverse.restype = i32
@@ -170,6 +172,18 @@ def kq_rht_quant_nvfp4(x, block: int, signs, codes, block_scales, tensor_scale,
                                     _ptr(codes), _ptr(block_scales), _ptr(tensor_scale),
                                     _ptr(workspace), ws_bytes, flags, _stream(stream)),
            "kq_rht_quant_nvfp4")
+
+
+def kq_rht_quant_int4_kv(x, signs, slot_mapping, codes_cache, scales_cache, zeros_cache,
+                         stream=None) -> None:
+    """Rotation (per-head H_128) + asymmetric INT4 g128 into KV-cache rows:
+    token t lands in row slot_mapping[t] (int64; negative = skip)."""
+    t, n = x.shape
+    _check(lib().kq_rht_quant_int4_kv(_ptr(x), _dtype_code(x), t, n, 128, _ptr(signs), 128,
+                                      _ptr(slot_mapping), codes_cache.shape[0],
+                                      _ptr(codes_cache), _ptr(scales_cache), _ptr(zeros_cache),
+                                      _stream(stream)),
+           "kq_rht_quant_int4_kv")
 
 
 def kq_rht_quant_mxfp4(x, block: int, signs, codes, scales, stream=None) -> None:

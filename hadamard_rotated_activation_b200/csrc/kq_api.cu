@@ -146,11 +146,11 @@ KQ_API kq_status kq_rht_quant_int4(const void* x, int dtype, int64_t tokens, int
   if (asym == 1 && kq::tcb_supported(g, dtype, x, tokens))
     return finish(kq::launch_tcb_asym(x, tokens, g, signs, codes,
                                       static_cast<uint16_t*>(scales),
-                                      static_cast<uint16_t*>(zeros), s));
+                                      static_cast<uint16_t*>(zeros), nullptr, 0, s));
   if (asym == 1 && kq::blk128_supported(g, dtype) && aligned(signs, 16))
     return finish(kq::launch_blk128_asym(x, tokens, g, signs, codes,
                                          static_cast<uint16_t*>(scales),
-                                         static_cast<uint16_t*>(zeros), s));
+                                         static_cast<uint16_t*>(zeros), nullptr, 0, s));
   if (asym == 0 && kq::tcp_supported(g, dtype, x, tokens) && aligned(signs, 8))
     return finish(kq::launch_tcp_int4(x, tokens, g, signs, codes, static_cast<float*>(scales),
                                       s));
@@ -163,6 +163,32 @@ KQ_API kq_status kq_rht_quant_int4(const void* x, int dtype, int64_t tokens, int
   return finish(kq::launch_int4_asym(x, dtype, tokens, g, signs, group, codes,
                                      static_cast<uint16_t*>(scales),
                                      static_cast<uint16_t*>(zeros), s));
+}
+
+KQ_API kq_status kq_rht_quant_int4_kv(const void* x, int dtype, int64_t tokens, int dim,
+                                      int block, const int8_t* signs, int group,
+                                      const int64_t* slot_mapping, int64_t num_slots,
+                                      uint8_t* codes_cache, uint16_t* scales_cache,
+                                      uint16_t* zeros_cache, kq_stream_t stream) {
+  kq::Geometry g;
+  kq_status st = check_common(x, dtype, tokens, dim, block, signs, &g);
+  if (st != KQ_OK) return st;
+  if (num_slots < 0) return KQ_ERR_INVALID_ARG;
+  if (tokens > 0 && (!slot_mapping || !codes_cache || !scales_cache || !zeros_cache))
+    return KQ_ERR_INVALID_ARG;
+  if (dtype != KQ_BF16 || group != 128 || g.b != 128 || g.paley) return KQ_ERR_UNSUPPORTED;
+  if (!aligned(codes_cache, 16) || !aligned(scales_cache, 2) || !aligned(zeros_cache, 2) ||
+      !aligned(slot_mapping, 8) || !aligned(signs, 16))
+    return KQ_ERR_MISALIGNED;
+  if (tokens == 0) return KQ_OK;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (kq::tcb_supported(g, dtype, x, tokens))
+    return finish(kq::launch_tcb_asym(x, tokens, g, signs, codes_cache, scales_cache,
+                                      zeros_cache, slot_mapping, num_slots, s));
+  if (kq::blk128_supported(g, dtype))
+    return finish(kq::launch_blk128_asym(x, tokens, g, signs, codes_cache, scales_cache,
+                                         zeros_cache, slot_mapping, num_slots, s));
+  return KQ_ERR_UNSUPPORTED;
 }
 
 KQ_API kq_status kq_rht_quant_nvfp4(const void* x, int dtype, int64_t tokens, int dim,

@@ -39,6 +39,8 @@ struct Params {
   float* tensor_scale;          // NVFP4 t (device): read if static, written if dynamic
   NvWorkspace* ws;              // NVFP4 dynamic: gmax (read) / row stats (written)
   int64_t units;                // T * n / 128
+  const int64_t* slots;         // asym: cache row of each input row, or null
+  int64_t num_slots;
   int n;
   float e_coef;                 // E = e_coef * max|S_hat| (rounded up)
 };
@@ -487,7 +489,8 @@ k_blk128_asym(Params P) {
     // (S c) + (1.5 2^23 + z) rounds S c + z to an integer in the low bits
     const float magic = 12582912.0f + zf;
     const float2 m2 = make_float2(magic, magic);
-    uint4* dst = reinterpret_cast<uint4*>(P.codes + u * (B / 2));
+    const int64_t ou = active ? kv_unit(P.slots, P.num_slots, kpr, u) : -1;
+    uint4* dst = reinterpret_cast<uint4*>(P.codes + ou * (B / 2));
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       uint32_t words[4];
@@ -502,13 +505,13 @@ k_blk128_asym(Params P) {
         }
         words[w] = pack_u4x8(q);
       }
-      if (active) dst[k] = make_uint4(words[0], words[1], words[2], words[3]);
+      if (ou >= 0) dst[k] = make_uint4(words[0], words[1], words[2], words[3]);
     }
-    if (active) {
+    if (ou >= 0) {
       uint16_t zh;
       asm("cvt.rn.f16.f32 %0, %1;" : "=h"(zh) : "f"(zf));
-      P.scales16[u] = (uint16_t)s16;
-      P.zeros16[u] = zh;
+      P.scales16[ou] = (uint16_t)s16;
+      P.zeros16[ou] = zh;
     }
   }
 }
@@ -577,13 +580,16 @@ cudaError_t launch_blk128_nvfp4(const void* x, int64_t tokens, const Geometry& g
 
 cudaError_t launch_blk128_asym(const void* x, int64_t tokens, const Geometry& g,
                                const int8_t* signs, uint8_t* codes, uint16_t* scales,
-                               uint16_t* zeros, cudaStream_t s) {
+                               uint16_t* zeros, const int64_t* slots, int64_t num_slots,
+                               cudaStream_t s) {
   blk::Params P{};
   P.x = static_cast<const uint16_t*>(x);
   P.signs = signs;
   P.codes = codes;
   P.scales16 = scales;
   P.zeros16 = zeros;
+  P.slots = slots;
+  P.num_slots = num_slots;
   P.units = tokens * (g.n / blk::B);
   P.n = g.n;
   P.e_coef = e_coef_128();

@@ -69,6 +69,19 @@ __device__ __forceinline__ bool paley_negative(int a, int c) {
   return (w >> (k & 31)) & 1u;
 }
 
+// ------------------------------------------------------------ KV-cache rows
+// Output unit of input unit u (kpr units of 128 per row) when rows go to the
+// cache rows a slot mapping names: slot[u / kpr] * kpr + u % kpr, or -1 when
+// the row's slot is negative (padding) or not below num_slots; u itself
+// without a mapping.
+__device__ __forceinline__ int64_t kv_unit(const int64_t* slots, int64_t num_slots, int kpr,
+                                           int64_t u) {
+  if (!slots) return u;
+  const int64_t t = u / kpr;
+  const int64_t sl = __ldg(slots + t);
+  return (sl >= 0 && sl < num_slots) ? sl * kpr + (u - t * kpr) : -1;
+}
+
 // ------------------------------------------------------------ transform spec
 struct Geometry {
   int n;          // row length (dim)

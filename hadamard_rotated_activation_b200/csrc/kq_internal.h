@@ -51,7 +51,8 @@ cudaError_t launch_blk128_nvfp4(const void* x, int64_t tokens, const Geometry& g
                                 float* tensor_scale, NvWorkspace* ws, cudaStream_t s);
 cudaError_t launch_blk128_asym(const void* x, int64_t tokens, const Geometry& g,
                                const int8_t* signs, uint8_t* codes, uint16_t* scales,
-                               uint16_t* zeros, cudaStream_t s);
+                               uint16_t* zeros, const int64_t* slots, int64_t num_slots,
+                            cudaStream_t s);
 
 // Warp-per-row kernels for full-row transforms of 2048 or 4096 (kq_rowwarp.cu).
 bool rowwarp_supported(const Geometry& g, int dtype);
@@ -97,7 +98,8 @@ cudaError_t launch_dequant_rht_inv(int fmt, const uint8_t* codes, const void* sc
 bool tcb_supported(const Geometry& g, int dtype, const void* x, int64_t tokens);
 cudaError_t launch_tcb_asym(const void* x, int64_t tokens, const Geometry& g,
                             const int8_t* signs, uint8_t* codes, uint16_t* scales,
-                            uint16_t* zeros, cudaStream_t s);
+                            uint16_t* zeros, const int64_t* slots, int64_t num_slots,
+                            cudaStream_t s);
 // NVFP4 dequant + inverse rotation of 4096-wide rows on the tensor cores.
 bool tci_supported(const Geometry& g, const uint8_t* codes, const uint8_t* scales,
                    const int8_t* signs, const void* out);

@@ -77,6 +77,8 @@ struct Params {
   uint16_t* scales16;           // fp16 [units]
   uint16_t* zeros16;            // fp16 [units]
   int64_t units;                // tokens * n / 128 (>= 128)
+  const int64_t* slots;         // cache row of each input row, or null
+  int64_t num_slots;
   int64_t tiles;
   int kpr;                      // column blocks per row, n / 128
 };
@@ -442,14 +444,15 @@ k_tcb128_asym(const __grid_constant__ CUtensorMap tmap, Params P) {
         const int kc = r4 * 32 + lane, l2 = kc >> 2, p2 = kc & 3;
         const uint4 val =
             *reinterpret_cast<const uint4*>(wbuf + l2 * 64 + ((p2 ^ ((l2 >> 1) & 3)) << 4));
-        if (ub + l2 >= u_lo)
-          *reinterpret_cast<uint4*>(P.codes + (ub + l2) * 64 + p2 * 16) = val;
+        const int64_t ou = ub + l2 >= u_lo ? kv_unit(P.slots, P.num_slots, P.kpr, ub + l2) : -1;
+        if (ou >= 0) *reinterpret_cast<uint4*>(P.codes + ou * 64 + p2 * 16) = val;
       }
-      if (y0 + m >= u_lo) {
+      const int64_t om = y0 + m >= u_lo ? kv_unit(P.slots, P.num_slots, P.kpr, y0 + m) : -1;
+      if (om >= 0) {
         uint16_t zh;
         asm("cvt.rn.f16.f32 %0, %1;" : "=h"(zh) : "f"(zf));
-        P.scales16[y0 + m] = (uint16_t)s16;
-        P.zeros16[y0 + m] = zh;
+        P.scales16[om] = (uint16_t)s16;
+        P.zeros16[om] = zh;
       }
       __syncwarp();
     }
@@ -475,12 +478,15 @@ bool tcb_supported(const Geometry& g, int dtype, const void* x, int64_t tokens) 
 
 cudaError_t launch_tcb_asym(const void* x, int64_t tokens, const Geometry& g,
                             const int8_t* signs, uint8_t* codes, uint16_t* scales,
-                            uint16_t* zeros, cudaStream_t s) {
+                            uint16_t* zeros, const int64_t* slots, int64_t num_slots,
+                            cudaStream_t s) {
   tcb::Params P{};
   P.signs = signs;
   P.codes = codes;
   P.scales16 = scales;
   P.zeros16 = zeros;
+  P.slots = slots;
+  P.num_slots = num_slots;
   P.units = tokens * (g.n / tcb::B);
   P.tiles = (P.units + 127) / 128;
   P.kpr = g.n / tcb::B;

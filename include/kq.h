@@ -146,6 +146,28 @@ KQ_API kq_status kq_rht_quant_int4(const void* x, int dtype, int64_t tokens,
                                    kq_stream_t stream);
 
 /*
+ * kq_rht_quant_int4_kv -- kq_rht_quant_int4 with asym = 1 that writes each
+ * token straight into a KV cache (QuaRot reviews, final comments: the KV
+ * cache at 4 bits with a per-head 128-point Hadamard): token t's codes,
+ * scales and zero points go to cache row slot_mapping[t] instead of row t.
+ * A negative slot skips the token (padding); slots at or above num_slots
+ * are skipped too (nothing is written).  Two tokens with the same slot:
+ * either one's row ends up there.
+ * x: bf16 [tokens, dim]; block = 128 and group = 128 (one Hadamard block per
+ * head); signs: int8[dim] or NULL, 16-byte aligned.  slot_mapping: int64
+ * [tokens] in device memory, 8-byte aligned.  codes_cache: [num_slots, dim/2]
+ * (16-byte aligned); scales_cache, zeros_cache: fp16 [num_slots, dim/128].
+ * Rows not named by the mapping are left as they are.  Errors: as
+ * kq_rht_quant_int4, KQ_ERR_UNSUPPORTED for another dtype, block or group.
+ */
+KQ_API kq_status kq_rht_quant_int4_kv(const void* x, int dtype, int64_t tokens,
+                                      int dim, int block, const int8_t* signs,
+                                      int group, const int64_t* slot_mapping,
+                                      int64_t num_slots, uint8_t* codes_cache,
+                                      uint16_t* scales_cache, uint16_t* zeros_cache,
+                                      kq_stream_t stream);
+
+/*
  * kq_rht_quant_nvfp4 -- rotation fused with NVFP4 quantization (NVFP4 thread,
  * krylov_schur section 3 table: E2M1 codes + one E4M3 scale per 16 elements,
  * 4.50 bits per element; per-tensor fp32 scale).

@@ -101,6 +101,17 @@ def test_argument_errors(L):
     assert L.kq_rht(None, 1, 0, 4096, 0, None, None, 0, None) == kq.KQ_OK
     assert d(2, None, None, None, None, 0, 4096, 0, None, None) == kq.KQ_OK
     assert L.kq_workspace_size(4, 4095, 0) == 0
+    # KV writer: bf16, block 128, group 128; all buffers present and aligned
+    v = L.kq_rht_quant_int4_kv
+    assert v(P, 1, 0, 4096, 128, None, 128, Q, 16, Q, Q, Q, None) == kq.KQ_OK
+    assert v(P, 1, 4, 4096, 128, None, 128, Q, -1, Q, Q, Q, None) == kq.KQ_ERR_INVALID_ARG
+    assert v(P, 1, 4, 4096, 128, None, 128, None, 16, Q, Q, Q, None) == kq.KQ_ERR_INVALID_ARG
+    assert v(P, 0, 4, 4096, 128, None, 128, Q, 16, Q, Q, Q, None) == kq.KQ_ERR_UNSUPPORTED
+    assert v(P, 1, 4, 4096, 0, None, 128, Q, 16, Q, Q, Q, None) == kq.KQ_ERR_UNSUPPORTED
+    assert v(P, 1, 4, 4096, 128, None, 64, Q, 16, Q, Q, Q, None) == kq.KQ_ERR_UNSUPPORTED
+    assert v(P, 1, 4, 4096, 128, None, 128, Q + 4, 16, Q, Q, Q, None) == kq.KQ_ERR_MISALIGNED
+    assert v(P, 1, 4, 4096, 128, P + 8, 128, Q, 16, Q, Q, Q, None) == kq.KQ_ERR_MISALIGNED
+    assert v(P, 1, 4, 4096, 128, None, 128, Q, 16, Q + 8, Q, Q, None) == kq.KQ_ERR_MISALIGNED
     # mxfp4: the rotation's checks, codes 16-byte aligned
     m = L.kq_rht_quant_mxfp4
     assert m(P, 1, 0, 4096, 0, None, Q, Q, None) == kq.KQ_OK

@@ -362,3 +362,33 @@ def test_full_size_mxfp4_c4():
     codes, scales = P.gpu_mxfp4(inp)
     y = oracle.rht(inp.values[rows], inp.signs, w.block)
     P.check_mxfp4(codes[rows], scales[rows], y)
+
+
+# -------------------------------------------------------- KV-cache writer
+@pytest.mark.parametrize("tokens,num_slots", [(43, 64), (3, 8), (4 * 148 * 6 + 3, 4000)])
+def test_kv_cache_writer(tokens, num_slots):
+    """Asymmetric INT4 g128 of per-head H_128 rotations, written to the cache
+    rows a slot mapping names: named rows hold the oracle's result, the rest
+    keep their previous contents."""
+    w = wl.WORKLOADS["c5"].with_tokens(tokens)
+    inp = wl.make_inputs(w)
+    rng = np.random.default_rng(tokens)
+    slots = rng.permutation(num_slots)[:tokens].astype(np.int64) if tokens <= num_slots \
+        else rng.integers(0, num_slots, tokens)
+    slots[rng.random(tokens) < 0.1] = -1                 # padding
+    slots[rng.random(tokens) < 0.05] = num_slots + 3     # out of range: skipped
+    dev = "cuda"
+    x = torch.from_numpy(inp.stored.view(np.int16)).to(dev).view(torch.bfloat16)
+    sm = torch.from_numpy(slots).to(dev)
+    cc = torch.full((num_slots, w.dim // 2), 0xAB, dtype=torch.uint8, device=dev)
+    sc = torch.full((num_slots, w.dim // 128), 7.0, dtype=torch.float16, device=dev)
+    zc = torch.full((num_slots, w.dim // 128), -3.0, dtype=torch.float16, device=dev)
+    kq.kq_rht_quant_int4_kv(x, None, sm, cc, sc, zc)
+    torch.cuda.synchronize()
+    cc, sc, zc = cc.cpu().numpy(), sc.cpu().numpy(), zc.cpu().numpy()
+    ok = (slots >= 0) & (slots < num_slots)
+    y = oracle.rht(inp.values[ok], None, 128)
+    P.check_int4_asym(cc[slots[ok]], sc[slots[ok]], zc[slots[ok]], y)
+    untouched = np.setdiff1d(np.arange(num_slots), slots[ok])
+    assert np.all(cc[untouched] == 0xAB)
+    assert np.all(sc[untouched] == 7.0) and np.all(zc[untouched] == -3.0)
