@@ -39,6 +39,7 @@ KQ_FMT_MXFP4 = 3
 C_SYMBOLS = (
     "kq_rht", "kq_rht_quant_int4", "kq_rht_quant_nvfp4", "kq_dequant",
     "kq_dequant_rht_inverse", "kq_rht_quant_mxfp4", "kq_rht_quant_int4_kv",
+    "kq_device_errors", "kq_diag_wait_timeout",
     "kq_workspace_size", "kq_status_str", "kq_last_cuda_error", "kq_version",
     "kq_rht_quant_nvfp4_dynamic_noalloc", "kq_diag_tc_steps",
 )
@@ -82,6 +83,10 @@ def lib() -> ctypes.CDLL:
     L.kq_rht_quant_mxfp4.restype = i32
     L.kq_rht_quant_int4_kv.argtypes = [vp, i32, i64, i32, i32, vp, i32, vp, i64, vp, vp, vp, vp]
     L.kq_rht_quant_int4_kv.restype = i32
+    L.kq_device_errors.argtypes = [vp]
+    L.kq_device_errors.restype = i32
+    L.kq_diag_wait_timeout.argtypes = [ctypes.c_longlong, vp]
+    L.kq_diag_wait_timeout.restype = i32
     L.kq_dequant_rht_inverse.argtypes = [i32, vp, vp, vp, vp, i64, i32, i32, i32, vp, vp, i32,
                                          vp]
     L.kq_dequant_rht_inverse.restype = i32
@@ -229,6 +234,21 @@ def kq_diag_tc_steps(a, b, d1, d2, status, stream=None) -> None:
     status one int32 (0 = the waits completed)."""
     _check(lib().kq_diag_tc_steps(_ptr(a), _ptr(b), _ptr(d1), _ptr(d2), _ptr(status),
                                   _stream(stream)), "kq_diag_tc_steps")
+
+
+def kq_device_errors():
+    """The five error words of the tensor-core kernel families (read and
+    cleared): 4096-wide, 12288-wide, block-128 GEMM, fused inverse,
+    diagnostic.  All zero: no bounded wait ran out since the last call."""
+    buf = (ctypes.c_uint * 5)()
+    _check(lib().kq_device_errors(buf), "kq_device_errors")
+    return list(buf)
+
+
+def kq_diag_wait_timeout(limit_cycles: int, stream=None) -> None:
+    """Diagnostic: a wait that nothing satisfies, bounded by limit_cycles."""
+    _check(lib().kq_diag_wait_timeout(int(limit_cycles), _stream(stream)),
+           "kq_diag_wait_timeout")
 
 
 def kq_workspace_size(tokens: int, dim: int, block: int) -> int:

@@ -279,6 +279,21 @@ KQ_API kq_status kq_dequant_rht_inverse(int fmt, const uint8_t* codes, const voi
                                            group, signs, out, bf16, s));
 }
 
+KQ_API kq_status kq_device_errors(unsigned int* flags) {
+  if (!flags) return KQ_ERR_INVALID_ARG;
+  cudaError_t e = kq::take_tc_errors(&flags[0]);
+  if (e == cudaSuccess) e = kq::take_tcp_errors(&flags[1]);
+  if (e == cudaSuccess) e = kq::take_tcb_errors(&flags[2]);
+  if (e == cudaSuccess) e = kq::take_tci_errors(&flags[3]);
+  if (e == cudaSuccess) e = kq::take_diag_errors(&flags[4]);
+  return finish(e);
+}
+
+KQ_API kq_status kq_diag_wait_timeout(long long limit_cycles, kq_stream_t stream) {
+  if (limit_cycles <= 0 || limit_cycles > 4000000000ll) return KQ_ERR_INVALID_ARG;
+  return finish(kq::launch_diag_wait(limit_cycles, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 KQ_API size_t kq_workspace_size(int64_t tokens, int dim, int block) {
   kq::Geometry g;
   if (tokens < 0 || make_geometry(dim, block, &g) != KQ_OK) return 0;

@@ -107,4 +107,12 @@ cudaError_t launch_tcinv_nvfp4(const uint8_t* codes, const uint8_t* scales,
                                const float* tensor_scale, int64_t tokens, const Geometry& g,
                                const int8_t* signs, void* out, int out_bf16, cudaStream_t s);
 
+// Error words of the kernel families (read and cleared; device-synchronous).
+cudaError_t take_tc_errors(unsigned int* out);
+cudaError_t take_tcp_errors(unsigned int* out);
+cudaError_t take_tcb_errors(unsigned int* out);
+cudaError_t take_tci_errors(unsigned int* out);
+cudaError_t take_diag_errors(unsigned int* out);
+cudaError_t launch_diag_wait(long long limit_cycles, cudaStream_t s);
+
 }  // namespace kq

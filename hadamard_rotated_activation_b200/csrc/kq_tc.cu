@@ -1029,4 +1029,12 @@ int tc_error_flag() {
   return (int)v;
 }
 
+// Reads and clears the error word of the tc kernels (device-synchronous).
+cudaError_t take_tc_errors(unsigned int* out) {
+  const unsigned int zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(out, tc::g_tc_error, sizeof(unsigned int));
+  if (e != cudaSuccess) return e;
+  return cudaMemcpyToSymbol(tc::g_tc_error, &zero, sizeof(unsigned int));
+}
+
 }  // namespace kq

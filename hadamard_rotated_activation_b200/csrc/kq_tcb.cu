@@ -506,4 +506,12 @@ cudaError_t launch_tcb_asym(const void* x, int64_t tokens, const Geometry& g,
   return cudaGetLastError();
 }
 
+// Reads and clears the error word of the tcb kernels (device-synchronous).
+cudaError_t take_tcb_errors(unsigned int* out) {
+  const unsigned int zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(out, tcb::g_tcb_error, sizeof(unsigned int));
+  if (e != cudaSuccess) return e;
+  return cudaMemcpyToSymbol(tcb::g_tcb_error, &zero, sizeof(unsigned int));
+}
+
 }  // namespace kq

@@ -398,4 +398,12 @@ cudaError_t launch_tcinv_nvfp4(const uint8_t* codes, const uint8_t* scales,
   return cudaGetLastError();
 }
 
+// Reads and clears the error word of the tci kernels (device-synchronous).
+cudaError_t take_tci_errors(unsigned int* out) {
+  const unsigned int zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(out, tci::g_tci_error, sizeof(unsigned int));
+  if (e != cudaSuccess) return e;
+  return cudaMemcpyToSymbol(tci::g_tci_error, &zero, sizeof(unsigned int));
+}
+
 }  // namespace kq

@@ -619,4 +619,12 @@ cudaError_t launch_tcp_rot(const void* x, int64_t tokens, const Geometry& g,
   return launch_tcp<tcp::kRot>(x, signs, P, g, s);
 }
 
+// Reads and clears the error word of the tcp kernels (device-synchronous).
+cudaError_t take_tcp_errors(unsigned int* out) {
+  const unsigned int zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(out, tcp::g_tcp_error, sizeof(unsigned int));
+  if (e != cudaSuccess) return e;
+  return cudaMemcpyToSymbol(tcp::g_tcp_error, &zero, sizeof(unsigned int));
+}
+
 }  // namespace kq

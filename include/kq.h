@@ -246,6 +246,29 @@ KQ_API kq_status kq_dequant_rht_inverse(int fmt, const uint8_t* codes,
                                         int out_dtype, kq_stream_t stream);
 
 /*
+ * kq_device_errors -- failure reports of the tensor-core kernels.  Every
+ * wait of those kernels is bounded (about two seconds); when one runs out the
+ * kernel records it in its family's error word and returns without writing
+ * the affected outputs, instead of hanging.  flags: host array of 5 words,
+ * filled and then cleared on the device: [0] the 4096-wide kernels (bit 0: a
+ * wait ran out; bit 1: the fix-up queue stayed full, a block kept its
+ * provisional scale; bit 2: a fix-up warp waited too long), [1] the
+ * 12288-wide kernel, [2] the block-128 GEMM kernel, [3] the fused dequant +
+ * inverse kernel, [4] kq_diag_wait_timeout (bit 0).  All zero: no failure
+ * since the last call.  The read synchronizes the device.  The pages have no
+ * counterpart to this entry point.
+ */
+KQ_API kq_status kq_device_errors(unsigned int* flags);
+
+/*
+ * kq_diag_wait_timeout -- diagnostic, no page counterpart: one CTA waits on
+ * a barrier that nothing arrives at, with a limit of limit_cycles clock
+ * cycles (1 .. 4e9), then sets bit 0 of word [4] of kq_device_errors and
+ * exits.  It exercises the bounded-wait failure path without any fault.
+ */
+KQ_API kq_status kq_diag_wait_timeout(long long limit_cycles, kq_stream_t stream);
+
+/*
  * kq_rht_quant_nvfp4_dynamic_noalloc -- kq_rht_quant_nvfp4 with
  * KQ_SCALE_DYNAMIC, for callers that cannot allocate device memory.  The
  * pages have no counterpart to this entry point; it exists for integration.

@@ -101,6 +101,9 @@ def test_argument_errors(L):
     assert L.kq_rht(None, 1, 0, 4096, 0, None, None, 0, None) == kq.KQ_OK
     assert d(2, None, None, None, None, 0, 4096, 0, None, None) == kq.KQ_OK
     assert L.kq_workspace_size(4, 4095, 0) == 0
+    assert L.kq_device_errors(None) == kq.KQ_ERR_INVALID_ARG
+    assert L.kq_diag_wait_timeout(0, None) == kq.KQ_ERR_INVALID_ARG
+    assert L.kq_diag_wait_timeout(5_000_000_000, None) == kq.KQ_ERR_INVALID_ARG
     # KV writer: bf16, block 128, group 128; all buffers present and aligned
     v = L.kq_rht_quant_int4_kv
     assert v(P, 1, 0, 4096, 128, None, 128, Q, 16, Q, Q, Q, None) == kq.KQ_OK
