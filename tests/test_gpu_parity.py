@@ -66,8 +66,13 @@ def test_rotation_other_shapes(dim, block, dtype):
     w = wl.Workload("x", 9, dim, dtype, block, True, wl.INT4_SYM, 0)
     inp = P.inputs_from_values(w, x, s)
     P.check_rotation(P.gpu_rht(inp), oracle.rht(x, s, block))
+    y = oracle.rht(x, s, block)
     q, sc = P.gpu_int4_sym(inp)
-    P.check_int4_sym(q, sc, oracle.rht(x, s, block))
+    P.check_int4_sym(q, sc, y)
+    codes, bs, ts = P.gpu_nvfp4(inp)
+    P.check_nvfp4(codes, bs, ts, y)
+    mc, ms = P.gpu_mxfp4(inp)
+    P.check_mxfp4(mc, ms, y)
 
 
 # ---------------------------------------------------------------- INT4
