@@ -145,6 +145,7 @@ __device__ __noinline__ void tile_exact_minmax(const uint8_t* tile, int m, doubl
   smin = lo;
 }
 
+template <bool kKv>
 __global__ void __launch_bounds__(kThreads, 1)
 k_tcb128_asym(const __grid_constant__ CUtensorMap tmap, Params P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -444,10 +445,12 @@ k_tcb128_asym(const __grid_constant__ CUtensorMap tmap, Params P) {
         const int kc = r4 * 32 + lane, l2 = kc >> 2, p2 = kc & 3;
         const uint4 val =
             *reinterpret_cast<const uint4*>(wbuf + l2 * 64 + ((p2 ^ ((l2 >> 1) & 3)) << 4));
-        const int64_t ou = ub + l2 >= u_lo ? kv_unit(P.slots, P.num_slots, P.kpr, ub + l2) : -1;
+        const int64_t ou =
+            ub + l2 < u_lo ? -1 : (kKv ? kv_unit(P.slots, P.num_slots, P.kpr, ub + l2) : ub + l2);
         if (ou >= 0) *reinterpret_cast<uint4*>(P.codes + ou * 64 + p2 * 16) = val;
       }
-      const int64_t om = y0 + m >= u_lo ? kv_unit(P.slots, P.num_slots, P.kpr, y0 + m) : -1;
+      const int64_t om =
+          y0 + m < u_lo ? -1 : (kKv ? kv_unit(P.slots, P.num_slots, P.kpr, y0 + m) : y0 + m);
       if (om >= 0) {
         uint16_t zh;
         asm("cvt.rn.f16.f32 %0, %1;" : "=h"(zh) : "f"(zf));
@@ -495,7 +498,7 @@ cudaError_t launch_tcb_asym(const void* x, int64_t tokens, const Geometry& g,
   if (!encode_tmap_bf16_2d(&map, x, 128, (uint64_t)P.units, 64, 128,
                            CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorNotSupported;
-  auto k = tcb::k_tcb128_asym;
+  auto k = slots ? tcb::k_tcb128_asym<true> : tcb::k_tcb128_asym<false>;
   cudaFuncSetAttribute((const void*)k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        (int)tcb::kSmemBytes);
   int dev = 0, sms = 0;
