@@ -109,6 +109,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   return sm100::mbar_wait(bar, parity, &g_tc_error);
 }
 
+// a * b + c on bf16 pairs, rounded once to nearest
+__device__ __forceinline__ uint32_t fma_bf16x2(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
 // D fp32, A = H_128 (K-major), B = staged tokens (MN-major), M = 128, N = 128.
 constexpr uint32_t kIdesc = idesc_bf16(128, kAccCols, 1);
 
@@ -520,62 +527,54 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
       if (signs) fence_async_smem();
       __syncwarp();
       mbar_arrive(&ready[s]);
-      // Each bf16 sum of 8 non-negative terms is at least (1 - 2^-8)^7 of the
-      // exact sum (round to nearest), so x (1 + 2^-4) bounds it from above,
-      // with room for the fp32 additions below.
-      float2 acc[4];
-#pragma unroll
-      for (int h = 0; h < 4; ++h)
-        acc[h] = make_float2(__uint_as_float(sacc[h] << 16) * (1.0f + 0x1p-4f),
-                             __uint_as_float(sacc[h] & 0xffff0000u) * (1.0f + 0x1p-4f));
-      float own = 0.0f;                       // this lane's sum |x'|
-#pragma unroll
-      for (int h = 0; h < 4; ++h) own += acc[h].x + acc[h].y;
       // The lane pair (hr = 0, 1) splits the chunk's 8 columns: each keeps
       // words 2 hr, 2 hr + 1, adds its partner's share of the step's sums and
-      // minima, and then takes the inclusive prefix over the steps: P_ks.
-      float2 pre[2];
-      uint32_t mk[2];
+      // minima, and then takes the inclusive prefix over the steps: P_ks.  All
+      // sums stay bf16 (round to nearest): a chain of at most 12 additions of
+      // non-negative terms is at least (1 - 2^-8)^12 > 1 / (1 + 2^-4) of the
+      // exact sum, so x (1 + 2^-4) bounds every one of them from above.
+      uint32_t pre[2], mk[2];
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
-        const float2 keep = hr ? acc[2 + j] : acc[j], send = hr ? acc[j] : acc[2 + j];
-        pre[j] = add2(keep, make_float2(__shfl_xor_sync(0xffffffffu, send.x, 1),
-                                        __shfl_xor_sync(0xffffffffu, send.y, 1)));
+        const uint32_t keep = hr ? sacc[2 + j] : sacc[j], send = hr ? sacc[j] : sacc[2 + j];
+        pre[j] = add_bf16x2(keep, __shfl_xor_sync(0xffffffffu, send, 1));
         const uint32_t mkeep = hr ? mn[2 + j] : mn[j], msend = hr ? mn[j] : mn[2 + j];
         mk[j] = min_bf16x2(mkeep, __shfl_xor_sync(0xffffffffu, msend, 1));
       }
+      const uint32_t s2 = add_bf16x2(add_bf16x2(sacc[0], sacc[1]), add_bf16x2(sacc[2], sacc[3]));
+      const float own = __uint_as_float(s2 << 16) + __uint_as_float(s2 & 0xffff0000u);
 #pragma unroll
       for (int off = 4; off < 32; off <<= 1) {
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
-          const float px = __shfl_up_sync(0xffffffffu, pre[j].x, off);
-          const float py = __shfl_up_sync(0xffffffffu, pre[j].y, off);
-          if (lane >= off) pre[j] = add2(pre[j], make_float2(px, py));
+          const uint32_t p = __shfl_up_sync(0xffffffffu, pre[j], off);
+          if (lane >= off) pre[j] = add_bf16x2(pre[j], p);
         }
       }
       // An input of step ks is truncated only if it is below 2^-18 of the
       // step's largest term, which is at most P_ks; each of the <= 16 such
-      // inputs of a column then loses less than 2^-25 P_ks.  Columns whose
-      // smallest input clears the threshold lose nothing.
-      float r = 0.0f;
-      constexpr float kTinyRel = 0x1p-18f * (1.0f + 0x1p-16f);
+      // inputs of a column then loses less than 2^-25 P_ks.  mk - c P_ks with
+      // c = 2^-18 (1 + 2^-4) is formed exactly and rounded once, which keeps
+      // its sign: a set sign bit marks a column that may lose bits.
+      uint32_t tiny[2];
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        if (__uint_as_float(mk[j] << 16) < pre[j].x * kTinyRel) r += pre[j].x;
-        if (__uint_as_float(mk[j] & 0xffff0000u) < pre[j].y * kTinyRel) r += pre[j].y;
+      for (int j = 0; j < 2; ++j) tiny[j] = fma_bf16x2(pre[j], 0xB688B688u, mk[j]);
+      float r = 0.0f;
+      if ((tiny[0] | tiny[1]) & 0x80008000u) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          if (tiny[j] & 0x00008000u) r += __uint_as_float(pre[j] << 16) * (1.0f + 0x1p-4f);
+          if (tiny[j] & 0x80000000u) r += __uint_as_float(pre[j] & 0xffff0000u) * (1.0f + 0x1p-4f);
+        }
       }
-      // W weights every input by the steps from its own on
-      const float wsum = (float)(8 - ks) * own;
-      const uint32_t mbits = redux_max(max(__float_as_uint(wsum), __float_as_uint(r)));
-      const float S = warp_sum_up(own, mbits);
-      const float W = warp_sum_up(wsum, mbits);
-      const float R = warp_sum_up(r, mbits);
+      // E / u = sum over lanes of own (2.5 (8 - ks) + 5 (1 + 5u)) (W weights
+      // every input by the steps from its own on) + 16 * 2^-25 / u * R, with
+      // the 2^-4 margin of the bf16 sums, all rounded up
+      const float wgt = (2.5f * (float)(8 - ks) + 5.000002f) * (1.0f + 0x1p-4f);
+      const float vl = __fadd_ru(__fmul_ru(own, wgt), __fmul_ru(r, 0x1.0001p+3f));
+      const float tot = warp_sum_up(vl, redux_max(__float_as_uint(vl)));
       if (lane == 0) {
-        // (2.5 W + 5 (1 + 5u) S) u + 16 * 2^-25 (1 + 2^-16) R, all rounded up,
-        // with 2^-10 relative slack for the fp32 sums above
-        const float e1 = __fmul_ru(__fadd_ru(__fmul_ru(2.5f, W), __fmul_ru(5.000002f, S)),
-                                   0x1p-24f);
-        const float e = __fmul_ru(__fadd_ru(e1, __fmul_ru(R, 0x1.0001p-21f)), 1.0f + 0x1p-10f);
+        const float e = __fmul_ru(__fmul_ru(tot, 0x1p-24f), 1.0f + 0x1p-10f);
         sE[((int)(k % kBRing) * kTok + t) * 2 + hc] = e;
         mbar_arrive(&bready[k % kBRing]);
       }
