@@ -31,11 +31,14 @@ namespace kq {
 constexpr int kThreads = 256;
 
 // ------------------------------------------------------------- row loading
-// buf[j] = s_j * x_j as fp32 (exact for bf16 and fp32 inputs).
+// buf[j] = s_j * x_j as fp32 or fp64 (exact for bf16 and fp32 inputs), in
+// 16-byte chunks so that every thread has few loads in flight in sequence.
+template <typename F>
 __device__ __forceinline__ void load_row(const uint16_t* __restrict__ xr,
                                          const int8_t* __restrict__ signs,
-                                         float* buf, int n) {
+                                         F* buf, int n) {
   const uint4* xv = reinterpret_cast<const uint4*>(xr);
+#pragma unroll 2
   for (int c = threadIdx.x; c < n / 8; c += blockDim.x) {
     const uint4 w = __ldg(xv + c);
     uint32_t s0 = 0, s1 = 0;
@@ -58,10 +61,12 @@ __device__ __forceinline__ void load_row(const uint16_t* __restrict__ xr,
   }
 }
 
+template <typename F>
 __device__ __forceinline__ void load_row(const float* __restrict__ xr,
                                          const int8_t* __restrict__ signs,
-                                         float* buf, int n) {
+                                         F* buf, int n) {
   const float4* xv = reinterpret_cast<const float4*>(xr);
+#pragma unroll 4
   for (int c = threadIdx.x; c < n / 4; c += blockDim.x) {
     float4 v = __ldg(xv + c);
     if (signs) {
@@ -71,19 +76,26 @@ __device__ __forceinline__ void load_row(const float* __restrict__ xr,
       v.z = __uint_as_float(__float_as_uint(v.z) ^ (((sw >> 23) & 1u) << 31));
       v.w = __uint_as_float(__float_as_uint(v.w) ^ (((sw >> 31) & 1u) << 31));
     }
-    reinterpret_cast<float4*>(buf)[c] = v;
+    if constexpr (sizeof(F) == 4) {
+      reinterpret_cast<float4*>(buf)[c] = v;
+    } else {
+      buf[4 * c] = v.x;
+      buf[4 * c + 1] = v.y;
+      buf[4 * c + 2] = v.z;
+      buf[4 * c + 3] = v.w;
+    }
   }
 }
 
 // -------------------------------------------------------- butterfly passes
 // One radix-R pass over strides h, 2h, ..., (R/2)h inside every m-segment.
-template <int R>
-__device__ __forceinline__ void fwht_pass(float* buf, int n, int h) {
+template <int R, typename F>
+__device__ __forceinline__ void fwht_pass(F* buf, int n, int h) {
   const int groups = n / R;
   for (int gi = threadIdx.x; gi < groups; gi += blockDim.x) {
     const int lo = gi % h, hi = gi / h;
     const int base = hi * h * R + lo;
-    float v[R];
+    F v[R];
 #pragma unroll
     for (int k = 0; k < R; ++k) v[k] = buf[base + k * h];
 #pragma unroll
@@ -91,7 +103,7 @@ __device__ __forceinline__ void fwht_pass(float* buf, int n, int h) {
 #pragma unroll
       for (int k = 0; k < R; ++k)
         if (!(k & s)) {
-          const float a = v[k], b = v[k | s];
+          const F a = v[k], b = v[k | s];
           v[k] = a + b;
           v[k | s] = a - b;
         }
@@ -101,8 +113,10 @@ __device__ __forceinline__ void fwht_pass(float* buf, int n, int h) {
   __syncthreads();
 }
 
-// Unnormalised Sylvester transform of every m-segment of buf (m | n).
-__device__ void fwht_smem(float* buf, int n, int m) {
+// Unnormalised Sylvester transform of every m-segment of buf (m | n), in
+// fp32 or fp64.
+template <typename F>
+__device__ void fwht_smem(F* buf, int n, int m) {
   int h = 1;
   while (h < m) {
     const int left = m / h;
@@ -122,15 +136,15 @@ __device__ void fwht_smem(float* buf, int n, int m) {
 // Paley-12 factor across the 12 segments of width m:
 // z[a m + beta] = sum_c P[a][c] w[c m + beta] (P = H12, or H12^T when
 // kTranspose), summed in the order c = 0..11.
-template <bool kTranspose>
-__device__ void paley_smem(float* buf, int m) {
+template <bool kTranspose, typename F>
+__device__ void paley_smem(F* buf, int m) {
   for (int beta = threadIdx.x; beta < m; beta += blockDim.x) {
-    float w[12], z[12];
+    F w[12], z[12];
 #pragma unroll
     for (int c = 0; c < 12; ++c) w[c] = buf[c * m + beta];
 #pragma unroll
     for (int a = 0; a < 12; ++a) {
-      float acc = (kTranspose ? paley_negative(0, a) : paley_negative(a, 0)) ? -w[0] : w[0];
+      F acc = (kTranspose ? paley_negative(0, a) : paley_negative(a, 0)) ? -w[0] : w[0];
 #pragma unroll
       for (int c = 1; c < 12; ++c) {
         const bool neg = kTranspose ? paley_negative(c, a) : paley_negative(a, c);
@@ -170,6 +184,7 @@ __device__ double exact_S(const T* __restrict__ xr, const int8_t* __restrict__ s
   const int ia = g.paley ? il / g.m : 0;
   const int ib = g.paley ? il - ia * g.m : il;
   double acc = 0.0;
+#pragma unroll 4
   for (int j = threadIdx.x; j < g.b; j += blockDim.x) {
     int ja = 0, jb = j;
     if (g.paley) {
@@ -604,17 +619,32 @@ k_nvfp4_rowstats(const T* __restrict__ x, const int8_t* __restrict__ signs,
   }
 }
 
-// Dynamic tensor scale, step 2: exact max|S| over the elements of the rows
-// that can hold the global maximum.  Each CTA screens a contiguous range of
-// rows with all its threads at once (one row's statistics per thread) and
-// then transforms only the candidates.
+// Block-wide max of doubles; `red` is shared scratch of >= 32 doubles.
+__device__ __forceinline__ double block_max_d(double v, double* red) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
+  __syncthreads();
+  if (lane == 0) red[wid] = v;
+  __syncthreads();
+  double t = red[0];
+  for (int i = 1; i < nw; ++i) t = fmax(t, red[i]);
+  return t;
+}
+
+// Dynamic tensor scale, step 2: max|S| over the rows that can hold the
+// global maximum, in fp64.  Each CTA screens a contiguous range of rows with
+// all its threads at once (one row's statistics per thread); a candidate row
+// is transformed whole in fp64 (exact inputs, fp64 butterflies and Paley
+// sums: the same precision as an fp64 dot product per output), so no
+// per-output candidate search is needed.
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
 k_nvfp4_global(const T* __restrict__ x, const int8_t* __restrict__ signs,
                NvWorkspace* __restrict__ ws, int64_t tokens, Geometry g) {
   extern __shared__ __align__(16) float smem[];
-  float* buf = smem;
-  double* red = reinterpret_cast<double*>(buf + g.n);
+  double* dbuf = reinterpret_cast<double*>(smem);   // g.n values
+  double* red = dbuf + g.n;
   __shared__ int64_t cand[kThreads];
   __shared__ int ncand;
   const float L = __uint_as_float(ws->lower_bits);
@@ -632,14 +662,15 @@ k_nvfp4_global(const T* __restrict__ x, const int8_t* __restrict__ signs,
     __syncthreads();
     const int nc = ncand;
     for (int c = 0; c < nc; ++c) {
-      const T* xr = x + cand[c] * g.n;
-      transform_row(xr, signs, buf, g, false);
-      // candidates from this kernel's own fp32 values and their own bound
-      const double Eg = error_bound(g, row_absmax(buf, g.n, red));
-      const double best = exact_max_abs(xr, signs, g, buf, 0, g.n,
-                                        thr_down((double)L - Eg), red);
+      load_row(x + cand[c] * g.n, signs, dbuf, g.n);
+      __syncthreads();
+      fwht_smem(dbuf, g.n, g.m);
+      if (g.paley) paley_smem<false>(dbuf, g.m);
+      double m = 0.0;
+      for (int i = threadIdx.x; i < g.n; i += blockDim.x) m = fmax(m, fabs(dbuf[i]));
+      m = block_max_d(m, red);
       if (threadIdx.x == 0)
-        atomicMax(&ws->gmax_bits, (unsigned long long)__double_as_longlong(best));
+        atomicMax(&ws->gmax_bits, (unsigned long long)__double_as_longlong(m));
       __syncthreads();
     }
     __syncthreads();   // every thread has read ncand before the next reset
@@ -861,6 +892,7 @@ cudaError_t launch_nvfp4(const void* x, int dtype, int64_t tokens, const Geometr
   const int nb = g.n / 16;
   const size_t smem = (size_t)g.n * 4 + (size_t)nb * (4 + 1 + 1) + 16 + 64 * 8;
   const size_t smem_stats = (size_t)g.n * 4 + 64 * 8;
+  const size_t smem_glob = (size_t)g.n * 8 + 64 * 8;
   cudaError_t err;
   if (ws) {
     err = cudaMemsetAsync(ws, 0, sizeof(NvWorkspace), s);
@@ -870,14 +902,14 @@ cudaError_t launch_nvfp4(const void* x, int dtype, int64_t tokens, const Geometr
       k1<<<grid_for((const void*)k1, smem_stats, tokens), kThreads, smem_stats, s>>>(
           static_cast<const uint16_t*>(x), signs, ws, tokens, g);
       auto k2 = k_nvfp4_global<uint16_t>;
-      k2<<<grid_for((const void*)k2, smem_stats, tokens), kThreads, smem_stats, s>>>(
+      k2<<<grid_for((const void*)k2, smem_glob, tokens), kThreads, smem_glob, s>>>(
           static_cast<const uint16_t*>(x), signs, ws, tokens, g);
     } else {
       auto k1 = k_nvfp4_rowstats<float>;
       k1<<<grid_for((const void*)k1, smem_stats, tokens), kThreads, smem_stats, s>>>(
           static_cast<const float*>(x), signs, ws, tokens, g);
       auto k2 = k_nvfp4_global<float>;
-      k2<<<grid_for((const void*)k2, smem_stats, tokens), kThreads, smem_stats, s>>>(
+      k2<<<grid_for((const void*)k2, smem_glob, tokens), kThreads, smem_glob, s>>>(
           static_cast<const float*>(x), signs, ws, tokens, g);
     }
     err = cudaGetLastError();
@@ -897,14 +929,14 @@ cudaError_t launch_nvfp4(const void* x, int dtype, int64_t tokens, const Geometr
 
 cudaError_t launch_nvfp4_global(const void* x, int dtype, int64_t tokens, const Geometry& g,
                                 const int8_t* signs, NvWorkspace* ws, cudaStream_t s) {
-  const size_t smem_stats = (size_t)g.n * 4 + 64 * 8;
+  const size_t smem_glob = (size_t)g.n * 8 + 64 * 8;
   if (dtype == 1) {
     auto k2 = k_nvfp4_global<uint16_t>;
-    k2<<<grid_for((const void*)k2, smem_stats, tokens), kThreads, smem_stats, s>>>(
+    k2<<<grid_for((const void*)k2, smem_glob, tokens), kThreads, smem_glob, s>>>(
         static_cast<const uint16_t*>(x), signs, ws, tokens, g);
   } else {
     auto k2 = k_nvfp4_global<float>;
-    k2<<<grid_for((const void*)k2, smem_stats, tokens), kThreads, smem_stats, s>>>(
+    k2<<<grid_for((const void*)k2, smem_glob, tokens), kThreads, smem_glob, s>>>(
         static_cast<const float*>(x), signs, ws, tokens, g);
   }
   return cudaGetLastError();
