@@ -154,6 +154,21 @@ def test_nvfp4_small_dynamic_and_static(key, tokens):
     assert np.array_equal(deq.view(np.uint32), want.view(np.uint32))
 
 
+@pytest.mark.parametrize("key,tokens", [("c2", 2500), ("c4", 2500)])
+def test_nvfp4_dynamic_every_row_a_candidate(key, tokens):
+    """Identical rows all reach the global lower bound, so the dynamic global
+    step transforms every row (more rows than its CTAs: several candidate
+    rows per CTA)."""
+    base = small_inputs(key, 1, with_edges=False)
+    w = base.workload
+    vals = np.repeat(base.values, tokens, axis=0)
+    inp = P.inputs_from_values(w, vals, base.signs)
+    y = np.repeat(oracle.rht(base.values, base.signs, w.block), tokens, axis=0)
+    codes, bs, ts = P.gpu_nvfp4(inp)
+    P.check_nvfp4(codes, bs, ts, y)
+    assert (codes == codes[:1]).all() and (bs == bs[:1]).all()
+
+
 def test_nvfp4_round_trip_c4_small():
     inp = small_inputs("c4", 37)
     w = inp.workload
