@@ -228,6 +228,42 @@ __device__ double exact_max_abs(const T* xr, const int8_t* signs, const Geometry
   return best;
 }
 
+// exact_S from a shared-memory copy xs of the sign-flipped row (fp32 holds
+// every bf16 or fp32 input exactly): the same terms in the same order.
+__device__ double exact_S_smem(const float* xs, const Geometry& g, int i, double* red) {
+  const int blk = i / g.b;
+  const int off = blk * g.b;
+  const int il = i - off;
+  const int ia = g.paley ? il / g.m : 0;
+  const int ib = g.paley ? il - ia * g.m : il;
+  double acc = 0.0;
+  for (int j = threadIdx.x; j < g.b; j += blockDim.x) {
+    int ja = 0, jb = j;
+    if (g.paley) {
+      ja = j / g.m;
+      jb = j - ja * g.m;
+    }
+    bool neg = (__popc(ib & jb) & 1) != 0;
+    if (g.paley) neg ^= paley_negative(ia, ja);
+    const double xv = (double)xs[off + j];
+    acc += neg ? -xv : xv;
+  }
+  return block_sum_d(acc, red);
+}
+
+__device__ double exact_max_abs_smem(const float* xs, const Geometry& g, const float* buf,
+                                     int lo, int hi, float thr, double* red) {
+  double best = 0.0;
+  int prev = lo - 1;
+  for (;;) {
+    const int c = next_candidate(buf, lo, hi, prev, thr, red);
+    if (c == INT_MAX) break;
+    best = fmax(best, fabs(exact_S_smem(xs, g, c, red)));
+    prev = c;
+  }
+  return best;
+}
+
 __device__ __forceinline__ float thr_down(double v) {
   return v > 0.0 ? __double2float_rd(v) : 0.0f;
 }
@@ -278,9 +314,16 @@ k_int4_sym(const T* __restrict__ x, const int8_t* __restrict__ signs,
   extern __shared__ __align__(16) float smem[];
   float* buf = smem;
   double* red = reinterpret_cast<double*>(buf + g.n);
+  float* xs = reinterpret_cast<float*>(red + 64);   // the sign-flipped row, for fix-ups
   for (int64_t row = blockIdx.x; row < tokens; row += gridDim.x) {
     const T* xr = x + row * g.n;
-    transform_row(xr, signs, buf, g, false);
+    load_row(xr, signs, buf, g.n);
+    __syncthreads();
+    for (int c = threadIdx.x; c < g.n / 4; c += blockDim.x)
+      reinterpret_cast<float4*>(xs)[c] = reinterpret_cast<const float4*>(buf)[c];
+    __syncthreads();
+    fwht_smem(buf, g.n, g.m);
+    if (g.paley) paley_smem<false>(buf, g.m);
     const float mh = row_absmax(buf, g.n, red);
     const double E = error_bound(g, mh);
     // scale32 = fp32(fp64(max|S| / sqrt(b)) / 7): decided by fp32 values only
@@ -291,8 +334,8 @@ k_int4_sym(const T* __restrict__ x, const int8_t* __restrict__ signs,
     if (lo_s == hi_s) {
       scale = lo_s;
     } else {
-      const double smax = exact_max_abs(xr, signs, g, buf, 0, g.n,
-                                        thr_down((double)mh - 2.0 * E), red);
+      const double smax = exact_max_abs_smem(xs, g, buf, 0, g.n,
+                                             thr_down((double)mh - 2.0 * E), red);
       scale = __double2float_rn((smax / g.sqrt_b) / 7.0);
     }
     if (threadIdx.x == 0) scales[row] = scale;
@@ -856,7 +899,7 @@ cudaError_t launch_rht(const void* x, int dtype, int64_t tokens, const Geometry&
 cudaError_t launch_int4_sym(const void* x, int dtype, int64_t tokens, const Geometry& g,
                             const int8_t* signs, uint8_t* codes, float* scales,
                             cudaStream_t s) {
-  const size_t smem = (size_t)g.n * sizeof(float) + 64 * sizeof(double);
+  const size_t smem = 2 * (size_t)g.n * sizeof(float) + 64 * sizeof(double);
   if (dtype == 1) {
     auto k = k_int4_sym<uint16_t>;
     k<<<grid_for((const void*)k, smem, tokens), kThreads, smem, s>>>(
