@@ -8,8 +8,9 @@
 //       -- a dense +-1 contraction, run on the tensor cores: D (TMEM, fp32) =
 //       A * B with A = H_128 (bf16 +-1, K-major, built in shared memory once)
 //       and B = the sign-flipped input x' of four tokens side by side
-//       (K = a, N = token*32 + beta; MN-major, 64-byte swizzle, one TMA box
-//       per token);
+//       (K = a, N = token*32 + beta; MN-major, 64-byte swizzle; one 4-D TMA
+//       box per tile puts the four tokens' 8-row swizzle atoms next to each
+//       other, so a K-step of B is 4 KB of contiguous shared memory);
 //   (2) the H_32 over beta, run by the epilogue thread that owns TMEM lane o:
 //       it reads the 32 columns of a token and finishes the transform with five
 //       butterfly stages in fp32 (four on f32x2 pairs).
@@ -64,6 +65,7 @@ namespace tc {
 
 constexpr int kTok = 4;                        // tokens per tile
 constexpr uint32_t kTokBytes = 128 * 32 * 2;   // one token: 128 rows of 32 bf16
+constexpr uint32_t kTokStride = 512;           // token t's atoms start at t * 512
 constexpr uint32_t kStageBytes = kTok * kTokBytes;   // 32 KB
 constexpr int kStages = 5;
 constexpr int kGroups = 2;                     // epilogue groups
@@ -124,10 +126,23 @@ __device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64
   sm100::mma_bf16(tmem_d, adesc, bdesc, kIdesc, accumulate);
 }
 
-// Byte offset of 16-byte chunk c (0..3) of row a of a staged token (128 rows
-// of 64 bytes, 64-byte swizzle: chunk position c ^ ((a >> 1) & 3)).
+// Byte offset of 16-byte chunk c (0..3) of row a of a staged token, from the
+// token's start (t * kTokStride): rows of 64 bytes in 8-row swizzle atoms,
+// the tile's four atoms of an 8-row group side by side (group a >> 3 at
+// 2 KB steps), 64-byte swizzle: chunk position c ^ ((a >> 1) & 3).
 __device__ __forceinline__ uint32_t tok_chunk(int a, int c) {
-  return (uint32_t)(a * 64 + ((c ^ ((a >> 1) & 3)) << 4));
+  return (uint32_t)((a >> 3) * 2048 + (a & 7) * 64 + ((c ^ ((a >> 1) & 3)) << 4));
+}
+
+// One tile: tokens tok0 .. tok0 + 3 (rows beyond the tensor read as zero)
+// as [16 row groups][4 tokens][8 rows][32 columns] bf16.
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, int tok0,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6];"
+      :: "r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(0), "r"(tok0),
+         "r"(0), "r"(smem_u32(bar)) : "memory");
 }
 
 // Exact S_i of token row `row` (bf16, natural order, in global memory),
@@ -371,10 +386,7 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
     for (int64_t k = 0; k < prefilled; ++k) {
       const int64_t tile = blockIdx.x + k * gridDim.x;
       mbar_expect_tx(&full[k], kStageBytes);
-#pragma unroll
-      for (int t = 0; t < kTok; ++t)
-        tma_load_2d(sB + k * kStageBytes + t * kTokBytes, &tmap, 0,
-                    (int)((tile * kTok + t) * 128), &full[k]);
+      tma_load_4d(sB + k * kStageBytes, &tmap, (int)(tile * kTok), &full[k]);
     }
   }
   // A = H_128, one 16-byte chunk (8 columns) per step
@@ -430,10 +442,7 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
         if (k >= kStages && !mbar_wait(&empty[s], (use - 1) & 1)) break;
         const int64_t tile = blockIdx.x + k * gridDim.x;
         mbar_expect_tx(&full[s], kStageBytes);
-#pragma unroll
-        for (int t = 0; t < kTok; ++t)
-          tma_load_2d(sB + s * kStageBytes + t * kTokBytes, &tmap, 0,
-                      (int)((tile * kTok + t) * 128), &full[s]);
+        tma_load_4d(sB + s * kStageBytes, &tmap, (int)(tile * kTok), &full[s]);
         issued = k + 1;
       }
       // no copy may still be in flight when the CTA exits (matters only after
@@ -457,9 +466,9 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
         for (int ks = 0; ks < 8; ++ks) {
           // A: K-major, K step of 16 = 32 bytes inside a 128-byte swizzle row
           const uint64_t adesc = smem_desc(a0 + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, 2);
-          // B: MN-major 64-byte swizzle atoms of 32 columns (one per token,
-          // 8 KB apart), 8-row groups 512 bytes apart; K step of 16 rows = 1 KB
-          const uint64_t bdesc = smem_desc(b0 + ks * 1024, kTokBytes, 512, 4);
+          // B: MN-major 64-byte swizzle atoms of 32 columns x 8 rows (one per
+          // token, 512 bytes apart), 8-row groups 2 KB apart; K step = 4 KB
+          const uint64_t bdesc = smem_desc(b0 + ks * 4096, kTokStride, 2048, 4);
           mma_bf16(tmem_d, adesc, bdesc, ks > 0 ? 1u : 0u);
         }
         mma_commit(&empty[s]);
@@ -489,7 +498,7 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
     for (int64_t k = 0; k < my_tiles; ++k) {
       const int s = (int)(k % kStages);
       if (!mbar_wait(&full[s], (uint32_t)(k / kStages) & 1)) break;
-      uint8_t* tok = sB + s * kStageBytes + t * kTokBytes;
+      uint8_t* tok = sB + s * kStageBytes + t * kTokStride;
       uint32_t sacc[4], mn[4];                    // bf16x2 sums and minima of |x'|
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
@@ -856,7 +865,7 @@ k_diag_steps(const uint16_t* __restrict__ a, const uint16_t* __restrict__ b, flo
   }
   for (int i = threadIdx.x; i < 128 * 128; i += blockDim.x) {
     const int k = i >> 7, n = i & 127, blk = n >> 5, beta = n & 31;
-    *reinterpret_cast<uint16_t*>(sB + blk * kTokBytes + tok_chunk(k, beta >> 3) + (beta & 7) * 2) =
+    *reinterpret_cast<uint16_t*>(sB + blk * kTokStride + tok_chunk(k, beta >> 3) + (beta & 7) * 2) =
         k < 32 ? b[k * 128 + n] : 0;
   }
   if (threadIdx.x == 0) {
@@ -877,7 +886,7 @@ k_diag_steps(const uint16_t* __restrict__ a, const uint16_t* __restrict__ b, flo
   for (int step = 0; step < 2; ++step) {
     if (threadIdx.x == 0) {
       const uint64_t adesc = smem_desc(smem_u32(sA) + step * 32, 16, 1024, 2);
-      const uint64_t bdesc = smem_desc(smem_u32(sB) + step * 1024, kTokBytes, 512, 4);
+      const uint64_t bdesc = smem_desc(smem_u32(sB) + step * 4096, kTokStride, 2048, 4);
       mma_bf16(tmem, adesc, bdesc, (uint32_t)step);
       mma_commit(bar);
     }
@@ -922,10 +931,21 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   return fn;
 }
 
-// [rows, 32] bf16 view of the input (rows of 64 bytes), 32 x 128 boxes (one
-// token), 64-byte swizzle.
+// The input as a 4-D tensor (32 columns, 8 rows, token, 16 row groups; a
+// token is 128 rows of 64 bytes), boxes of 4 tokens, 64-byte swizzle: the
+// shared-memory image is [row group][token][row][column].
 bool make_tmap(CUtensorMap* map, const void* x, int64_t rows) {
-  return encode_tmap_bf16_2d(map, x, 32, (uint64_t)rows, 32, 128, CU_TENSOR_MAP_SWIZZLE_64B);
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t gdim[4] = {32, 8, (cuuint64_t)(rows / 128), 16};
+  cuuint64_t gstride[3] = {64, 8192, 512};   // bytes: next row, next token, next 8 rows
+  cuuint32_t box[4] = {32, 8, 4, 16};
+  cuuint32_t estride[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(x), gdim,
+                   gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
 }
 
 constexpr size_t kSmemBytes = 1024 + 32768 + tc::kStages * tc::kStageBytes + 512 * 16 +
