@@ -114,10 +114,10 @@ __device__ __forceinline__ void fwht_pass(F* buf, int n, int h) {
 }
 
 // Unnormalised Sylvester transform of every m-segment of buf (m | n), in
-// fp32 or fp64.
+// fp32 or fp64; h0 > 1 skips the strides below h0 (already applied).
 template <typename F>
-__device__ void fwht_smem(F* buf, int n, int m) {
-  int h = 1;
+__device__ void fwht_smem(F* buf, int n, int m, int h0 = 1) {
+  int h = h0;
   while (h < m) {
     const int left = m / h;
     if (left >= 8) {
@@ -662,6 +662,60 @@ k_nvfp4_rowstats(const T* __restrict__ x, const int8_t* __restrict__ signs,
   }
 }
 
+// Inputs j0 .. j0 + 7 with the signs applied, exact in fp64.
+__device__ __forceinline__ void load8_f64(const uint16_t* __restrict__ xr,
+                                          const int8_t* __restrict__ signs, int j0,
+                                          double (&v)[8]) {
+  const uint4 w = __ldg(reinterpret_cast<const uint4*>(xr + j0));
+  const uint2 sv = signs ? __ldg(reinterpret_cast<const uint2*>(signs + j0)) : make_uint2(0, 0);
+  const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t sw = k < 2 ? sv.x : sv.y;
+    const uint32_t sb0 = (sw >> (16 * (k & 1) + 7)) & 1u;
+    const uint32_t sb1 = (sw >> (16 * (k & 1) + 15)) & 1u;
+    v[2 * k] = (double)__uint_as_float((ww[k] << 16) ^ (sb0 << 31));
+    v[2 * k + 1] = (double)__uint_as_float((ww[k] & 0xffff0000u) ^ (sb1 << 31));
+  }
+}
+__device__ __forceinline__ void load8_f64(const float* __restrict__ xr,
+                                          const int8_t* __restrict__ signs, int j0,
+                                          double (&v)[8]) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const float4 f = __ldg(reinterpret_cast<const float4*>(xr + j0) + h);
+    const uint32_t sw = signs ? __ldg(reinterpret_cast<const uint32_t*>(signs + j0) + h) : 0u;
+    const float e[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      v[4 * h + k] = (double)__uint_as_float(__float_as_uint(e[k]) ^ (((sw >> (8 * k + 7)) & 1u) << 31));
+  }
+}
+
+// Row j = 0 .. n-1 with the signs applied, in fp64, with the butterflies of
+// strides 1, 2 and 4 already done (each thread holds whole groups of eight).
+template <typename T>
+__device__ __forceinline__ void load_row_f64_h8(const T* __restrict__ xr,
+                                                const int8_t* __restrict__ signs, double* buf,
+                                                int n) {
+#pragma unroll 2
+  for (int gi = threadIdx.x; gi < n / 8; gi += blockDim.x) {
+    double v[8];
+    load8_f64(xr, signs, 8 * gi, v);
+#pragma unroll
+    for (int st = 1; st < 8; st <<= 1)
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (!(k & st)) {
+          const double a = v[k], b = v[k | st];
+          v[k] = a + b;
+          v[k | st] = a - b;
+        }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) buf[8 * gi + k] = v[k];
+  }
+}
+
 // Block-wide max of doubles; `red` is shared scratch of >= 32 doubles.
 __device__ __forceinline__ double block_max_d(double v, double* red) {
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
@@ -705,9 +759,9 @@ k_nvfp4_global(const T* __restrict__ x, const int8_t* __restrict__ signs,
     __syncthreads();
     const int nc = ncand;
     for (int c = 0; c < nc; ++c) {
-      load_row(x + cand[c] * g.n, signs, dbuf, g.n);
+      load_row_f64_h8(x + cand[c] * g.n, signs, dbuf, g.n);
       __syncthreads();
-      fwht_smem(dbuf, g.n, g.m);
+      fwht_smem(dbuf, g.n, g.m, 8);
       if (g.paley) paley_smem<false>(dbuf, g.m);
       double m = 0.0;
       for (int i = threadIdx.x; i < g.n; i += blockDim.x) m = fmax(m, fabs(dbuf[i]));
