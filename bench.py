@@ -74,6 +74,9 @@ def measured_peaks():
 
 
 KERNEL_HEADERS = ("kq_sm100.cuh", "kq_device.cuh", "kq_internal.h")
+# B200 HBM3e datasheet bandwidth (DGX figure), a second denominator beside the
+# measured copy peak
+DATASHEET_HBM_GBS = 8000.0
 
 
 def source_digest(files):
@@ -476,6 +479,7 @@ def main():
                                   if w.fmt == wl.NVFP4 else None),
         "tokens_per_s": round(tokens_s, 1),
         "frac_of_hbm_peak": round(gbs_rank / peak, 4),
+        "frac_of_datasheet_hbm": round(gbs_rank / DATASHEET_HBM_GBS, 4),
         "gpu_launches": launches * args.steps,
         "clocks": sampler.summary(),
         "roofline": {
