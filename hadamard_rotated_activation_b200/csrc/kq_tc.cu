@@ -433,7 +433,7 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
 
 
   if (warp == 0) {
-    // ================= TMA producer: one 128-row box per token
+    // ================= TMA producer: one 4-D box per tile (four tokens)
     if (lane == 0) {
       int64_t issued = prefilled;
       for (int64_t k = prefilled; k < my_tiles; ++k) {
