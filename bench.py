@@ -119,6 +119,7 @@ class ClockSampler:
     def __init__(self, torch_device):
         self.ok = False
         self.samples = []
+        self.busy = []          # samples taken while the GPU reported activity
         self.reasons = 0
         try:
             import pynvml
@@ -143,19 +144,44 @@ class ClockSampler:
         if not self.ok:
             return
         try:
-            self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+            mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+            util = self.nv.nvmlDeviceGetUtilizationRates(self.h).gpu
+            self.samples.append(mhz)
+            if util > 0:
+                self.busy.append(mhz)
             self.reasons |= int(self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
         except Exception:
             pass
 
+    def start(self, period_s=0.02):
+        """Samples every period_s on a thread until stop()."""
+        self._stop = threading.Event()
+
+        def run():
+            while not self._stop.is_set():
+                self.sample()
+                self._stop.wait(period_s)
+        self._thr = threading.Thread(target=run, daemon=True)
+        self._thr.start()
+        return self
+
+    def stop(self):
+        if getattr(self, "_thr", None) is not None:
+            self._stop.set()
+            self._thr.join()
+            self._thr = None
+
     def summary(self):
         names = [n for b, n in self.REASONS.items() if self.reasons & b and b != 0x1]
+        load = self.busy if self.busy else self.samples
         return {
-            "sm_mhz": statistics.median(self.samples) if self.samples else None,
+            "sm_mhz": statistics.median(load) if load else None,
             "sm_max_mhz": self.max_mhz,
             "reasons": names,
             "samples": len(self.samples),
-            "source": "nvml",
+            "samples_under_load": len(self.busy),
+            "source": "nvml, sampled every 20 ms from the first warm-up step to the end "
+                      "of the per-workload table",
         }
 
 
@@ -254,7 +280,43 @@ def cpu_threads():
         return os.cpu_count() or 1
 
 
-def run_cpu_baseline(w, seconds):
+def sample_outputs(w, inp, out_set, tscale, rows=256):
+    """The first `rows` rows of a timed step's inputs and outputs, on the host,
+    for the parity counts of the CPU-baseline leg."""
+    import numpy as np
+    r = min(rows, w.tokens)
+    return {"workload": w.with_tokens(r), "values": inp.values[:r], "signs": inp.signs,
+            "got": tuple(t[:r].cpu().numpy() for t in out_set[1:]
+                         if hasattr(t, "dim") and t.dim() >= 1 and t.shape[0] == w.tokens),
+            "tensor_scale": None if tscale is None else np.float32(tscale)}
+
+
+def sample_parity(oracle_mod, wl, samples):
+    """Counts of the sampled rows against the oracle: rows, codes, scales,
+    scale mismatches (must be 0), code differences within the 1e-5 boundary
+    window (reported) and outside it (must be 0).  NVFP4 is checked under the
+    timed call's own tensor scale."""
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import parity as P
+    out = {}
+    for name, smp in samples.items():
+        w = smp["workload"]
+        y = oracle_mod.rht(smp["values"], smp["signs"], w.block)
+        g = smp["got"]
+        if w.fmt == wl.NVFP4:
+            t = smp["tensor_scale"]
+            c = P.check_nvfp4(g[0], g[1], t, y, tensor_scale=t, strict=False, name=False)
+        elif w.fmt == wl.INT4_SYM:
+            c = P.check_int4_sym(g[0], g[1], y, strict=False, name=False)
+        else:
+            c = P.check_int4_asym(g[0], g[1], g[2], y, w.group, strict=False, name=False)
+        out[name] = c.as_dict()
+    return out
+
+
+def run_cpu_baseline(w, seconds, samples=None):
+    """The oracle timed on the host cores over a bounded sample of rows, and
+    (when `samples` holds GPU outputs) the parity counts of those outputs."""
     import oracle as oracle_mod
     from hadamard_rotated_activation_b200 import workloads as wl
     rows = cpu_sample_rows(oracle_mod, wl, w, seconds)
@@ -263,7 +325,7 @@ def run_cpu_baseline(w, seconds):
     oracle_step(oracle_mod, wl, inp, w)
     dt = time.perf_counter() - t0
     wb = w.with_tokens(rows)
-    return {
+    base = {
         "value": round(wb.algorithmic_bytes() / dt / 1e9, 6),
         "unit": "GB/s",
         "tokens_per_s": round(rows / dt, 3),
@@ -272,6 +334,11 @@ def run_cpu_baseline(w, seconds):
         "sample": f"{rows} of {w.tokens} rows of workload {w.key} "
                   f"(fp64 dense D.H + scalar quantizer), {dt:.2f} s wall",
     }
+    par = None
+    if samples:
+        par = {"rows_per_workload": "the first 256 rows of each timed call's output",
+               "counts": sample_parity(oracle_mod, wl, samples)}
+    return base, par
 
 
 # ------------------------------------------------------------ multi-rank
@@ -323,7 +390,7 @@ def run_reference(args, rank, world):
         "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic",
-        "config": workload_config(w, sample_rows=rows),
+        "config": workload_config(w, forward_only=True, sample_rows=rows),
         "tokens_per_s": round(rows / dt, 3),
         "cpu_baseline": {"value": round(gbs, 6), "unit": "GB/s", "cores": cpu_threads(),
                          "kind": "oracle",
@@ -334,9 +401,14 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
-def workload_config(w, **extra):
+def workload_config(w, forward_only=False, **extra):
+    desc = w.description
+    if forward_only and "; dequant + inverse round trip" in desc:
+        desc = desc.replace("; dequant + inverse round trip", "") + \
+            " (timed step: the forward rotation + quantization; the dequant + inverse " \
+            "round trip is timed separately, per_workload.c4_roundtrip)"
     d = {
-        "workload": f"{w.key}: {w.description}",
+        "workload": f"{w.key}: {desc}",
         "tokens": w.tokens, "dim": w.dim, "block": w.block,
         "input_dtype": w.dtype, "format": w.fmt, "seed": w.seed,
         "global_batch": w.tokens, "seq_len": None, "parallelism": "dp (independent batches)",
@@ -402,12 +474,12 @@ def main():
     set_bytes = w.algorithmic_bytes()
     sets = [make_set(x0 if i == 0 else x0.clone()) for i in range(n_sets(set_bytes))]
 
-    sampler = ClockSampler(dev)
+    sampler = ClockSampler(dev).start()
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
-    ms = time_steps(torch, step, sets, args.steps, args.warmup, sampler, stream)
+    ms = time_steps(torch, step, sets, args.steps, args.warmup, None, stream)
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
@@ -459,9 +531,11 @@ def main():
 
     k_e2e = max(3, min(args.steps, 50))
     ms_e2e = time_steps(torch, e2e_step, [None], k_e2e, max(3, min(args.warmup, 5)))
-    # the chunked path must give the device-resident path's result
-    if not torch.equal(outs_host[0], sets[0][1].cpu()):
-        raise SystemExit("end-to-end result differs from the device-resident step")
+    # the chunked path must give the device-resident path's result, every
+    # output (codes, scales and, for asymmetric INT4, zero points)
+    for h, i in zip(outs_host, out_idx):
+        if not torch.equal(h, sets[0][i].cpu()):
+            raise SystemExit(f"end-to-end output {i} differs from the device-resident step")
     ms_e2e = max_over_ranks(torch, dist, ms_e2e, dev)
     e2e_gbs = whole_job_gbs(alg, world, ms_e2e / k_e2e)
 
@@ -473,15 +547,17 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 6),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic",
-        "config": workload_config(w, l2="inputs larger than L2: %d rotating buffer sets"
+        "config": workload_config(w, forward_only=True,
+                                  l2="inputs larger than L2: %d rotating buffer sets"
                                   % len(sets),
-                                  tensor_scale="static (computed once by the dynamic path)"
+                                  tensor_scale="static: an input of the timed call, computed "
+                                  "once beforehand by the dynamic path (the dynamic two-pass "
+                                  "call is timed as dynamic_tensor_scale)"
                                   if w.fmt == wl.NVFP4 else None),
         "tokens_per_s": round(tokens_s, 1),
         "frac_of_hbm_peak": round(gbs_rank / peak, 4),
         "frac_of_datasheet_hbm": round(gbs_rank / DATASHEET_HBM_GBS, 4),
         "gpu_launches": launches * args.steps,
-        "clocks": sampler.summary(),
         "roofline": {
             "bound": "hbm", "achieved": round(gbs_rank, 3), "peak": peak, "unit": "GB/s",
             "frac": round(gbs_rank / peak, 4), "peak_kind": peak_kind,
@@ -495,10 +571,18 @@ def main():
                 "streams": "copy in / call / copy out"},
     }
 
+    samples = {"headline": sample_outputs(w, inp, sets[0], tscale)}
     if not args.no_extras and rank == 0:
-        line["per_workload"] = extras(torch, kq, wl, dev, peak, args)
+        line["per_workload"], more = extras(torch, kq, wl, dev, peak, args)
+        samples.update(more)
+        dyn = line["per_workload"].get(f"{w.key}_dynamic")
+        if dyn is not None:
+            line["dynamic_tensor_scale"] = {k: dyn[k] for k in ("ms", "GB/s", "frac",
+                                                                 "launches_per_step")}
+    sampler.stop()
+    line["clocks"] = sampler.summary()
     if not args.no_cpu_baseline and rank == 0 and world == 1:
-        line["cpu_baseline"] = run_cpu_baseline(w, args.cpu_seconds)
+        line["cpu_baseline"], line["parity"] = run_cpu_baseline(w, args.cpu_seconds, samples)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist is not None:
@@ -510,7 +594,7 @@ def extras(torch, kq, wl, dev, peak, args):
     """Per-workload forward timings (all five), NVFP4 dynamic, and the c4
     dequant + inverse round trip.  Not part of the headline value."""
     import numpy as np
-    out = {}
+    out, samples = {}, {}
     k = max(20, min(args.steps, 200))
     for key, w in wl.WORKLOADS.items():
         inp = wl.make_inputs(w)
@@ -540,6 +624,10 @@ def extras(torch, kq, wl, dev, peak, args):
             tkey = f"{key}_{w.fmt}" + ("_static" if mode == "static" else "")
             if mode != "dynamic" and ncu_traffic(tkey) is not None:
                 out[name]["traffic"] = round(ncu_traffic(tkey))
+            t_used = None
+            if w.fmt == wl.NVFP4:
+                t_used = float(sets[0][3].item())
+            samples[name] = sample_outputs(w, inp, sets[0], t_used)
             del sets
         if key == "c4":
             out.update(roundtrip(torch, kq, wl, dev, peak, k, 5, 0, x0, signs))
@@ -558,7 +646,7 @@ def extras(torch, kq, wl, dev, peak, args):
             del mx_sets
         del x0
         torch.cuda.empty_cache()
-    return out
+    return out, samples
 
 
 def roundtrip(torch, kq, wl, dev, peak, k, warmup, tokens=0, x0=None, signs=None):

@@ -41,7 +41,7 @@ C_SYMBOLS = (
     "kq_dequant_rht_inverse", "kq_rht_quant_mxfp4", "kq_rht_quant_int4_kv",
     "kq_device_errors", "kq_diag_wait_timeout",
     "kq_workspace_size", "kq_status_str", "kq_last_cuda_error", "kq_version",
-    "kq_rht_quant_nvfp4_dynamic_noalloc", "kq_diag_tc_steps",
+    "kq_rht_quant_nvfp4_dynamic_noalloc", "kq_diag_tc_steps", "kq_diag_fail_next_launch",
 )
 
 # Fixed device scratch of kq_rht_quant_nvfp4_dynamic_noalloc (see include/kq.h).
@@ -103,6 +103,8 @@ def lib() -> ctypes.CDLL:
     L.kq_version.restype = i32
     L.kq_diag_tc_steps.argtypes = [vp, vp, vp, vp, vp, vp]
     L.kq_diag_tc_steps.restype = i32
+    L.kq_diag_fail_next_launch.argtypes = [i32]
+    L.kq_diag_fail_next_launch.restype = None
     _lib = L
     return L
 

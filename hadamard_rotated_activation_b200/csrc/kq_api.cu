@@ -64,6 +64,23 @@ kq_status finish(cudaError_t e) {
   return KQ_OK;
 }
 
+// A simulated launch failure armed by kq_diag_fail_next_launch (this thread).
+thread_local int g_fail_next_launch = 0;
+
+// Runs a launcher (a validated call about to enqueue work) and turns its CUDA
+// error into a status; an armed simulated failure is taken instead, and then
+// nothing is enqueued.
+template <class F>
+kq_status dispatch(F&& launch) {
+  if (g_fail_next_launch != 0) {
+    const int e = g_fail_next_launch;
+    g_fail_next_launch = 0;
+    g_last_cuda_error = e;
+    return KQ_ERR_CUDA;
+  }
+  return finish(launch());
+}
+
 // Format-specific argument checks shared by kq_dequant and
 // kq_dequant_rht_inverse.
 kq_status check_dequant(int fmt, const uint8_t* codes, const void* scales, const void* zeros,
@@ -113,13 +130,17 @@ KQ_API kq_status kq_rht(const void* x, int dtype, int64_t tokens, int dim, int b
   if (!aligned(out, 16)) return KQ_ERR_MISALIGNED;
   if (tokens == 0) return KQ_OK;
   if (!(flags & KQ_INVERSE) && kq::tc_row_supported(g, dtype, x, tokens))
-    return finish(kq::launch_tc_rot(x, tokens, g, signs, out,
-                                    reinterpret_cast<cudaStream_t>(stream)));
+    return dispatch([&] {
+      return kq::launch_tc_rot(x, tokens, g, signs, out, reinterpret_cast<cudaStream_t>(stream));
+    });
   if (!(flags & KQ_INVERSE) && kq::tcp_supported(g, dtype, x, tokens) && aligned(signs, 8))
-    return finish(kq::launch_tcp_rot(x, tokens, g, signs, out,
-                                     reinterpret_cast<cudaStream_t>(stream)));
-  return finish(kq::launch_rht(x, dtype, tokens, g, signs, out, (flags & KQ_INVERSE) ? 1 : 0,
-                               reinterpret_cast<cudaStream_t>(stream)));
+    return dispatch([&] {
+      return kq::launch_tcp_rot(x, tokens, g, signs, out, reinterpret_cast<cudaStream_t>(stream));
+    });
+  return dispatch([&] {
+    return kq::launch_rht(x, dtype, tokens, g, signs, out, (flags & KQ_INVERSE) ? 1 : 0,
+                          reinterpret_cast<cudaStream_t>(stream));
+  });
 }
 
 KQ_API kq_status kq_rht_quant_int4(const void* x, int dtype, int64_t tokens, int dim,
@@ -144,25 +165,32 @@ KQ_API kq_status kq_rht_quant_int4(const void* x, int dtype, int64_t tokens, int
   if (tokens == 0) return KQ_OK;
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (asym == 1 && kq::tcb_supported(g, dtype, x, tokens))
-    return finish(kq::launch_tcb_asym(x, tokens, g, signs, codes,
-                                      static_cast<uint16_t*>(scales),
-                                      static_cast<uint16_t*>(zeros), nullptr, 0, s));
+    return dispatch([&] {
+      return kq::launch_tcb_asym(x, tokens, g, signs, codes, static_cast<uint16_t*>(scales),
+                                 static_cast<uint16_t*>(zeros), nullptr, 0, s);
+    });
   if (asym == 1 && kq::blk128_supported(g, dtype) && aligned(signs, 16))
-    return finish(kq::launch_blk128_asym(x, tokens, g, signs, codes,
-                                         static_cast<uint16_t*>(scales),
-                                         static_cast<uint16_t*>(zeros), nullptr, 0, s));
+    return dispatch([&] {
+      return kq::launch_blk128_asym(x, tokens, g, signs, codes, static_cast<uint16_t*>(scales),
+                                    static_cast<uint16_t*>(zeros), nullptr, 0, s);
+    });
   if (asym == 0 && kq::tcp_supported(g, dtype, x, tokens) && aligned(signs, 8))
-    return finish(kq::launch_tcp_int4(x, tokens, g, signs, codes, static_cast<float*>(scales),
-                                      s));
+    return dispatch([&] {
+      return kq::launch_tcp_int4(x, tokens, g, signs, codes, static_cast<float*>(scales), s);
+    });
   if (asym == 0 && kq::rowwarp_supported(g, dtype))
-    return finish(kq::launch_rowwarp_int4(x, dtype, tokens, g, signs, codes,
-                                          static_cast<float*>(scales), s));
+    return dispatch([&] {
+      return kq::launch_rowwarp_int4(x, dtype, tokens, g, signs, codes, static_cast<float*>(scales),
+                                     s);
+    });
   if (asym == 0)
-    return finish(kq::launch_int4_sym(x, dtype, tokens, g, signs, codes,
-                                      static_cast<float*>(scales), s));
-  return finish(kq::launch_int4_asym(x, dtype, tokens, g, signs, group, codes,
-                                     static_cast<uint16_t*>(scales),
-                                     static_cast<uint16_t*>(zeros), s));
+    return dispatch([&] {
+      return kq::launch_int4_sym(x, dtype, tokens, g, signs, codes, static_cast<float*>(scales), s);
+    });
+  return dispatch([&] {
+    return kq::launch_int4_asym(x, dtype, tokens, g, signs, group, codes,
+                                static_cast<uint16_t*>(scales), static_cast<uint16_t*>(zeros), s);
+  });
 }
 
 KQ_API kq_status kq_rht_quant_int4_kv(const void* x, int dtype, int64_t tokens, int dim,
@@ -183,11 +211,15 @@ KQ_API kq_status kq_rht_quant_int4_kv(const void* x, int dtype, int64_t tokens, 
   if (tokens == 0) return KQ_OK;
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (kq::tcb_supported(g, dtype, x, tokens))
-    return finish(kq::launch_tcb_asym(x, tokens, g, signs, codes_cache, scales_cache,
-                                      zeros_cache, slot_mapping, num_slots, s));
+    return dispatch([&] {
+      return kq::launch_tcb_asym(x, tokens, g, signs, codes_cache, scales_cache, zeros_cache,
+                                 slot_mapping, num_slots, s);
+    });
   if (kq::blk128_supported(g, dtype))
-    return finish(kq::launch_blk128_asym(x, tokens, g, signs, codes_cache, scales_cache,
-                                         zeros_cache, slot_mapping, num_slots, s));
+    return dispatch([&] {
+      return kq::launch_blk128_asym(x, tokens, g, signs, codes_cache, scales_cache, zeros_cache,
+                                    slot_mapping, num_slots, s);
+    });
   return KQ_ERR_UNSUPPORTED;
 }
 
@@ -213,18 +245,24 @@ KQ_API kq_status kq_rht_quant_nvfp4(const void* x, int dtype, int64_t tokens, in
   }
   if (tokens == 0) return KQ_OK;
   if (kq::blk128_supported(g, dtype) && aligned(signs, 16) && aligned(block_scales, 8))
-    return finish(kq::launch_blk128_nvfp4(x, tokens, g, signs, codes, block_scales,
-                                          tensor_scale, ws,
-                                          reinterpret_cast<cudaStream_t>(stream)));
+    return dispatch([&] {
+      return kq::launch_blk128_nvfp4(x, tokens, g, signs, codes, block_scales, tensor_scale, ws,
+                                     reinterpret_cast<cudaStream_t>(stream));
+    });
   if (kq::tc_row_supported(g, dtype, x, tokens) && aligned(block_scales, 8))
-    return finish(kq::launch_tc_nvfp4(x, tokens, g, signs, codes, block_scales, tensor_scale,
-                                      ws, reinterpret_cast<cudaStream_t>(stream)));
+    return dispatch([&] {
+      return kq::launch_tc_nvfp4(x, tokens, g, signs, codes, block_scales, tensor_scale, ws,
+                                 reinterpret_cast<cudaStream_t>(stream));
+    });
   if (kq::rowwarp_supported(g, dtype) && aligned(block_scales, 8))
-    return finish(kq::launch_rowwarp_nvfp4(x, dtype, tokens, g, signs, codes, block_scales,
-                                           tensor_scale, ws,
-                                           reinterpret_cast<cudaStream_t>(stream)));
-  return finish(kq::launch_nvfp4(x, dtype, tokens, g, signs, codes, block_scales,
-                                 tensor_scale, ws, reinterpret_cast<cudaStream_t>(stream)));
+    return dispatch([&] {
+      return kq::launch_rowwarp_nvfp4(x, dtype, tokens, g, signs, codes, block_scales, tensor_scale,
+                                      ws, reinterpret_cast<cudaStream_t>(stream));
+    });
+  return dispatch([&] {
+    return kq::launch_nvfp4(x, dtype, tokens, g, signs, codes, block_scales, tensor_scale, ws,
+                            reinterpret_cast<cudaStream_t>(stream));
+  });
 }
 
 KQ_API kq_status kq_rht_quant_mxfp4(const void* x, int dtype, int64_t tokens, int dim,
@@ -238,8 +276,8 @@ KQ_API kq_status kq_rht_quant_mxfp4(const void* x, int dtype, int64_t tokens, in
   if (tokens == 0) return KQ_OK;
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (kq::tc_row_supported(g, dtype, x, tokens))
-    return finish(kq::launch_tc_mxfp4(x, tokens, g, signs, codes, scales, s));
-  return finish(kq::launch_mxfp4(x, dtype, tokens, g, signs, codes, scales, s));
+    return dispatch([&] { return kq::launch_tc_mxfp4(x, tokens, g, signs, codes, scales, s); });
+  return dispatch([&] { return kq::launch_mxfp4(x, dtype, tokens, g, signs, codes, scales, s); });
 }
 
 KQ_API kq_status kq_dequant(int fmt, const uint8_t* codes, const void* scales,
@@ -251,8 +289,10 @@ KQ_API kq_status kq_dequant(int fmt, const uint8_t* codes, const void* scales,
                                      group, out);
   if (st != KQ_OK) return st;
   if (tokens == 0) return KQ_OK;
-  return finish(kq::launch_dequant(fmt, codes, scales, zeros, tensor_scale, tokens, dim,
-                                   group, out, reinterpret_cast<cudaStream_t>(stream)));
+  return dispatch([&] {
+    return kq::launch_dequant(fmt, codes, scales, zeros, tensor_scale, tokens, dim, group, out,
+                              reinterpret_cast<cudaStream_t>(stream));
+  });
 }
 
 KQ_API kq_status kq_dequant_rht_inverse(int fmt, const uint8_t* codes, const void* scales,
@@ -273,10 +313,14 @@ KQ_API kq_status kq_dequant_rht_inverse(int fmt, const uint8_t* codes, const voi
   const int bf16 = out_dtype == KQ_BF16 ? 1 : 0;
   if (fmt == KQ_FMT_NVFP4 &&
       kq::tci_supported(g, codes, static_cast<const uint8_t*>(scales), signs, out))
-    return finish(kq::launch_tcinv_nvfp4(codes, static_cast<const uint8_t*>(scales),
-                                         tensor_scale, tokens, g, signs, out, bf16, s));
-  return finish(kq::launch_dequant_rht_inv(fmt, codes, scales, zeros, tensor_scale, tokens, g,
-                                           group, signs, out, bf16, s));
+    return dispatch([&] {
+      return kq::launch_tcinv_nvfp4(codes, static_cast<const uint8_t*>(scales), tensor_scale,
+                                    tokens, g, signs, out, bf16, s);
+    });
+  return dispatch([&] {
+    return kq::launch_dequant_rht_inv(fmt, codes, scales, zeros, tensor_scale, tokens, g, group,
+                                      signs, out, bf16, s);
+  });
 }
 
 KQ_API kq_status kq_device_errors(unsigned int* flags) {
@@ -291,7 +335,9 @@ KQ_API kq_status kq_device_errors(unsigned int* flags) {
 
 KQ_API kq_status kq_diag_wait_timeout(long long limit_cycles, kq_stream_t stream) {
   if (limit_cycles <= 0 || limit_cycles > 4000000000ll) return KQ_ERR_INVALID_ARG;
-  return finish(kq::launch_diag_wait(limit_cycles, reinterpret_cast<cudaStream_t>(stream)));
+  return dispatch([&] {
+    return kq::launch_diag_wait(limit_cycles, reinterpret_cast<cudaStream_t>(stream));
+  });
 }
 
 KQ_API size_t kq_workspace_size(int64_t tokens, int dim, int block) {
@@ -313,6 +359,8 @@ KQ_API const char* kq_status_str(int status) {
 
 KQ_API int kq_last_cuda_error(void) { return g_last_cuda_error; }
 
+KQ_API void kq_diag_fail_next_launch(int cuda_error) { g_fail_next_launch = cuda_error; }
+
 KQ_API int kq_version(void) { return (1 << 16) | 0; }
 
 KQ_API kq_status kq_diag_tc_steps(const uint16_t* a, const uint16_t* b, float* d1, float* d2,
@@ -321,8 +369,9 @@ KQ_API kq_status kq_diag_tc_steps(const uint16_t* a, const uint16_t* b, float* d
   if (!aligned(a, 2) || !aligned(b, 2) || !aligned(d1, 4) || !aligned(d2, 4) ||
       !aligned(status, 4))
     return KQ_ERR_MISALIGNED;
-  return finish(kq::launch_diag_tc_steps(a, b, d1, d2, status,
-                                         reinterpret_cast<cudaStream_t>(stream)));
+  return dispatch([&] {
+    return kq::launch_diag_tc_steps(a, b, d1, d2, status, reinterpret_cast<cudaStream_t>(stream));
+  });
 }
 
 }  // extern "C"

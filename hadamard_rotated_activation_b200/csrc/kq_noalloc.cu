@@ -9,7 +9,10 @@
 //
 // The array lives in every GPU that loads the library until the process exits.
 // Host code only sees a host-side stand-in for it, so its device address is
-// looked up once per device (with that device current) and cached.
+// looked up with the device current and cached per device and context.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <cstdint>
 #include <mutex>
 
@@ -26,8 +29,26 @@ __device__ __align__(256) unsigned char g_nvfp4_scratch[kScratchBytes];
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void* g_scratch_ptr[kMaxDevices] = {};
+CUcontext g_scratch_ctx[kMaxDevices] = {};
 
-// Device address of g_nvfp4_scratch on the current device (nullptr on error).
+// The driver's cuCtxGetCurrent, through the runtime (no link against libcuda).
+PFN_cuCtxGetCurrent_v4000 get_ctx_fn() {
+  static PFN_cuCtxGetCurrent_v4000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+  });
+  return fn;
+}
+
+// Device address of g_nvfp4_scratch in the current context (nullptr on
+// error).  The address is cached per device together with the context it was
+// looked up in: after cudaDeviceReset, or with another context current, the
+// module is loaded anew at another address and the lookup is repeated.
 void* scratch_on_current_device(cudaError_t* err) {
   int dev = 0;
   *err = cudaGetDevice(&dev);
@@ -36,12 +57,28 @@ void* scratch_on_current_device(cudaError_t* err) {
     *err = cudaErrorInvalidDevice;
     return nullptr;
   }
+  PFN_cuCtxGetCurrent_v4000 cur = get_ctx_fn();
+  if (!cur) {
+    *err = cudaErrorDeviceUninitialized;
+    return nullptr;
+  }
+  CUcontext ctx = nullptr;
+  if (cur(&ctx) != CUDA_SUCCESS) {
+    *err = cudaErrorDeviceUninitialized;
+    return nullptr;
+  }
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_ptr[dev]) {
+  if (!ctx || !g_scratch_ptr[dev] || g_scratch_ctx[dev] != ctx) {
+    // the lookup also creates the device's primary context if none is current
     void* p = nullptr;
     *err = cudaGetSymbolAddress(&p, g_nvfp4_scratch);
     if (*err != cudaSuccess) return nullptr;
+    if (!ctx && (cur(&ctx) != CUDA_SUCCESS || !ctx)) {
+      *err = cudaErrorDeviceUninitialized;
+      return nullptr;
+    }
     g_scratch_ptr[dev] = p;
+    g_scratch_ctx[dev] = ctx;
   }
   return g_scratch_ptr[dev];
 }

@@ -286,8 +286,10 @@ KQ_API kq_status kq_diag_wait_timeout(long long limit_cycles, kq_stream_t stream
  * The call allocates nothing and calls no allocating routine.
  *
  * The first call on each device looks up the array's device address (with
- * that device current) and caches it; make that first call before any stream
- * capture.  All calls share the one array and it keeps the last call's
+ * that device current) and caches it together with the current CUDA context;
+ * a call in another context (another context made current, or the primary
+ * context recreated after cudaDeviceReset) looks it up again.  Make the first
+ * call in each context before any stream capture.  All calls share the one array and it keeps the last call's
  * contents (each call clears what must start at zero), so calls that overlap
  * on the GPU -- on different streams or from different threads -- race and
  * must be serialized by the caller.
@@ -306,6 +308,17 @@ KQ_API const char* kq_status_str(int status);
 
 /* The CUDA error code behind the calling thread's last KQ_ERR_CUDA (0 if none). */
 KQ_API int kq_last_cuda_error(void);
+
+/*
+ * Diagnostic (the pages have no counterpart): arms a simulated launch failure
+ * for the calling thread.  The next call of an entry point that passes its
+ * argument checks and would enqueue work enqueues nothing, returns
+ * KQ_ERR_CUDA and sets kq_last_cuda_error() to cuda_error; that disarms it.
+ * Calls rejected by their checks, and calls with tokens == 0, leave it armed.
+ * 0 disarms.  It lets the error path of every entry point be tested on a
+ * machine without a GPU, and without making a GPU fail.
+ */
+KQ_API void kq_diag_fail_next_launch(int cuda_error);
 
 /* ABI version: (major << 16) | minor. */
 KQ_API int kq_version(void);

@@ -152,3 +152,52 @@ def test_python_binding_rejects_host_tensors(L):
     x = torch.zeros(2, 64)
     with pytest.raises(ValueError):
         kq.kq_rht(x, 0, None, torch.zeros(2, 64))
+
+
+# cudaErrorLaunchOutOfResources, a launch failure a real GPU can report
+_LAUNCH_ERR = 701
+
+
+def test_launch_failure_reaches_the_caller(L):
+    """A simulated launch failure (armed by kq_diag_fail_next_launch, so that
+    nothing is launched and no GPU is needed) comes back from each entry point
+    as KQ_ERR_CUDA with the CUDA error in kq_last_cuda_error()."""
+    ws = L.kq_workspace_size(4, 4096, 0)
+    calls = {
+        "kq_rht": lambda: L.kq_rht(P, kq.KQ_BF16, 4, 4096, 0, None, Q, 0, None),
+        "kq_rht inverse": lambda: L.kq_rht(P, kq.KQ_F32, 4, 12288, 0, None, Q, kq.KQ_INVERSE,
+                                           None),
+        "kq_rht_quant_int4 sym": lambda: L.kq_rht_quant_int4(P, 1, 4, 12288, 0, None, 0, 0, Q,
+                                                            Q, None, None),
+        "kq_rht_quant_int4 asym": lambda: L.kq_rht_quant_int4(P, 1, 4, 4096, 128, None, 128, 1,
+                                                             Q, Q, Q, None),
+        "kq_rht_quant_nvfp4 static": lambda: L.kq_rht_quant_nvfp4(
+            P, 1, 4, 4096, 0, None, Q, Q, Q, None, 0, kq.KQ_SCALE_STATIC, None),
+        "kq_rht_quant_nvfp4 dynamic": lambda: L.kq_rht_quant_nvfp4(
+            P, 1, 4, 4096, 128, None, Q, Q, Q, P, ws, kq.KQ_SCALE_DYNAMIC, None),
+        "kq_rht_quant_mxfp4": lambda: L.kq_rht_quant_mxfp4(P, 1, 4, 4096, 0, None, Q, Q, None),
+        "kq_dequant": lambda: L.kq_dequant(kq.KQ_FMT_INT4_SYM, P, Q, None, None, 4, 4096, 0, Q,
+                                           None),
+        "kq_dequant_rht_inverse": lambda: L.kq_dequant_rht_inverse(
+            kq.KQ_FMT_NVFP4, P, Q, None, Q, 4, 4096, 0, 0, None, Q, kq.KQ_F32, None),
+        "kq_rht_quant_int4_kv": lambda: L.kq_rht_quant_int4_kv(P, 1, 4, 4096, 128, None, 128, P,
+                                                               8, Q, Q, Q, None),
+        "kq_diag_wait_timeout": lambda: L.kq_diag_wait_timeout(1000, None),
+    }
+    try:
+        for name, call in calls.items():
+            L.kq_diag_fail_next_launch(_LAUNCH_ERR)
+            assert call() == kq.KQ_ERR_CUDA, name
+            assert L.kq_last_cuda_error() == _LAUNCH_ERR, name
+        # a call its checks reject, or a no-op call, does not take the failure
+        L.kq_diag_fail_next_launch(_LAUNCH_ERR + 1)
+        assert L.kq_rht(P + 2, 1, 4, 4096, 0, None, Q, 0, None) == kq.KQ_ERR_MISALIGNED
+        assert L.kq_rht(P, 1, 0, 4096, 0, None, Q, 0, None) == kq.KQ_OK
+        assert L.kq_rht(P, 1, 4, 4096, 0, None, Q, 0, None) == kq.KQ_ERR_CUDA
+        assert L.kq_last_cuda_error() == _LAUNCH_ERR + 1
+        # the Python binding raises with the CUDA error in the message
+        L.kq_diag_fail_next_launch(_LAUNCH_ERR)
+        with pytest.raises(kq.KQError, match="701"):
+            kq._check(L.kq_rht(P, 1, 4, 4096, 0, None, Q, 0, None), "kq_rht")
+    finally:
+        L.kq_diag_fail_next_launch(0)

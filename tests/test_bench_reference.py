@@ -42,3 +42,37 @@ def test_reference_arm_other_ranks_print_nothing(monkeypatch, capsys):
                                       "--warmup", "1"])
     bench.run_reference(bench.parse_args(), 1, 2)
     assert capsys.readouterr().out == ""
+
+
+def test_sample_parity_counts_on_cpu():
+    """The parity counts the CPU-baseline leg attaches to the bench line: the
+    oracle's own outputs give zero mismatches; a flipped scale is counted."""
+    import numpy as np
+    import bench
+    import oracle
+    from hadamard_rotated_activation_b200 import workloads as wl
+
+    samples = {}
+    for key in ("c1", "c5", "c4"):
+        w = wl.WORKLOADS[key].with_tokens(3)
+        inp = wl.make_inputs(w)
+        y = oracle.rht(inp.values, inp.signs, w.block)
+        t = None
+        if w.fmt == wl.INT4_SYM:
+            q, s = oracle.int4_sym_per_token(y)
+            got = (oracle.pack_nibbles(q), s)
+        elif w.fmt == wl.INT4_ASYM:
+            u, s, z = oracle.int4_asym_group(y, w.group)
+            got = (oracle.pack_nibbles(u), s, z)
+        else:
+            c, b, t = oracle.nvfp4(y)
+            got = (oracle.pack_nibbles(c), b)
+        samples[key] = {"workload": w, "values": inp.values, "signs": inp.signs, "got": got,
+                        "tensor_scale": t}
+    out = bench.sample_parity(oracle, wl, samples)
+    for key, c in out.items():
+        assert c["rows"] == 3 and c["scale_mismatch"] == 0 and c["bad"] == 0, (key, c)
+    b = samples["c4"]["got"][1].copy()
+    b[0, 0] ^= 1
+    samples["c4"]["got"] = (samples["c4"]["got"][0], b)
+    assert bench.sample_parity(oracle, wl, {"c4": samples["c4"]})["c4"]["scale_mismatch"] >= 1

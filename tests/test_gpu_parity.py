@@ -3,8 +3,9 @@
 Small cases span several CTAs and a ragged row count, plus degenerate rows
 (zeros, a single spike, constant, alternating, tiny, huge).  Full-size cases
 run each workload at its published size in the launch configuration the
-benchmark times and compare sampled rows (or every row where a global
-quantity such as the NVFP4 tensor scale needs them).
+benchmark times and compare every row (in row chunks on the CPU); the
+counts of every comparison, near-boundary code differences included, are
+printed at the end of the session.
 """
 import numpy as np
 import pytest
@@ -221,41 +222,46 @@ def _sample_rows(t, k, seed):
 
 @pytest.mark.parametrize("key", ["c1", "c3", "c5"])
 def test_full_size_per_token_formats(key):
+    """Every row of the workload at its full size, in the launch the benchmark
+    times, against the oracle (row chunks on the CPU)."""
     w = wl.WORKLOADS[key]
-    inp = wl.make_inputs(w)
-    rows = _sample_rows(w.tokens, 48, 1)
-    if key == "c3":
-        # include the sink rows
-        big = np.argsort(-np.abs(inp.values).max(axis=1))[:10]
-        rows = np.unique(np.concatenate([rows, big]))
-    y = oracle.rht(inp.values[rows], inp.signs, w.block)
-    if w.fmt == wl.INT4_SYM:
-        codes, scales = P.gpu_int4_sym(inp)
-        P.check_int4_sym(codes[rows], scales[rows], y)
-    else:
-        codes, scales, zeros = P.gpu_int4_asym(inp, w.group)
-        P.check_int4_asym(codes[rows], scales[rows], zeros[rows], y, w.group)
+    inp = P.full_inputs(key)
+    got = P.gpu_int4_sym(inp) if w.fmt == wl.INT4_SYM else P.gpu_int4_asym(inp, w.group)
+    c = P.check_all_rows(f"full {key} {w.fmt}", inp, got)
+    assert c.rows == w.tokens and c.scale_mismatch == 0 and c.bad == 0
 
 
 @pytest.mark.parametrize("key", ["c2", "c4"])
 def test_full_size_nvfp4(key):
+    """Dynamic tensor scale: the global scale equals the oracle's, and every
+    row's block scales and codes match under it."""
     w = wl.WORKLOADS[key]
-    inp = wl.make_inputs(w)
-    y = oracle.rht(inp.values, inp.signs, w.block)       # every row: global amax
+    inp = P.full_inputs(key)
     codes, bs, ts = P.gpu_nvfp4(inp)
-    t_ref = oracle.nvfp4_tensor_scale(y)
+    t_ref = P.oracle_tensor_scale(inp)
     assert np.float32(ts).view(np.uint32) == t_ref.view(np.uint32)
-    rows = _sample_rows(w.tokens, 96, 2)
-    gmax_row = int(np.argmax(np.abs(y).max(axis=1)))
-    rows = np.unique(np.append(rows, gmax_row))
-    P.check_nvfp4(codes[rows], bs[rows], ts, y[rows], tensor_scale=t_ref)
+    c = P.check_all_rows(f"full {key} nvfp4 dynamic", inp, (codes, bs, ts), tensor_scale=t_ref)
+    assert c.rows == w.tokens and c.scale_mismatch == 0 and c.bad == 0
     if key == "c4":
+        # round trip through the two calls (dequant, then the inverse rotation)
         deq = P.gpu_dequant(kq.KQ_FMT_NVFP4, codes, bs, None, ts, w.tokens, w.dim)
         winv = wl.Workload("inv", w.tokens, w.dim, wl.F32, w.block, True, w.fmt, 0)
         back = P.gpu_rht(wl.Inputs(winv, deq.astype(np.float64), deq, inp.signs),
                          inverse=True)
-        want = oracle.rht_inverse(deq[rows].astype(np.float64), inp.signs, w.block)
-        P.check_rotation(back[rows], want)
+        for r0, r1 in P.row_chunks(w.tokens, w.dim):
+            want = oracle.rht_inverse(deq[r0:r1].astype(np.float64), inp.signs, w.block)
+            P.check_rotation(back[r0:r1], want)
+
+
+def test_full_size_nvfp4_static_headline():
+    """The call the benchmark's headline times: the 16384 x 4096 batch with a
+    static tensor scale (the oracle's own), every row."""
+    w = wl.WORKLOADS["c4"]
+    inp = P.full_inputs("c4")
+    t_ref = P.oracle_tensor_scale(inp)
+    codes, bs, ts = P.gpu_nvfp4(inp, tensor_scale=t_ref)
+    c = P.check_all_rows("full c4 nvfp4 static", inp, (codes, bs, ts), tensor_scale=t_ref)
+    assert c.rows == w.tokens and c.scale_mismatch == 0 and c.bad == 0
 
 
 # ------------------------------------------------ dequant + inverse rotation
@@ -325,13 +331,14 @@ def test_dequant_rht_inverse_zero_tokens():
 
 def test_full_size_dequant_rht_inverse_c4():
     """The benchmark's round-trip launch (16384 x 4096 NVFP4 -> fp32) on random
-    codes; sampled rows against the oracle, and every row against the
-    two-call path (dequant, then the inverse rotation) within fp32 rounding."""
+    codes: every row against the oracle, and against the two-call path
+    (dequant, then the inverse rotation) within fp32 rounding."""
     w = wl.WORKLOADS["c4"]
     ci = wl.make_coded_inputs(w)
     got = P.gpu_dequant_rht_inverse(ci)
-    rows = _rows_with_tail(w.tokens, 64, 5)
-    P.check_rotation(got[rows], P.oracle_dequant_rht_inverse(ci, rows))
+    for r0, r1 in P.row_chunks(w.tokens, w.dim):
+        rows = np.arange(r0, r1)
+        P.check_rotation(got[rows], P.oracle_dequant_rht_inverse(ci, rows))
     deq = P.gpu_dequant(kq.KQ_FMT_NVFP4, ci.codes, ci.scales, None, ci.tensor_scale,
                         w.tokens, w.dim)
     winv = wl.Workload("inv", w.tokens, w.dim, wl.F32, w.block, True, w.fmt, 0)
@@ -377,11 +384,14 @@ def test_mxfp4_round_trip_fused():
 
 def test_full_size_mxfp4_c4():
     w = wl.WORKLOADS["c4"]
-    inp = wl.make_inputs(w)
-    rows = _sample_rows(w.tokens, 96, 7)
+    inp = P.full_inputs("c4")
     codes, scales = P.gpu_mxfp4(inp)
-    y = oracle.rht(inp.values[rows], inp.signs, w.block)
-    P.check_mxfp4(codes[rows], scales[rows], y)
+    total = P.Counts()
+    for r0, r1 in P.row_chunks(w.tokens, w.dim):
+        y = oracle.rht(inp.values[r0:r1], inp.signs, w.block)
+        total = total + P.check_mxfp4(codes[r0:r1], scales[r0:r1], y, name=False)
+    P.record("full c4 mxfp4", total)
+    assert total.rows == w.tokens
 
 
 # -------------------------------------------------------- KV-cache writer

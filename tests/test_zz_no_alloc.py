@@ -69,3 +69,45 @@ def test_noalloc_rejects_too_many_tokens():
     P = 1 << 20
     st = L.kq_rht_quant_nvfp4_dynamic_noalloc(P, kq.KQ_BF16, big, 4096, 0, None, P, P, P, None)
     assert st == kq.KQ_ERR_UNSUPPORTED
+
+
+def _call_pair(L, x, s, tokens, dim, block, stream):
+    """(reference with a fresh workspace, allocation-free) outputs of one input."""
+    c_ref, b_ref, t_ref, ws = kq.empty_nvfp4(tokens, dim, block)
+    st = L.kq_rht_quant_nvfp4(x.data_ptr(), kq.KQ_BF16, tokens, dim, block, s.data_ptr(),
+                              c_ref.data_ptr(), b_ref.data_ptr(), t_ref.data_ptr(),
+                              ws.data_ptr(), ws.numel(), kq.KQ_SCALE_DYNAMIC, stream)
+    assert st == kq.KQ_OK, kq.status_str(st)
+    c = torch.full_like(c_ref, 0xAB)
+    b = torch.full_like(b_ref, 0xCD)
+    t = torch.full_like(t_ref, -1.0)
+    st = L.kq_rht_quant_nvfp4_dynamic_noalloc(x.data_ptr(), kq.KQ_BF16, tokens, dim, block,
+                                              s.data_ptr(), c.data_ptr(), b.data_ptr(),
+                                              t.data_ptr(), stream)
+    assert st == kq.KQ_OK, kq.status_str(st)
+    torch.cuda.synchronize()
+    return (c_ref, b_ref, t_ref), (c, b, t)
+
+
+@pytest.mark.parametrize("dim", [2048, 12288])
+def test_noalloc_dirty_scratch_header_only_paths(dim):
+    """Paths that clear only the scratch's header (the warp-per-row kernel for
+    2048-wide rows, the row-per-CTA kernel for 12288) rely on their statistics
+    pass rewriting every row entry before the global step reads it: a larger
+    call leaves the scratch dirty, then a smaller call must still match."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    L = kq.lib()
+    stream = torch.cuda.current_stream().cuda_stream
+    big, small = 600, 37
+    w = wl.Workload("c4", big, dim, wl.BF16, 0, True, wl.NVFP4, seed=dim)
+    inp = wl.make_inputs(w)
+    x = torch.from_numpy(inp.stored.view(np.int16)).cuda().view(torch.bfloat16)
+    s = torch.from_numpy(inp.signs).cuda()
+    # the small call's rows get the largest values, so stale entries of the
+    # big call (smaller maxima) cannot hide a missed rewrite
+    x_small = (x[:small].float() * 4).to(torch.bfloat16).contiguous()
+    for xx, n in ((x, big), (x_small, small)):
+        ref, got = _call_pair(L, xx, s, n, dim, 0, stream)
+        for a, b in zip(ref, got):
+            assert torch.equal(a.view(torch.uint8), b.view(torch.uint8))
