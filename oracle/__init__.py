@@ -15,6 +15,9 @@ What it computes, in plain fp64 numpy:
     16 elements, fp32 tensor scale), plus their dequantizers -- `quant.py`.
   * The number formats E2M1, E4M3 and fp16 written from their public
     definitions -- `formats.py`.
+  * The 4-bit GEMM that consumes NVFP4 activations and weights, C = A_hat .
+    B_hat^T in float64, and the tensor-core scale-factor layout of the block
+    scales -- `gemm.py` (imported as `oracle.gemm`).
 
 Every function cites the passage of the source pages it follows.  Readings of
 points the pages leave open are listed in the module docstrings.
@@ -24,6 +27,7 @@ closed forms, brute force on tiny inputs, invariants (orthogonality, norm
 preservation, exact inverse, half-step bounds) and exhaustive format tables.
 """
 
+from . import gemm  # noqa: F401
 from .hadamard import hadamard, paley12, sylvester, quadratic_residues  # noqa: F401
 from .rht import rht, rht_inverse, rht_unnormalized  # noqa: F401
 from .formats import (  # noqa: F401

@@ -18,7 +18,7 @@ import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 PINS = ["test_oracle_hadamard.py", "test_oracle_rht.py", "test_oracle_quant.py",
-        "test_oracle_formats.py"]
+        "test_oracle_formats.py", "test_oracle_gemm.py"]
 
 # (name, oracle file, text, replacement)
 MUTANTS = [
@@ -43,6 +43,11 @@ MUTANTS = [
      "even = tie & ((np.arange(8) & 1) == 1)[None, :]"),
     ("E4M3 exponent bias 8", "formats.py",
      "mag = (1.0 + m / 8.0) * 2.0 ** (e - 7)", "mag = (1.0 + m / 8.0) * 2.0 ** (e - 8)"),
+    ("GEMM without the B tensor scale", "gemm.py",
+     "* (np.float64(np.float32(ta)) * np.float64(np.float32(tb)))", "* np.float64(np.float32(ta))"),
+    ("scale layout with row groups and lanes swapped", "gemm.py",
+     "np.ascontiguousarray(t.transpose(0, 3, 2, 1, 4)).reshape(-1)",
+     "np.ascontiguousarray(t.transpose(0, 3, 1, 2, 4)).reshape(-1)"),
 ]
 
 
