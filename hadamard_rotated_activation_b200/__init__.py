@@ -30,6 +30,7 @@ KQ_BF16 = 1
 KQ_INVERSE = 1
 KQ_SCALE_STATIC = 2
 KQ_SCALE_DYNAMIC = 4
+KQ_SCALES_MMA = 8
 
 KQ_FMT_INT4_SYM = 0
 KQ_FMT_INT4_ASYM = 1
@@ -42,6 +43,7 @@ C_SYMBOLS = (
     "kq_device_errors", "kq_diag_wait_timeout",
     "kq_workspace_size", "kq_status_str", "kq_last_cuda_error", "kq_version",
     "kq_rht_quant_nvfp4_dynamic_noalloc", "kq_diag_tc_steps", "kq_diag_fail_next_launch",
+    "kq_gemm_nvfp4",
 )
 
 # Fixed device scratch of kq_rht_quant_nvfp4_dynamic_noalloc (see include/kq.h).
@@ -105,6 +107,8 @@ def lib() -> ctypes.CDLL:
     L.kq_diag_tc_steps.restype = i32
     L.kq_diag_fail_next_launch.argtypes = [i32]
     L.kq_diag_fail_next_launch.restype = None
+    L.kq_gemm_nvfp4.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, i32, vp]
+    L.kq_gemm_nvfp4.restype = i32
     _lib = L
     return L
 
@@ -168,13 +172,17 @@ def kq_rht_quant_int4(x, block: int, signs, group: int, asym: bool, codes, scale
 
 
 def kq_rht_quant_nvfp4(x, block: int, signs, codes, block_scales, tensor_scale,
-                       workspace=None, dynamic: bool = True, stream=None) -> None:
+                       workspace=None, dynamic: bool = True, stream=None,
+                       mma_layout: bool = False) -> None:
     """Rotation + NVFP4 (E2M1 codes, E4M3 scale per 16, fp32 tensor scale).
     dynamic=True computes and writes the tensor scale (needs `workspace` of
-    kq_workspace_size bytes); dynamic=False reads it."""
+    kq_workspace_size bytes); dynamic=False reads it.  mma_layout=True writes
+    the block scales in the tensor-core layout kq_gemm_nvfp4 reads (a buffer
+    of sf_mma_bytes(tokens, dim) bytes)."""
     t, n = x.shape
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    flags = KQ_SCALE_DYNAMIC if dynamic else KQ_SCALE_STATIC
+    flags = (KQ_SCALE_DYNAMIC if dynamic else KQ_SCALE_STATIC) | (KQ_SCALES_MMA if mma_layout
+                                                                   else 0)
     _check(lib().kq_rht_quant_nvfp4(_ptr(x), _dtype_code(x), t, n, block, _ptr(signs),
                                     _ptr(codes), _ptr(block_scales), _ptr(tensor_scale),
                                     _ptr(workspace), ws_bytes, flags, _stream(stream)),
@@ -212,6 +220,19 @@ def kq_rht_quant_nvfp4_dynamic_noalloc(x, block: int, signs, codes, block_scales
         _ptr(tensor_scale), _stream(stream)), "kq_rht_quant_nvfp4_dynamic_noalloc")
 
 
+def kq_gemm_nvfp4(a_codes, a_scales, a_tensor_scale, b_codes, b_scales, b_tensor_scale, c,
+                  stream=None) -> None:
+    """C = ta tb A_q B_q^T on the block-scaled tensor cores: A [m, k/2] and B
+    [n, k/2] packed E2M1 codes with block scales in the tensor-core layout
+    (kq_rht_quant_nvfp4(..., mma_layout=True)); C [m, n] fp32 or bf16."""
+    m, kb = a_codes.shape
+    n = b_codes.shape[0]
+    _check(lib().kq_gemm_nvfp4(_ptr(a_codes), _ptr(a_scales), _ptr(a_tensor_scale),
+                               _ptr(b_codes), _ptr(b_scales), _ptr(b_tensor_scale), m, n,
+                               2 * kb, _ptr(c), _dtype_code(c), _stream(stream)),
+           "kq_gemm_nvfp4")
+
+
 def kq_dequant(fmt: int, codes, scales, zeros, tensor_scale, tokens: int, dim: int,
                group: int, out, stream=None) -> None:
     """Codes and scales back to fp32 (exact product, one rounding)."""
@@ -239,10 +260,11 @@ def kq_diag_tc_steps(a, b, d1, d2, status, stream=None) -> None:
 
 
 def kq_device_errors():
-    """The five error words of the tensor-core kernel families (read and
+    """The six error words of the tensor-core kernel families (read and
     cleared): 4096-wide, 12288-wide, block-128 GEMM, fused inverse,
-    diagnostic.  All zero: no bounded wait ran out since the last call."""
-    buf = (ctypes.c_uint * 5)()
+    diagnostic, NVFP4 GEMM.  All zero: no bounded wait ran out since the last
+    call."""
+    buf = (ctypes.c_uint * 6)()
     _check(lib().kq_device_errors(buf), "kq_device_errors")
     return list(buf)
 
@@ -283,11 +305,21 @@ def empty_mxfp4(tokens: int, dim: int, device="cuda"):
             torch.empty((tokens, dim // 32), dtype=torch.uint8, device=device))
 
 
-def empty_nvfp4(tokens: int, dim: int, block: int = 0, device="cuda"):
-    """(codes, block_scales, tensor_scale, workspace) for kq_rht_quant_nvfp4."""
+def sf_mma_bytes(rows: int, dim: int) -> int:
+    """Bytes of NVFP4 block scales in the tensor-core layout: rows padded to a
+    multiple of 128, dim / 16 scales a row (dim % 64 == 0)."""
+    return -(-rows // 128) * 128 * (dim // 16)
+
+
+def empty_nvfp4(tokens: int, dim: int, block: int = 0, device="cuda", mma_layout=False):
+    """(codes, block_scales, tensor_scale, workspace) for kq_rht_quant_nvfp4;
+    with mma_layout the block scales are a flat buffer of sf_mma_bytes."""
     import torch
     ws = kq_workspace_size(tokens, dim, block)
+    scales = (torch.zeros((sf_mma_bytes(tokens, dim),), dtype=torch.uint8, device=device)
+              if mma_layout else
+              torch.empty((tokens, dim // 16), dtype=torch.uint8, device=device))
     return (torch.empty((tokens, dim // 2), dtype=torch.uint8, device=device),
-            torch.empty((tokens, dim // 16), dtype=torch.uint8, device=device),
+            scales,
             torch.empty((1,), dtype=torch.float32, device=device),
             torch.empty((max(ws, 16),), dtype=torch.uint8, device=device))

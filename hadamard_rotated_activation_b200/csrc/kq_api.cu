@@ -42,6 +42,7 @@ kq_status make_geometry(int dim, int block, kq::Geometry* g) {
   g->depth = ilog2(g->m) + (g->paley ? 11 : 0);
   g->sqrt_b = std::sqrt((double)b);
   g->inv_sqrt_b = (float)(1.0 / g->sqrt_b);
+  g->sf_kc4 = 0;
   return KQ_OK;
 }
 
@@ -233,9 +234,16 @@ KQ_API kq_status kq_rht_quant_nvfp4(const void* x, int dtype, int64_t tokens, in
   if (st != KQ_OK) return st;
   if (tokens > 0 && (!codes || !block_scales || !tensor_scale)) return KQ_ERR_INVALID_ARG;
   const int mode = flags & (KQ_SCALE_STATIC | KQ_SCALE_DYNAMIC);
-  if ((flags & ~(KQ_SCALE_STATIC | KQ_SCALE_DYNAMIC)) != 0) return KQ_ERR_INVALID_ARG;
+  if ((flags & ~(KQ_SCALE_STATIC | KQ_SCALE_DYNAMIC | KQ_SCALES_MMA)) != 0)
+    return KQ_ERR_INVALID_ARG;
   if (mode != KQ_SCALE_STATIC && mode != KQ_SCALE_DYNAMIC) return KQ_ERR_INVALID_ARG;
   if (!aligned(codes, 16) || !aligned(tensor_scale, 4)) return KQ_ERR_MISALIGNED;
+  if (flags & KQ_SCALES_MMA) {
+    // tensor-core scale-factor layout: whole 4-block atoms per row
+    if (dim % 64 != 0) return KQ_ERR_UNSUPPORTED;
+    if (!aligned(block_scales, 16)) return KQ_ERR_MISALIGNED;
+    g.sf_kc4 = dim / 64;
+  }
   kq::NvWorkspace* ws = nullptr;
   if (mode == KQ_SCALE_DYNAMIC) {
     if ((tokens > 0 && !workspace) || ws_bytes < nv_workspace_bytes(tokens))
@@ -323,6 +331,30 @@ KQ_API kq_status kq_dequant_rht_inverse(int fmt, const uint8_t* codes, const voi
   });
 }
 
+KQ_API kq_status kq_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_scales,
+                               const float* a_tensor_scale, const uint8_t* b_codes,
+                               const uint8_t* b_scales, const float* b_tensor_scale, int64_t m,
+                               int64_t n, int64_t k, void* c, int c_dtype, kq_stream_t stream) {
+  if (m < 0 || n <= 0 || k <= 0) return KQ_ERR_INVALID_ARG;
+  if (c_dtype != KQ_F32 && c_dtype != KQ_BF16) return KQ_ERR_UNSUPPORTED;
+  if (n % 128 != 0 || k % 256 != 0) return KQ_ERR_UNSUPPORTED;
+  // TMA coordinates are 32-bit: rows and row bytes below 2^31
+  if (m >= (int64_t(1) << 31) || n >= (int64_t(1) << 31) || k >= (int64_t(1) << 32))
+    return KQ_ERR_UNSUPPORTED;
+  if (m == 0) return KQ_OK;
+  if (!a_codes || !a_scales || !a_tensor_scale || !b_codes || !b_scales || !b_tensor_scale || !c)
+    return KQ_ERR_INVALID_ARG;
+  if (!aligned(a_codes, 16) || !aligned(b_codes, 16) || !aligned(a_scales, 16) ||
+      !aligned(b_scales, 16) || !aligned(c, 16) || !aligned(a_tensor_scale, 4) ||
+      !aligned(b_tensor_scale, 4))
+    return KQ_ERR_MISALIGNED;
+  return dispatch([&] {
+    return kq::launch_gemm_nvfp4(a_codes, a_scales, a_tensor_scale, b_codes, b_scales,
+                                 b_tensor_scale, m, n, k, c, c_dtype == KQ_BF16 ? 1 : 0,
+                                 reinterpret_cast<cudaStream_t>(stream));
+  });
+}
+
 KQ_API kq_status kq_device_errors(unsigned int* flags) {
   if (!flags) return KQ_ERR_INVALID_ARG;
   cudaError_t e = kq::take_tc_errors(&flags[0]);
@@ -330,6 +362,7 @@ KQ_API kq_status kq_device_errors(unsigned int* flags) {
   if (e == cudaSuccess) e = kq::take_tcb_errors(&flags[2]);
   if (e == cudaSuccess) e = kq::take_tci_errors(&flags[3]);
   if (e == cudaSuccess) e = kq::take_diag_errors(&flags[4]);
+  if (e == cudaSuccess) e = kq::take_gemm_errors(&flags[5]);
   return finish(e);
 }
 
@@ -361,7 +394,7 @@ KQ_API int kq_last_cuda_error(void) { return g_last_cuda_error; }
 
 KQ_API void kq_diag_fail_next_launch(int cuda_error) { g_fail_next_launch = cuda_error; }
 
-KQ_API int kq_version(void) { return (1 << 16) | 0; }
+KQ_API int kq_version(void) { return (1 << 16) | 1; }
 
 KQ_API kq_status kq_diag_tc_steps(const uint16_t* a, const uint16_t* b, float* d1, float* d2,
                                   unsigned int* status, kq_stream_t stream) {

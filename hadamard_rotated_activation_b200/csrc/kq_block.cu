@@ -43,6 +43,7 @@ struct Params {
   int64_t num_slots;
   int n;
   float e_coef;                 // E = e_coef * max|S_hat| (rounded up)
+  int sf_kc4;                   // NVFP4 scale layout (Geometry::sf_kc4)
 };
 
 __device__ __forceinline__ int stage_chunk(int unit, int c);
@@ -381,7 +382,17 @@ k_blk128_nvfp4(Params P) {
       }
       if (active) dst[k] = make_uint4(words[0], words[1], words[2], words[3]);
     }
-    if (active) *reinterpret_cast<uint2*>(P.scales8 + u * (B / 16)) = make_uint2(sc[0], sc[1]);
+    if (active) {
+      if (P.sf_kc4 == 0) {
+        *reinterpret_cast<uint2*>(P.scales8 + u * (B / 16)) = make_uint2(sc[0], sc[1]);
+      } else {
+        // blocks 8 kk .. 8 kk + 7 of the row: two words of the tensor-core layout
+        const int c0 = (int)(u & (kpr - 1)) * (B / 16);
+        *reinterpret_cast<uint32_t*>(P.scales8 + sf_offset(row, c0, P.n / 16, P.sf_kc4)) = sc[0];
+        *reinterpret_cast<uint32_t*>(P.scales8 + sf_offset(row, c0 + 4, P.n / 16, P.sf_kc4)) =
+            sc[1];
+      }
+    }
   }
 }
 
@@ -563,6 +574,7 @@ cudaError_t launch_blk128_nvfp4(const void* x, int64_t tokens, const Geometry& g
   P.units = tokens * (g.n / blk::B);
   P.n = g.n;
   P.e_coef = e_coef_128();
+  P.sf_kc4 = g.sf_kc4;
   if (ws) {
     cudaError_t e = cudaMemsetAsync(ws, 0, kNvWorkspaceHeader + (size_t)tokens * sizeof(float2), s);
     if (e != cudaSuccess) return e;

@@ -91,7 +91,21 @@ struct Geometry {
   int depth;      // roundings along any input -> output path of the fp32 transform
   float inv_sqrt_b;
   double sqrt_b;
+  int sf_kc4;     // NVFP4 block scales: 0 = row-major [T, n/16]; else the tensor-core
+                  // scale-factor layout with sf_kc4 = n/64 atoms per 128-row block
 };
+
+// Byte offset of the NVFP4 block scale of 16-block c in row `row` (nb blocks a
+// row).  Row-major when kc4 == 0.  Otherwise the layout a tcgen05 block-scaled
+// MMA takes from tensor memory: 512-byte atoms of 128 rows x 4 blocks, lane
+// row % 32 holding 16 bytes, byte 4 ((row / 32) % 4) + c % 4; atoms ordered by
+// c / 4 within a 128-row block, then by row block.  Four blocks 4j .. 4j+3 of
+// a row are one aligned 32-bit word in both layouts.
+__device__ __forceinline__ int64_t sf_offset(int64_t row, int c, int nb, int kc4) {
+  if (kc4 == 0) return row * nb + c;
+  return (((row >> 7) * kc4 + (c >> 2)) << 9) + ((row & 31) << 4) + (((row >> 5) & 3) << 2) +
+         (c & 3);
+}
 
 // Rigorous bound on |S_hat - S| for every output of one Hadamard block, from
 // the computed maximum |S_hat| of that block (or any larger value).

@@ -27,6 +27,21 @@ constexpr size_t kNvWorkspaceHeader = 16;
 bool encode_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
                          uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swizzle);
 
+// General 2-D tensor map: `rows` rows of `row_bytes` bytes (a multiple of 16),
+// `cols` elements of the given type a row, boxes of box_cols x box_rows.
+bool encode_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
+                    uint32_t elem_bytes, uint64_t cols, uint64_t rows, uint64_t row_bytes,
+                    uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swizzle);
+
+// NVFP4 x NVFP4 GEMM on the block-scaled tensor cores (kq_gemm.cu):
+// C[M, N] = t_a t_b sum_k A[m][k] B[n][k], codes K-major, block scales in the
+// tensor-core layout (Geometry::sf_kc4), C fp32 or bf16 row-major.
+cudaError_t launch_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_scales,
+                              const float* a_tscale, const uint8_t* b_codes,
+                              const uint8_t* b_scales, const float* b_tscale, int64_t m,
+                              int64_t n, int64_t k, void* c, int c_bf16, cudaStream_t s);
+cudaError_t take_gemm_errors(unsigned int* out);
+
 // Records a CUDA error for kq_last_cuda_error() on the calling thread.
 void set_last_cuda_error(int err);
 

@@ -44,6 +44,7 @@ struct Params {
   NvWorkspace* ws;              // NVFP4 dynamic
   int64_t tokens;
   float gamma;                  // gamma_L with a safety factor (rounded up)
+  int sf_kc4;                   // NVFP4 scale layout (Geometry::sf_kc4)
 };
 
 __device__ __forceinline__ void bfly2(float2& a, float2& b) {
@@ -430,10 +431,17 @@ k_rowwarp(Params P) {
       cw[k] = make_uint4(words[0], words[1], words[2], words[3]);
     }
     store_row_codes<N>(tbuf, cw, P.codes + row * (N / 2));
-    if (NB == 8)
+    if (P.sf_kc4 != 0) {
+      // one or two words of the tensor-core layout
+#pragma unroll
+      for (int j = 0; j < NB / 4; ++j)
+        *reinterpret_cast<uint32_t*>(P.scales8 + sf_offset(row, lane * NB + 4 * j, N / 16,
+                                                           P.sf_kc4)) = sc[j];
+    } else if (NB == 8) {
       *reinterpret_cast<uint2*>(P.scales8 + row * (N / 16) + lane * NB) = make_uint2(sc[0], sc[1]);
-    else
+    } else {
       *reinterpret_cast<uint32_t*>(P.scales8 + row * (N / 16) + lane * NB) = sc[0];
+    }
   }
 }
 
@@ -500,6 +508,7 @@ cudaError_t launch_rowwarp_nvfp4(const void* x, int dtype, int64_t tokens, const
   P.tensor_scale = tensor_scale;
   P.ws = ws;
   P.tokens = tokens;
+  P.sf_kc4 = g.sf_kc4;
   P.gamma = gamma_for(g.n == 4096 ? 12 : 11);
   if (ws) {
     cudaError_t e = cudaMemsetAsync(ws, 0, kNvWorkspaceHeader, s);

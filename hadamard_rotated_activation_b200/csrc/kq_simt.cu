@@ -554,7 +554,7 @@ k_nvfp4(const T* __restrict__ x, const int8_t* __restrict__ signs,
         }
         crow[k] = make_uint2(w0, w1);
       }
-      bscales[row * nb + k] = (uint8_t)sc;
+      bscales[sf_offset(row, k, nb, g.sf_kc4)] = (uint8_t)sc;
     }
     __syncthreads();
   }

@@ -102,6 +102,7 @@ struct Params {
   float* out;                   // kRot: fp32 [T, n]
   int64_t tokens;
   int64_t tiles;
+  int sf_kc4;                   // NVFP4 scale layout (Geometry::sf_kc4)
 };
 
 // --------------------------------------------------------------- helpers
@@ -722,7 +723,8 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
         if (valid) {
           *reinterpret_cast<uint4*>(P.codes + token * (N / 2) + o * 16) =
               make_uint4(words[0], words[1], words[2], words[3]);
-          *reinterpret_cast<uint16_t*>(P.scales8 + token * (N / 16) + o * 2) = (uint16_t)sc;
+          *reinterpret_cast<uint16_t*>(P.scales8 + sf_offset(token, o * 2, N / 16, P.sf_kc4)) =
+              (uint16_t)sc;
         }
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
@@ -815,7 +817,7 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
             nvfp4_block_words(reinterpret_cast<const float2*>(fe.v), code, inv_bt, ts, srcp, w0,
                               w1);
             *reinterpret_cast<uint2*>(P.codes + token * (N / 2) + blk * 8) = make_uint2(w0, w1);
-            P.scales8[token * (N / 16) + blk] = (uint8_t)code;
+            P.scales8[sf_offset(token, blk, N / 16, P.sf_kc4)] = (uint8_t)code;
           }
           __syncwarp();
           if (lane == 0) st_release(&fq->cons[h % kQ], h + 1);
@@ -983,6 +985,22 @@ bool encode_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t cols, uint
   return r == CUDA_SUCCESS;
 }
 
+bool encode_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
+                    uint32_t elem_bytes, uint64_t cols, uint64_t rows, uint64_t row_bytes,
+                    uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swizzle) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t gstride[1] = {(cuuint64_t)row_bytes};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estride[2] = {1, 1};
+  (void)elem_bytes;
+  CUresult r = enc(map, dtype, 2, const_cast<void*>(base), gdim, gstride, box, estride,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool tc_row_supported(const Geometry& g, int dtype, const void* x, int64_t tokens) {
   // TMA: 16-byte aligned base, int32 row coordinates
   return dtype == 1 && !g.paley && g.b == g.n && g.n == 4096 &&
@@ -999,6 +1017,7 @@ cudaError_t launch_tc_nvfp4(const void* x, int64_t tokens, const Geometry& g,
   P.tensor_scale = tensor_scale;
   P.ws = ws;
   P.tokens = tokens;
+  P.sf_kc4 = g.sf_kc4;
   cudaError_t e;
   if (ws) {
     e = cudaMemsetAsync(ws, 0, kNvWorkspaceHeader + (size_t)tokens * sizeof(float2), s);

@@ -109,7 +109,8 @@ typedef enum { KQ_F32 = 0, KQ_BF16 = 1 } kq_dtype;
 enum {
   KQ_INVERSE = 1,        /* kq_rht: inverse transform x = D H^T y / sqrt(b) */
   KQ_SCALE_STATIC = 2,   /* kq_rht_quant_nvfp4: *tensor_scale is an input */
-  KQ_SCALE_DYNAMIC = 4   /* kq_rht_quant_nvfp4: *tensor_scale is computed and written */
+  KQ_SCALE_DYNAMIC = 4,  /* kq_rht_quant_nvfp4: *tensor_scale is computed and written */
+  KQ_SCALES_MMA = 8      /* kq_rht_quant_nvfp4: block scales in the tensor-core layout */
 };
 
 /* formats for kq_dequant */
@@ -180,6 +181,15 @@ KQ_API kq_status kq_rht_quant_int4_kv(const void* x, int dtype, int64_t tokens,
  * entry do not matter and are clobbered.  Static mode ignores it.
  * codes: [tokens, dim/2]; block_scales: E4M3 [tokens, dim/16]; tensor_scale:
  * one fp32 in device memory.
+ * KQ_SCALES_MMA (optional, needs dim % 64 == 0 and 16-byte aligned
+ * block_scales) writes the block scales instead in the scale-factor layout of
+ * the tcgen05 block-scaled MMA, which kq_gemm_nvfp4 reads: 512-byte atoms of
+ * 128 rows x 4 blocks; the scale of row r, block c sits at byte
+ * ((r / 128) * (dim / 64) + c / 4) * 512 + (r % 32) * 16 + ((r / 32) % 4) * 4 + c % 4.
+ * The buffer then holds ceil(tokens / 128) * 128 * dim / 16 bytes; the bytes of
+ * the padding rows are not written.  Codes and scale values are the same as
+ * without the flag.  kq_dequant and kq_dequant_rht_inverse read the row-major
+ * layout only.
  */
 KQ_API kq_status kq_rht_quant_nvfp4(const void* x, int dtype, int64_t tokens,
                                     int dim, int block, const int8_t* signs,
@@ -246,15 +256,44 @@ KQ_API kq_status kq_dequant_rht_inverse(int fmt, const uint8_t* codes,
                                         int out_dtype, kq_stream_t stream);
 
 /*
+ * kq_gemm_nvfp4 -- the 4-bit GEMM that consumes rotated, NVFP4-quantized
+ * activations (QuaRot reviews, review 2 and review 4 Strengths: the speedup of
+ * the rotated 4-bit path is the 4-bit GEMM; review 3 Questions: with Y = X H^T
+ * applied to activations and weights alike, X W^T is unchanged), run on the
+ * block-scaled tensor cores:
+ *   C[m][n] = ta * tb * sum_k (E2M1(a[m][k]) E4M3(sa[m][k/16]))
+ *                             (E2M1(b[n][k]) E4M3(sb[n][k/16])),
+ * accumulated in fp32, scaled by ta * tb (fp32) and stored as fp32 or bf16.
+ *   a_codes  [m, k/2] packed E2M1 codes (element 2i in the low nibble), as
+ *            kq_rht_quant_nvfp4 writes them;  b_codes [n, k/2] likewise.
+ *   a_scales, b_scales  E4M3 block scales in the KQ_SCALES_MMA layout, buffers
+ *            of ceil(rows / 128) * 128 * k / 16 bytes (padding rows are read;
+ *            their products reach only output rows that are not stored).
+ *   a_tensor_scale, b_tensor_scale  one fp32 each, device memory.
+ *   c        [m, n] row-major, c_dtype KQ_F32 or KQ_BF16 (round to nearest even).
+ * Device pointers owned by the caller, 16-byte aligned (tensor scales 4);
+ * C must not alias the inputs.  Supported: m >= 0 (m == 0 is a no-op),
+ * n % 128 == 0, k % 256 == 0.  Errors: KQ_ERR_INVALID_ARG (null pointer,
+ * non-positive n or k), KQ_ERR_UNSUPPORTED (shape or c_dtype),
+ * KQ_ERR_MISALIGNED, KQ_ERR_CUDA; nothing is launched on an error.
+ */
+KQ_API kq_status kq_gemm_nvfp4(const uint8_t* a_codes, const uint8_t* a_scales,
+                               const float* a_tensor_scale, const uint8_t* b_codes,
+                               const uint8_t* b_scales, const float* b_tensor_scale,
+                               int64_t m, int64_t n, int64_t k, void* c, int c_dtype,
+                               kq_stream_t stream);
+
+/*
  * kq_device_errors -- failure reports of the tensor-core kernels.  Every
  * wait of those kernels is bounded (about two seconds); when one runs out the
  * kernel records it in its family's error word and returns without writing
- * the affected outputs, instead of hanging.  flags: host array of 5 words,
+ * the affected outputs, instead of hanging.  flags: host array of 6 words,
  * filled and then cleared on the device: [0] the 4096-wide kernels (bit 0: a
  * wait ran out; bit 1: the fix-up queue stayed full, a block kept its
  * provisional scale; bit 2: a fix-up warp waited too long), [1] the
  * 12288-wide kernel, [2] the block-128 GEMM kernel, [3] the fused dequant +
- * inverse kernel, [4] kq_diag_wait_timeout (bit 0).  All zero: no failure
+ * inverse kernel, [4] kq_diag_wait_timeout (bit 0), [5] the NVFP4 GEMM
+ * (since ABI version 1.1; 1.0 had 5 words).  All zero: no failure
  * since the last call.  The read synchronizes the device.  The pages have no
  * counterpart to this entry point.
  */

@@ -201,3 +201,32 @@ def test_launch_failure_reaches_the_caller(L):
             kq._check(L.kq_rht(P, 1, 4, 4096, 0, None, Q, 0, None), "kq_rht")
     finally:
         L.kq_diag_fail_next_launch(0)
+
+
+def test_gemm_and_scale_layout_validation(L):
+    """Host-side checks of kq_gemm_nvfp4 and of the KQ_SCALES_MMA flag."""
+    g = L.kq_gemm_nvfp4
+    ok = (P, Q, P, Q, P, Q)
+    assert g(*ok, 0, 4096, 4096, Q, kq.KQ_F32, None) == kq.KQ_OK          # m = 0: no-op
+    assert g(*ok, -1, 4096, 4096, Q, kq.KQ_F32, None) == kq.KQ_ERR_INVALID_ARG
+    assert g(*ok, 4, 0, 4096, Q, kq.KQ_F32, None) == kq.KQ_ERR_INVALID_ARG
+    assert g(*ok, 4, 4096, 4096, Q, 7, None) == kq.KQ_ERR_UNSUPPORTED
+    assert g(*ok, 4, 4000, 4096, Q, kq.KQ_F32, None) == kq.KQ_ERR_UNSUPPORTED   # n % 128
+    assert g(*ok, 4, 4096, 4000, Q, kq.KQ_F32, None) == kq.KQ_ERR_UNSUPPORTED   # k % 256
+    assert g(None, Q, P, Q, P, Q, 4, 4096, 4096, Q, kq.KQ_F32, None) == kq.KQ_ERR_INVALID_ARG
+    assert g(P + 8, Q, P, Q, P, Q, 4, 4096, 4096, Q, kq.KQ_F32, None) == kq.KQ_ERR_MISALIGNED
+    assert g(*ok, 4, 4096, 4096, Q + 8, kq.KQ_BF16, None) == kq.KQ_ERR_MISALIGNED
+    f = L.kq_rht_quant_nvfp4
+    mma = kq.KQ_SCALE_STATIC | kq.KQ_SCALES_MMA
+    assert f(P, 1, 0, 4096, 0, None, Q, Q, Q, None, 0, mma, None) == kq.KQ_OK
+    assert f(P, 1, 4, 32, 0, None, Q, Q, Q, None, 0, mma, None) == kq.KQ_ERR_UNSUPPORTED
+    assert f(P, 1, 4, 4096, 0, None, Q, Q + 4, Q, None, 0, mma, None) == kq.KQ_ERR_MISALIGNED
+    assert f(P, 1, 4, 4096, 0, None, Q, Q, Q, None, 0, mma | 16, None) == kq.KQ_ERR_INVALID_ARG
+    try:
+        L.kq_diag_fail_next_launch(_LAUNCH_ERR)
+        assert g(*ok, 4, 4096, 4096, Q, kq.KQ_F32, None) == kq.KQ_ERR_CUDA
+        assert L.kq_last_cuda_error() == _LAUNCH_ERR
+        L.kq_diag_fail_next_launch(_LAUNCH_ERR)
+        assert f(P, 1, 4, 4096, 0, None, Q, Q, Q, None, 0, mma, None) == kq.KQ_ERR_CUDA
+    finally:
+        L.kq_diag_fail_next_launch(0)
