@@ -631,6 +631,7 @@ def extras(torch, kq, wl, dev, peak, args):
             del sets
         if key == "c4":
             out.update(roundtrip(torch, kq, wl, dev, peak, k, 5, 0, x0, signs))
+            out["c4_gemm_consumer"] = gemm_consumer(torch, kq, wl, dev, x0, signs, k)
             # the same batch as MXFP4 (E8M0 scale per 32 elements)
             mx_sets = [(x0 if i == 0 else x0.clone(),) + kq.empty_mxfp4(w.tokens, w.dim)
                        for i in range(n_sets(w.tokens * w.dim * 2))]
@@ -647,6 +648,52 @@ def extras(torch, kq, wl, dev, peak, args):
         del x0
         torch.cuda.empty_cache()
     return out, samples
+
+
+def fp4_peak_tflops():
+    """Dense FP4 tensor peak: the measured bf16 GEMM burst figure times the
+    nominal FP4 / bf16 ratio (9 / 2.25 = 4), or the fallback bf16 figure x 4."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return 4.0 * float(json.load(f)["bf16_tflops"]), "measured bf16 burst x 4"
+    except Exception:
+        return 4.0 * 1590.0, "fallback bf16 x 4"
+
+
+def gemm_consumer(torch, kq, wl, dev, x0, signs, k):
+    """The 4-bit GEMM that consumes the c4 batch: its rotated NVFP4 codes
+    (static tensor scale, block scales in the tensor-core layout) times a
+    4096 x 4096 weight rotated and quantized by the same call, fp32 out.  One
+    launch per step; the 268 MB output exceeds the L2 on every step."""
+    import numpy as np
+    t, n = x0.shape
+    rng = np.random.default_rng(44)
+    wt = wl.round_to_bf16(rng.standard_normal((n, n)) / np.sqrt(n))
+    wdev = torch.from_numpy(wl.bf16_bits(wt).view(np.int16)).to(dev).view(torch.bfloat16)
+    ops = []
+    for src, rows in ((x0, t), (wdev, n)):
+        c0, b0, t0, ws = kq.empty_nvfp4(rows, n, 0)
+        kq.kq_rht_quant_nvfp4(src, 0, signs, c0, b0, t0, ws, dynamic=True)
+        cm, bm, tm, _ = kq.empty_nvfp4(rows, n, 0, mma_layout=True)
+        tm.copy_(t0)
+        kq.kq_rht_quant_nvfp4(src, 0, signs, cm, bm, tm, None, dynamic=False, mma_layout=True)
+        ops.append((cm, bm, tm))
+    (ca, sa, ta), (cb, sb, tb) = ops
+    outs = [torch.empty((t, n), dtype=torch.float32, device=dev) for _ in range(2)]
+
+    def step(o):
+        kq.kq_gemm_nvfp4(ca, sa, ta, cb, sb, tb, o)
+    kk = max(5, min(k, 50))
+    ms = time_steps(torch, step, outs, kk, 3) / kk
+    flops = 2.0 * t * n * n
+    tf = flops / (ms * 1e-3) / 1e12
+    peak, kind = fp4_peak_tflops()
+    return {"ms": round(ms, 5), "TFLOP/s": round(tf, 1), "frac": round(tf / peak, 4),
+            "shape": f"M={t} N={n} K={n}", "flops": flops, "launches_per_step": 1,
+            "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": round(peak, 1),
+                         "unit": "TFLOP/s", "frac": round(tf / peak, 4), "peak_kind": kind,
+                         "traffic": None}}
 
 
 def roundtrip(torch, kq, wl, dev, peak, k, warmup, tokens=0, x0=None, signs=None):

@@ -43,7 +43,7 @@ C_SYMBOLS = (
     "kq_device_errors", "kq_diag_wait_timeout",
     "kq_workspace_size", "kq_status_str", "kq_last_cuda_error", "kq_version",
     "kq_rht_quant_nvfp4_dynamic_noalloc", "kq_diag_tc_steps", "kq_diag_fail_next_launch",
-    "kq_gemm_nvfp4",
+    "kq_gemm_nvfp4", "kq_diag_tc_steps_f16",
 )
 
 # Fixed device scratch of kq_rht_quant_nvfp4_dynamic_noalloc (see include/kq.h).
@@ -107,6 +107,8 @@ def lib() -> ctypes.CDLL:
     L.kq_diag_tc_steps.restype = i32
     L.kq_diag_fail_next_launch.argtypes = [i32]
     L.kq_diag_fail_next_launch.restype = None
+    L.kq_diag_tc_steps_f16.argtypes = [vp, vp, vp, vp, vp, vp]
+    L.kq_diag_tc_steps_f16.restype = i32
     L.kq_gemm_nvfp4.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, i32, vp]
     L.kq_gemm_nvfp4.restype = i32
     _lib = L
@@ -251,12 +253,13 @@ def kq_dequant_rht_inverse(fmt: int, codes, scales, zeros, tensor_scale, tokens:
            "kq_dequant_rht_inverse")
 
 
-def kq_diag_tc_steps(a, b, d1, d2, status, stream=None) -> None:
+def kq_diag_tc_steps(a, b, d1, d2, status, stream=None, fp16=False) -> None:
     """Two tensor-core accumulation steps on caller data (diagnostic; see
-    include/kq.h): a bf16 [128, 32], b bf16 [32, 128], d1/d2 fp32 [128, 128],
-    status one int32 (0 = the waits completed)."""
-    _check(lib().kq_diag_tc_steps(_ptr(a), _ptr(b), _ptr(d1), _ptr(d2), _ptr(status),
-                                  _stream(stream)), "kq_diag_tc_steps")
+    include/kq.h): a bf16 (fp16 with fp16=True) [128, 32], b [32, 128], d1/d2
+    fp32 [128, 128], status one int32 (0 = the waits completed)."""
+    fn = lib().kq_diag_tc_steps_f16 if fp16 else lib().kq_diag_tc_steps
+    _check(fn(_ptr(a), _ptr(b), _ptr(d1), _ptr(d2), _ptr(status), _stream(stream)),
+           "kq_diag_tc_steps")
 
 
 def kq_device_errors():

@@ -396,15 +396,26 @@ KQ_API void kq_diag_fail_next_launch(int cuda_error) { g_fail_next_launch = cuda
 
 KQ_API int kq_version(void) { return (1 << 16) | 1; }
 
-KQ_API kq_status kq_diag_tc_steps(const uint16_t* a, const uint16_t* b, float* d1, float* d2,
-                                  unsigned int* status, kq_stream_t stream) {
+static kq_status diag_tc_steps(const uint16_t* a, const uint16_t* b, float* d1, float* d2,
+                               unsigned int* status, int fp16, kq_stream_t stream) {
   if (!a || !b || !d1 || !d2 || !status) return KQ_ERR_INVALID_ARG;
   if (!aligned(a, 2) || !aligned(b, 2) || !aligned(d1, 4) || !aligned(d2, 4) ||
       !aligned(status, 4))
     return KQ_ERR_MISALIGNED;
   return dispatch([&] {
-    return kq::launch_diag_tc_steps(a, b, d1, d2, status, reinterpret_cast<cudaStream_t>(stream));
+    return kq::launch_diag_tc_steps(a, b, d1, d2, status, fp16,
+                                    reinterpret_cast<cudaStream_t>(stream));
   });
+}
+
+KQ_API kq_status kq_diag_tc_steps(const uint16_t* a, const uint16_t* b, float* d1, float* d2,
+                                  unsigned int* status, kq_stream_t stream) {
+  return diag_tc_steps(a, b, d1, d2, status, 0, stream);
+}
+
+KQ_API kq_status kq_diag_tc_steps_f16(const uint16_t* a, const uint16_t* b, float* d1,
+                                      float* d2, unsigned int* status, kq_stream_t stream) {
+  return diag_tc_steps(a, b, d1, d2, status, 1, stream);
 }
 
 }  // extern "C"

@@ -94,7 +94,7 @@ cudaError_t launch_tcp_int4(const void* x, int64_t tokens, const Geometry& g,
 cudaError_t launch_tcp_rot(const void* x, int64_t tokens, const Geometry& g,
                            const int8_t* signs, float* out, cudaStream_t s);
 cudaError_t launch_diag_tc_steps(const uint16_t* a, const uint16_t* b, float* d1, float* d2,
-                                 unsigned int* status, cudaStream_t s);
+                                 unsigned int* status, int fp16, cudaStream_t s);
 
 cudaError_t launch_tc_mxfp4(const void* x, int64_t tokens, const Geometry& g,
                             const int8_t* signs, uint8_t* codes, uint8_t* scales,

@@ -852,7 +852,7 @@ k_tc4096(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ si
 // tokens.  One CTA of 128 threads.
 __global__ void __launch_bounds__(128, 1)
 k_diag_steps(const uint16_t* __restrict__ a, const uint16_t* __restrict__ b, float* d1,
-             float* d2, unsigned int* status) {
+             float* d2, unsigned int* status, uint32_t idesc) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -889,7 +889,7 @@ k_diag_steps(const uint16_t* __restrict__ a, const uint16_t* __restrict__ b, flo
     if (threadIdx.x == 0) {
       const uint64_t adesc = smem_desc(smem_u32(sA) + step * 32, 16, 1024, 2);
       const uint64_t bdesc = smem_desc(smem_u32(sB) + step * 4096, kTokStride, 2048, 4);
-      mma_bf16(tmem, adesc, bdesc, (uint32_t)step);
+      sm100::mma_bf16(tmem, adesc, bdesc, idesc, (uint32_t)step);
       mma_commit(bar);
     }
     ok = mbar_wait(bar, (uint32_t)step) && ok;
@@ -1053,11 +1053,14 @@ cudaError_t launch_tc_rot(const void* x, int64_t tokens, const Geometry& g, cons
 }
 
 cudaError_t launch_diag_tc_steps(const uint16_t* a, const uint16_t* b, float* d1, float* d2,
-                                 unsigned int* status, cudaStream_t s) {
+                                 unsigned int* status, int fp16, cudaStream_t s) {
   constexpr int kDiagSmem = 1024 + 32768 + (int)tc::kStageBytes + 64;
   cudaFuncSetAttribute((const void*)tc::k_diag_steps, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        kDiagSmem);
-  tc::k_diag_steps<<<1, 128, kDiagSmem, s>>>(a, b, d1, d2, status);
+  // kind::f16 with bf16 operands (the forward kernels) or fp16 operands (the
+  // fused dequant + inverse kernel): A and B format fields 1 (bf16) or 0 (fp16)
+  const uint32_t idesc = fp16 ? (tc::kIdesc & ~((7u << 7) | (7u << 10))) : tc::kIdesc;
+  tc::k_diag_steps<<<1, 128, kDiagSmem, s>>>(a, b, d1, d2, status, idesc);
   return cudaGetLastError();
 }
 

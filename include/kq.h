@@ -378,6 +378,14 @@ KQ_API int kq_version(void);
 KQ_API kq_status kq_diag_tc_steps(const uint16_t* a, const uint16_t* b, float* d1, float* d2,
                                   unsigned int* status, kq_stream_t stream);
 
+/*
+ * Diagnostic: the same two steps with fp16 operands (a and b hold fp16 bits),
+ * the operand type of the fused dequant + inverse kernel.  Arguments, layout
+ * and errors as kq_diag_tc_steps.  The pages have no counterpart.
+ */
+KQ_API kq_status kq_diag_tc_steps_f16(const uint16_t* a, const uint16_t* b, float* d1,
+                                      float* d2, unsigned int* status, kq_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

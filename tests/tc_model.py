@@ -47,3 +47,23 @@ def mma_step(terms) -> float:
     emax = max(_floor_log2(t) for t in nz)
     grid = Fraction(2) ** (emax - 25)
     return to_f32_rz(sum(_trunc_to(t, grid) for t in nz))
+
+
+def mma_step_vec(terms: np.ndarray) -> np.ndarray:
+    """mma_step for many outputs at once: terms float64 [..., T] holding the
+    exact products and accumulator (T <= 64; every term a bf16 or fp16 value
+    times +-1, or an fp32 accumulator).  Exact in float64: dividing by the
+    power-of-two grid and truncating is exact, the truncated terms are
+    integers of at most 27 bits on that grid (|t| < 2^(emax+1)), so their sum
+    (under 2^33 grid units) is exact in any order; the final truncation to
+    fp32 is again a power-of-two scaling and a truncation.  Returns float32."""
+    t = np.asarray(terms, dtype=np.float64)
+    mx = np.max(np.abs(t), axis=-1)
+    nz = mx > 0
+    _, ex = np.frexp(np.where(nz, mx, 1.0))          # mx = f 2^ex, 0.5 <= f < 1
+    grid = np.ldexp(1.0, (ex - 1) - 25)[..., None]
+    s = np.sum(np.trunc(t / grid) * grid, axis=-1)
+    _, es = np.frexp(np.where(s != 0, np.abs(s), 1.0))
+    ulp = np.ldexp(1.0, np.maximum(es - 1, -126) - 23)
+    r = np.trunc(s / ulp) * ulp
+    return np.where(nz, r, 0.0).astype(np.float32)

@@ -30,8 +30,13 @@ def test_words_clear_after_ordinary_calls():
     kq.kq_rht_quant_nvfp4(x, 0, s, c, bs, ts, ws, dynamic=True)
     out = torch.empty((w.tokens, w.dim), dtype=torch.float32, device="cuda")
     kq.kq_rht(x, 0, s, out)
+    cm, bm, tm, _ = kq.empty_nvfp4(w.tokens, w.dim, 0, mma_layout=True)
+    tm.copy_(ts)
+    kq.kq_rht_quant_nvfp4(x, 0, s, cm, bm, tm, None, dynamic=False, mma_layout=True)
+    g = torch.empty((w.tokens, 128), dtype=torch.float32, device="cuda")
+    kq.kq_gemm_nvfp4(cm, bm, tm, cm[:128], bm[:kq.sf_mma_bytes(128, w.dim)], tm, g)
     torch.cuda.synchronize()
-    assert kq.kq_device_errors() == [0, 0, 0, 0, 0]
+    assert kq.kq_device_errors() == [0, 0, 0, 0, 0, 0]
 
 
 def test_bounded_wait_reports_and_clears():
