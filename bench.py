@@ -57,6 +57,9 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--roundtrip-only", action="store_true",
                    help="time only the c4 dequant + inverse round trip (one JSON line)")
+    p.add_argument("--gemm-only", action="store_true",
+                   help="time only the NVFP4 GEMM consumer of the c4 batch (one JSON line; "
+                        "--tokens sets M)")
     p.add_argument("--cpu-seconds", type=float, default=12.0,
                    help="target CPU time of the oracle baseline sample")
     return p.parse_args()
@@ -453,6 +456,16 @@ def main():
         if rank == 0:
             print(json.dumps(roundtrip(torch, kq, wl, dev, peak, args.steps, args.warmup,
                                        args.tokens)), flush=True)
+        if dist is not None:
+            dist.destroy_process_group()
+        return
+    if args.gemm_only:
+        if rank == 0:
+            inp = wl.make_inputs(w)
+            x0 = device_input(torch, inp, wl, dev)
+            sg = torch.from_numpy(inp.signs).to(dev)
+            print(json.dumps({"c4_gemm_consumer": gemm_consumer(torch, kq, wl, dev, x0, sg,
+                                                                 args.steps)}), flush=True)
         if dist is not None:
             dist.destroy_process_group()
         return

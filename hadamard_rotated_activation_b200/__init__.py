@@ -31,6 +31,9 @@ KQ_INVERSE = 1
 KQ_SCALE_STATIC = 2
 KQ_SCALE_DYNAMIC = 4
 KQ_SCALES_MMA = 8
+KQ_DYN_STATS = 16
+KQ_DYN_EXACT = 32
+KQ_DYN_QUANT = 64
 
 KQ_FMT_INT4_SYM = 0
 KQ_FMT_INT4_ASYM = 1
@@ -175,7 +178,7 @@ def kq_rht_quant_int4(x, block: int, signs, group: int, asym: bool, codes, scale
 
 def kq_rht_quant_nvfp4(x, block: int, signs, codes, block_scales, tensor_scale,
                        workspace=None, dynamic: bool = True, stream=None,
-                       mma_layout: bool = False) -> None:
+                       mma_layout: bool = False, phases: int = 0) -> None:
     """Rotation + NVFP4 (E2M1 codes, E4M3 scale per 16, fp32 tensor scale).
     dynamic=True computes and writes the tensor scale (needs `workspace` of
     kq_workspace_size bytes); dynamic=False reads it.  mma_layout=True writes
@@ -183,8 +186,8 @@ def kq_rht_quant_nvfp4(x, block: int, signs, codes, block_scales, tensor_scale,
     of sf_mma_bytes(tokens, dim) bytes)."""
     t, n = x.shape
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    flags = (KQ_SCALE_DYNAMIC if dynamic else KQ_SCALE_STATIC) | (KQ_SCALES_MMA if mma_layout
-                                                                   else 0)
+    flags = ((KQ_SCALE_DYNAMIC if dynamic else KQ_SCALE_STATIC) |
+             (KQ_SCALES_MMA if mma_layout else 0) | phases)
     _check(lib().kq_rht_quant_nvfp4(_ptr(x), _dtype_code(x), t, n, block, _ptr(signs),
                                     _ptr(codes), _ptr(block_scales), _ptr(tensor_scale),
                                     _ptr(workspace), ws_bytes, flags, _stream(stream)),
@@ -220,6 +223,47 @@ def kq_rht_quant_nvfp4_dynamic_noalloc(x, block: int, signs, codes, block_scales
     _check(lib().kq_rht_quant_nvfp4_dynamic_noalloc(
         _ptr(x), _dtype_code(x), t, n, block, _ptr(signs), _ptr(codes), _ptr(block_scales),
         _ptr(tensor_scale), _stream(stream)), "kq_rht_quant_nvfp4_dynamic_noalloc")
+
+
+def sharded_dynamic_protocol(run_phase, lower, gmax, all_reduce_max, empty: bool) -> None:
+    """The order of a sharded dynamic NVFP4 call on one rank: phase 1, MAX
+    over the ranks of the lower bound (`lower`, the workspace's bytes 0-3 as
+    int32), phase 2, MAX of the exact maximum (`gmax`, bytes 8-15 as int64),
+    phase 3.  Every rank takes both collectives, a rank with no rows too (it
+    contributes zeros).  run_phase(flag) runs one phase of the library."""
+    if empty:
+        lower.zero_()
+        gmax.zero_()
+    else:
+        run_phase(KQ_DYN_STATS)
+    all_reduce_max(lower)
+    if not empty:
+        run_phase(KQ_DYN_EXACT)
+    all_reduce_max(gmax)
+    if not empty:
+        run_phase(KQ_DYN_QUANT)
+
+
+def nvfp4_dynamic_sharded(x, block: int, signs, codes, block_scales, tensor_scale, workspace,
+                          all_reduce_max, stream=None, mma_layout: bool = False) -> None:
+    """Dynamic NVFP4 of a tensor whose rows are split over ranks: every rank
+    gets the tensor scale of the whole tensor (the single-call result).
+    all_reduce_max(t) reduces a one-element int32 or int64 device tensor in
+    place with MAX over the ranks (torch.distributed.all_reduce with
+    ReduceOp.MAX, say).  See kq_rht_quant_nvfp4 in include/kq.h."""
+    torch = _torch()
+    ws8 = workspace.view(-1)
+
+    def run(flag):
+        kq_rht_quant_nvfp4(x, block, signs, codes, block_scales, tensor_scale, workspace, True,
+                           stream=stream, mma_layout=mma_layout, phases=flag)
+    sharded_dynamic_protocol(run, ws8[0:4].view(torch.int32), ws8[8:16].view(torch.int64),
+                             all_reduce_max, x.shape[0] == 0)
+
+
+def _torch():
+    import torch
+    return torch
 
 
 def kq_gemm_nvfp4(a_codes, a_scales, a_tensor_scale, b_codes, b_scales, b_tensor_scale, c,

@@ -43,6 +43,7 @@ kq_status make_geometry(int dim, int block, kq::Geometry* g) {
   g->sqrt_b = std::sqrt((double)b);
   g->inv_sqrt_b = (float)(1.0 / g->sqrt_b);
   g->sf_kc4 = 0;
+  g->dyn = 0;
   return KQ_OK;
 }
 
@@ -234,9 +235,12 @@ KQ_API kq_status kq_rht_quant_nvfp4(const void* x, int dtype, int64_t tokens, in
   if (st != KQ_OK) return st;
   if (tokens > 0 && (!codes || !block_scales || !tensor_scale)) return KQ_ERR_INVALID_ARG;
   const int mode = flags & (KQ_SCALE_STATIC | KQ_SCALE_DYNAMIC);
-  if ((flags & ~(KQ_SCALE_STATIC | KQ_SCALE_DYNAMIC | KQ_SCALES_MMA)) != 0)
+  constexpr int kPhases = KQ_DYN_STATS | KQ_DYN_EXACT | KQ_DYN_QUANT;
+  if ((flags & ~(KQ_SCALE_STATIC | KQ_SCALE_DYNAMIC | KQ_SCALES_MMA | kPhases)) != 0)
     return KQ_ERR_INVALID_ARG;
   if (mode != KQ_SCALE_STATIC && mode != KQ_SCALE_DYNAMIC) return KQ_ERR_INVALID_ARG;
+  if ((flags & kPhases) && mode != KQ_SCALE_DYNAMIC) return KQ_ERR_INVALID_ARG;
+  g.dyn = (flags & kPhases) / KQ_DYN_STATS;
   if (!aligned(codes, 16) || !aligned(tensor_scale, 4)) return KQ_ERR_MISALIGNED;
   if (flags & KQ_SCALES_MMA) {
     // tensor-core scale-factor layout: whole 4-block atoms per row

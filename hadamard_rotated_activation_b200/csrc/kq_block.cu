@@ -576,13 +576,22 @@ cudaError_t launch_blk128_nvfp4(const void* x, int64_t tokens, const Geometry& g
   P.e_coef = e_coef_128();
   P.sf_kc4 = g.sf_kc4;
   if (ws) {
-    cudaError_t e = cudaMemsetAsync(ws, 0, kNvWorkspaceHeader + (size_t)tokens * sizeof(float2), s);
-    if (e != cudaSuccess) return e;
-    auto k1 = blk::k_blk128_nvfp4<1>;
-    const size_t sm1 = blk_smem(g.n, signs != nullptr);
-    k1<<<blk_grid((const void*)k1, P.units, sm1), blk::kThreads, sm1, s>>>(P);
-    e = launch_nvfp4_global(x, 1, tokens, g, signs, ws, s);
-    if (e != cudaSuccess) return e;
+    const int ph = g.dyn ? g.dyn : 7;
+    if (ph & 1) {
+      cudaError_t e =
+          cudaMemsetAsync(ws, 0, kNvWorkspaceHeader + (size_t)tokens * sizeof(float2), s);
+      if (e != cudaSuccess) return e;
+      auto k1 = blk::k_blk128_nvfp4<1>;
+      const size_t sm1 = blk_smem(g.n, signs != nullptr);
+      k1<<<blk_grid((const void*)k1, P.units, sm1), blk::kThreads, sm1, s>>>(P);
+      e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+    }
+    if (ph & 2) {
+      cudaError_t e = launch_nvfp4_global(x, 1, tokens, g, signs, ws, s);
+      if (e != cudaSuccess) return e;
+    }
+    if (!(ph & 4)) return cudaSuccess;
   }
   auto k0 = blk::k_blk128_nvfp4<0>;
   const size_t sm0 = blk_smem(g.n, signs != nullptr);

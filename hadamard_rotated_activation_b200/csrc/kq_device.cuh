@@ -93,6 +93,8 @@ struct Geometry {
   double sqrt_b;
   int sf_kc4;     // NVFP4 block scales: 0 = row-major [T, n/16]; else the tensor-core
                   // scale-factor layout with sf_kc4 = n/64 atoms per 128-row block
+  int dyn;        // dynamic NVFP4 phases to run (bit 0 statistics, 1 exact maximum,
+                  // 2 quantization); 0 = all three
 };
 
 // Byte offset of the NVFP4 block scale of 16-block c in row `row` (nb blocks a

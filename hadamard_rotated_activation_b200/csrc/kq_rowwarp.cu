@@ -511,12 +511,18 @@ cudaError_t launch_rowwarp_nvfp4(const void* x, int dtype, int64_t tokens, const
   P.sf_kc4 = g.sf_kc4;
   P.gamma = gamma_for(g.n == 4096 ? 12 : 11);
   if (ws) {
-    cudaError_t e = cudaMemsetAsync(ws, 0, kNvWorkspaceHeader, s);
-    if (e != cudaSuccess) return e;
-    e = dispatch<rw::kNvStats>(g.n, P, s);
-    if (e != cudaSuccess) return e;
-    e = launch_nvfp4_global(x, dtype, tokens, g, signs, ws, s);
-    if (e != cudaSuccess) return e;
+    const int ph = g.dyn ? g.dyn : 7;
+    if (ph & 1) {
+      cudaError_t e = cudaMemsetAsync(ws, 0, kNvWorkspaceHeader, s);
+      if (e != cudaSuccess) return e;
+      e = dispatch<rw::kNvStats>(g.n, P, s);
+      if (e != cudaSuccess) return e;
+    }
+    if (ph & 2) {
+      cudaError_t e = launch_nvfp4_global(x, dtype, tokens, g, signs, ws, s);
+      if (e != cudaSuccess) return e;
+    }
+    if (!(ph & 4)) return cudaSuccess;
   }
   return dispatch<rw::kNvfp4>(g.n, P, s);
 }

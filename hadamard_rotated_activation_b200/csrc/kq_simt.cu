@@ -992,25 +992,36 @@ cudaError_t launch_nvfp4(const void* x, int dtype, int64_t tokens, const Geometr
   const size_t smem_glob = (size_t)g.n * 8 + 64 * 8;
   cudaError_t err;
   if (ws) {
-    err = cudaMemsetAsync(ws, 0, sizeof(NvWorkspace), s);
-    if (err != cudaSuccess) return err;
-    if (dtype == 1) {
-      auto k1 = k_nvfp4_rowstats<uint16_t>;
-      k1<<<grid_for((const void*)k1, smem_stats, tokens), kThreads, smem_stats, s>>>(
-          static_cast<const uint16_t*>(x), signs, ws, tokens, g);
-      auto k2 = k_nvfp4_global<uint16_t>;
-      k2<<<grid_for((const void*)k2, smem_glob, tokens), kThreads, smem_glob, s>>>(
-          static_cast<const uint16_t*>(x), signs, ws, tokens, g);
-    } else {
-      auto k1 = k_nvfp4_rowstats<float>;
-      k1<<<grid_for((const void*)k1, smem_stats, tokens), kThreads, smem_stats, s>>>(
-          static_cast<const float*>(x), signs, ws, tokens, g);
-      auto k2 = k_nvfp4_global<float>;
-      k2<<<grid_for((const void*)k2, smem_glob, tokens), kThreads, smem_glob, s>>>(
-          static_cast<const float*>(x), signs, ws, tokens, g);
+    const int ph = g.dyn ? g.dyn : 7;
+    if (ph & 1) {
+      err = cudaMemsetAsync(ws, 0, sizeof(NvWorkspace), s);
+      if (err != cudaSuccess) return err;
+      if (dtype == 1) {
+        auto k1 = k_nvfp4_rowstats<uint16_t>;
+        k1<<<grid_for((const void*)k1, smem_stats, tokens), kThreads, smem_stats, s>>>(
+            static_cast<const uint16_t*>(x), signs, ws, tokens, g);
+      } else {
+        auto k1 = k_nvfp4_rowstats<float>;
+        k1<<<grid_for((const void*)k1, smem_stats, tokens), kThreads, smem_stats, s>>>(
+            static_cast<const float*>(x), signs, ws, tokens, g);
+      }
+      err = cudaGetLastError();
+      if (err != cudaSuccess) return err;
     }
-    err = cudaGetLastError();
-    if (err != cudaSuccess) return err;
+    if (ph & 2) {
+      if (dtype == 1) {
+        auto k2 = k_nvfp4_global<uint16_t>;
+        k2<<<grid_for((const void*)k2, smem_glob, tokens), kThreads, smem_glob, s>>>(
+            static_cast<const uint16_t*>(x), signs, ws, tokens, g);
+      } else {
+        auto k2 = k_nvfp4_global<float>;
+        k2<<<grid_for((const void*)k2, smem_glob, tokens), kThreads, smem_glob, s>>>(
+            static_cast<const float*>(x), signs, ws, tokens, g);
+      }
+      err = cudaGetLastError();
+      if (err != cudaSuccess) return err;
+    }
+    if (!(ph & 4)) return cudaSuccess;
   }
   if (dtype == 1) {
     auto k = k_nvfp4<uint16_t>;

@@ -1020,12 +1020,18 @@ cudaError_t launch_tc_nvfp4(const void* x, int64_t tokens, const Geometry& g,
   P.sf_kc4 = g.sf_kc4;
   cudaError_t e;
   if (ws) {
-    e = cudaMemsetAsync(ws, 0, kNvWorkspaceHeader + (size_t)tokens * sizeof(float2), s);
-    if (e != cudaSuccess) return e;
-    e = launch_tc<tc::kNvStats>(x, signs, P, s);
-    if (e != cudaSuccess) return e;
-    e = launch_nvfp4_global(x, 1, tokens, g, signs, ws, s);
-    if (e != cudaSuccess) return e;
+    const int ph = g.dyn ? g.dyn : 7;
+    if (ph & 1) {
+      e = cudaMemsetAsync(ws, 0, kNvWorkspaceHeader + (size_t)tokens * sizeof(float2), s);
+      if (e != cudaSuccess) return e;
+      e = launch_tc<tc::kNvStats>(x, signs, P, s);
+      if (e != cudaSuccess) return e;
+    }
+    if (ph & 2) {
+      e = launch_nvfp4_global(x, 1, tokens, g, signs, ws, s);
+      if (e != cudaSuccess) return e;
+    }
+    if (!(ph & 4)) return cudaSuccess;
   }
   return launch_tc<tc::kNvfp4>(x, signs, P, s);
 }

@@ -110,7 +110,10 @@ enum {
   KQ_INVERSE = 1,        /* kq_rht: inverse transform x = D H^T y / sqrt(b) */
   KQ_SCALE_STATIC = 2,   /* kq_rht_quant_nvfp4: *tensor_scale is an input */
   KQ_SCALE_DYNAMIC = 4,  /* kq_rht_quant_nvfp4: *tensor_scale is computed and written */
-  KQ_SCALES_MMA = 8      /* kq_rht_quant_nvfp4: block scales in the tensor-core layout */
+  KQ_SCALES_MMA = 8,     /* kq_rht_quant_nvfp4: block scales in the tensor-core layout */
+  KQ_DYN_STATS = 16,     /* KQ_SCALE_DYNAMIC: run the statistics phase (see below) */
+  KQ_DYN_EXACT = 32,     /* KQ_SCALE_DYNAMIC: run the exact-maximum phase */
+  KQ_DYN_QUANT = 64      /* KQ_SCALE_DYNAMIC: run the quantization phase */
 };
 
 /* formats for kq_dequant */
@@ -181,6 +184,22 @@ KQ_API kq_status kq_rht_quant_int4_kv(const void* x, int dtype, int64_t tokens,
  * entry do not matter and are clobbered.  Static mode ignores it.
  * codes: [tokens, dim/2]; block_scales: E4M3 [tokens, dim/16]; tensor_scale:
  * one fp32 in device memory.
+ * Dynamic mode runs three phases on the stream: (1) statistics -- the
+ * workspace is cleared, each row's computed max |S| and error bound are
+ * written, and bytes 0-3 of the workspace receive a lower bound on max |S|
+ * over the rows (an fp32); (2) exact maximum -- rows whose upper bound
+ * reaches that lower bound are transformed exactly and bytes 8-15 receive
+ * max |S| over them (an fp64, unnormalized); (3) quantization with
+ * t = fp32(max|S| / sqrt(b) / 2688), written to *tensor_scale.  Flags
+ * KQ_DYN_STATS, KQ_DYN_EXACT and KQ_DYN_QUANT select a subset (none: all
+ * three).  A tensor split over ranks (QuaRot reviews, final comments: RHT
+ * per batch of data is data parallelism) gets the tensor scale of the whole
+ * tensor by running phase 1 on every rank, an all-reduce(max) of bytes 0-3
+ * of every rank's workspace (as int32: a non-negative fp32 orders like its
+ * bits), phase 2, an all-reduce(max) of bytes 8-15 (as int64), then phase 3:
+ * the rank holding the largest row finds it among its candidates, so every
+ * rank gets the single-tensor result.  A rank with no rows sets both words
+ * to zero itself (tokens == 0 launches nothing).
  * KQ_SCALES_MMA (optional, needs dim % 64 == 0 and 16-byte aligned
  * block_scales) writes the block scales instead in the scale-factor layout of
  * the tcgen05 block-scaled MMA, which kq_gemm_nvfp4 reads: 512-byte atoms of

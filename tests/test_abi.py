@@ -230,3 +230,21 @@ def test_gemm_and_scale_layout_validation(L):
         assert f(P, 1, 4, 4096, 0, None, Q, Q, Q, None, 0, mma, None) == kq.KQ_ERR_CUDA
     finally:
         L.kq_diag_fail_next_launch(0)
+
+
+def test_dynamic_phase_flags_validation(L):
+    f = L.kq_rht_quant_nvfp4
+    ws = L.kq_workspace_size(4, 4096, 0)
+    static = kq.KQ_SCALE_STATIC
+    dyn = kq.KQ_SCALE_DYNAMIC
+    for ph in (kq.KQ_DYN_STATS, kq.KQ_DYN_EXACT, kq.KQ_DYN_QUANT):
+        assert f(P, 1, 4, 4096, 0, None, Q, Q, Q, None, 0, static | ph, None) == \
+            kq.KQ_ERR_INVALID_ARG
+        assert f(P, 1, 0, 4096, 0, None, Q, Q, Q, P, ws, dyn | ph, None) == kq.KQ_OK
+    assert f(P, 1, 4, 4096, 0, None, Q, Q, Q, P, ws, dyn | 128, None) == kq.KQ_ERR_INVALID_ARG
+    try:
+        L.kq_diag_fail_next_launch(_LAUNCH_ERR)
+        assert f(P, 1, 4, 4096, 0, None, Q, Q, Q, P, ws, dyn | kq.KQ_DYN_EXACT, None) == \
+            kq.KQ_ERR_CUDA
+    finally:
+        L.kq_diag_fail_next_launch(0)
