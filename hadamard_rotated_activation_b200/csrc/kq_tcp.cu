@@ -4,39 +4,46 @@
 // quantized to per-token symmetric INT4 (QuaRot reviews, review 2 Summary:
 // RTN INT4 of the rotated activations), or written out rotated (fp32).
 //
-// A row of n = 12288 values is viewed as 96 rows of 128 (index j = a*128 +
-// beta, a = a12*8 + a8).  Since H_1024 = H_8 kron H_128 (Sylvester, natural
-// order), H_12 kron H_1024 = H_96 kron H_128 with H_96 = H_12 kron H_8, and the
-// transform splits into
-//   (1) a mix over a: D[o][beta] = sum_a H_96[o][a] x'[a*128+beta], run on the
-//       tensor cores: D (TMEM, fp32) = A * B with A = H_96 zero-padded to 128 x
-//       128 (bf16 +-1, K-major, built in shared memory once) and B = the
-//       sign-flipped token (K = a, N = beta; MN-major, 128-byte swizzle, two
-//       TMA boxes of 64 columns);
-//   (2) the H_128 over beta, run by the two epilogue threads of TMEM lane o
-//       (o < 96): each reads all 128 columns, does the beta6 stage for its
-//       output half, then six butterfly stages in fp32 on 64 values; it then
-//       holds 64 contiguous outputs o*128 + oh*64 .. +63.
+// Index split.  Sylvester's H_1024 in natural order is H_128 kron H_8, so a
+// row index is j = i12*1024 + c*8 + d (i12 < 12, c < 128, d < 8) and
+//   H[(i12o, co, do)][(i12, c, d)] = H_12[i12o][i12] H_128[co][c] H_8[do][d].
+// The transform runs in three stages:
+//   (1) the mix over c on the tensor cores: D[co][(i12, d)] = sum_c H_128[co][c]
+//       x'[i12*1024 + c*8 + d], D (TMEM, fp32, 128 lanes x 96 columns) = A * B
+//       with A = H_128 (bf16 +-1, K-major, 128-byte swizzle, built in shared
+//       memory once) and B = the sign-flipped token as the bulk copy left it
+//       (K = c, N = i12*8 + d; MN-major without swizzle: a core matrix is the
+//       8 values d of 8 consecutive c, 128 contiguous bytes; the next c octet
+//       is 128 bytes on, the next i12 2048 bytes on);
+//   (2) the H_8 over d, three butterfly stages in registers, by the epilogue
+//       thread that owns TMEM lane co;
+//   (3) the H_12 over i12 in the same thread, Paley construction I (q = 11):
+//       with z_k = x_{1+k}, W_i = sum over r in {0,1,3,4,5,9} of z_{(i+r) mod 11}
+//       (zero and the quadratic residues mod 11) and T = sum of all twelve,
+//       y_0 = T and y_{1+i} = 2 W_i - T; W_i = q_i + q_{i+3} + v_{i+5} with the
+//       pair sums q_k = z_k + z_{k+1}, v_k = z_k + z_{k+4}: 61 operations.
+// The thread then holds outputs i12o*1024 + co*8 + do: twelve runs of eight
+// contiguous values, one 32-bit word of nibbles each.
 //
 // Exact scale.  The per-token scale fp32(max|y| / 7), y = S / sqrt(n), needs
 // max|S| exactly.  With the accumulation model of tcgen05.mma (see the
-// 4096-wide kernel: step k adds at most 2.5 u P_k plus the truncation of
-// inputs far below the step's largest term, at most 8 u P_k more; P_k =
-// partial column sum of |x|) the six steps err by at most 63 u C_beta per
-// column (C_beta = sum_a |x'[a][beta]|), and the seven fp32 stages by 7.01 u
-// sum|x| more, so |S_hat_i - S_i| <= 70.1 u sum|x| <= 70.1 u ||S||_2 (Cauchy-
-// Schwarz and ||S||_2 = sqrt(n) ||x||_2) <= E = 72 u ||S_hat||_2.  Every
-// output within 2E of the largest |S_hat| is recomputed exactly in fp64 by
-// the whole epilogue group from the staged token, which the epilogue holds
-// until then.
+// 4096-wide kernel: a K = 16 step adds at most 2.5 u P_k plus the truncation
+// of inputs far below the step's largest term, at most 8 u P_k more; P_k =
+// partial column sum of |x|) the eight steps err by at most 84 u C_n per
+// column n (C_n = its sum of |x'|); the H_8 stages add at most 3 u and the
+// H_12 formulas (at most seven roundings on a path, and the doubling) 16 u
+// of the sum of |x| over their cone, so |S_hat_i - S_i| <= 103 u sum|x| <=
+// 103 u ||S||_2 (Cauchy-Schwarz, ||S||_2 = sqrt(n) ||x||_2) <= E = 108 u
+// ||S_hat||_2.  Every output within 2E of the largest |S_hat| is recomputed
+// exactly in fp64 by the epilogue group from the staged token, which the
+// epilogue holds until then.
 //
-// Warp roles (20 warps): 0 TMA producer, 1 MMA issuer + TMEM owner, 2-3 sign
-// flip, 4-11 and 12-19 two epilogue groups taking alternate tokens.  In a
-// group, warp w reads TMEM lane quarter w % 4 (quarter 3 holds the zero
-// padding of A and only helps with reductions and fix-ups), and the two warps
-// of a quarter split the row's outputs into halves (beta6 = 0, 1), so a thread
-// holds 64 values.  Every wait is bounded; on timeout the kernel
-// records an error code and returns.
+// Warp roles (12 warps): 0 producer (one bulk copy per token), 1 MMA issuer +
+// TMEM owner, 2-3 sign flip, 4-7 and 8-11 two epilogue groups taking
+// alternate tokens; warp w reads TMEM lane quarter w % 4, so every group has
+// one warp on each scheduler.  A thread keeps its 96 values in registers, so
+// the accumulator is handed back to the MMA as soon as it is read.  Every wait
+// is bounded; on timeout the kernel records an error code and returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -54,47 +61,52 @@ namespace tcp {
 using namespace sm100;
 
 constexpr int N = 12288;
-constexpr int kRows = 96;                          // a
-constexpr int kCols = 128;                         // beta
-constexpr uint32_t kHalfBytes = kRows * 128;       // 96 rows x 64 columns (bf16)
-constexpr uint32_t kStageBytes = 2 * kHalfBytes;   // one token, 24 KB
-constexpr int kStages = 5;
-constexpr int kAcc = 4;                            // TMEM accumulators (128 columns each)
-constexpr int kTmemCols = kAcc * kCols;
-// 20 warps: 0 TMA, 1 MMA; epilogue group g owns warps 4 + 8g .. 11 + 8g
-// except those in lane quarter 3 (A's zero padding), which flip signs with
-// warps 2 and 3.
-constexpr int kSignWarps = 6;
-constexpr int kGroupWarps = 6;                     // per epilogue group: 3 lane quarters x 2 halves
-constexpr int kGroupThreads = 32 * kGroupWarps;
-constexpr int kThreads = 32 * 20;
-__device__ __forceinline__ bool is_sign_warp(int w) { return w == 2 || w == 3 || (w >= 4 && (w & 3) == 3); }
-__device__ __forceinline__ int sign_index(int w) { return w < 4 ? w - 2 : 2 + (w - 7) / 4; }
+constexpr int kCols = 96;                          // accumulator columns: i12 * 8 + d
+constexpr uint32_t kStageBytes = N * 2;            // one token, natural order
+constexpr int kStages = 7;
+constexpr int kAcc = 4;                            // TMEM accumulators (128 columns apart)
+constexpr int kTmemCols = 512;
+constexpr int kGroups = 2;
+constexpr int kSignWarps = 2;
+constexpr int kGroupThreads = 128;                 // one warp per TMEM lane quarter
+constexpr int kThreads = 32 * (2 + kSignWarps + 4 * kGroups);
 constexpr int kChunks = N / 8;                     // 16-byte chunks per token
+constexpr int kSignLanes = 32 * kSignWarps;
+constexpr int kSignPer = kChunks / kSignLanes;     // chunks per sign lane
 constexpr int kMaxCand = 32;                       // fix-up candidates handled per token
-constexpr double kBoundC = 72.0 * 0x1p-24;         // E = kBoundC ||S_hat||_2
-static_assert(kChunks % (32 * kSignWarps) == 0 && (kChunks / 2) % (32 * kSignWarps) == 0,
-              "sign warps split the chunks (and each half) evenly");
-static_assert(kChunks % kGroupThreads == 0, "an epilogue group splits the chunks evenly");
+constexpr double kBoundC = 108.0 * 0x1p-24;        // E = kBoundC ||S_hat||_2
+static_assert(kChunks % kSignLanes == 0, "sign lanes split the chunks evenly");
+static_assert(kAcc % kGroups == 0, "each group owns whole accumulators");
 
 __device__ unsigned int g_tcp_error = 0;           // nonzero: a wait timed out
 
 enum { kInt4 = 0, kRot = 1 };
 
 struct Params {
+  const uint16_t* x;     // bf16 [T, n]
   uint8_t* codes;        // kInt4: [T, n/2]
   float* scales;         // kInt4: [T]
   float* out;            // kRot: fp32 [T, n]
   int64_t tokens;
   double sqrt_n;         // IEEE sqrt(12288)
+  double rcp_sqrt_n;     // fp64 1 / sqrt_n, correctly rounded
 };
+
+// a / b correctly rounded for finite a, from rb = RN(1 / b): q0 = RN(a rb) is
+// within an ulp, its residual a - q0 b is exact under an FMA, and one
+// correction step gives the rounded quotient (Markstein's theorem for fused
+// multiply-add); a short dependent chain instead of a division routine.
+__device__ __forceinline__ double div_rn(double a, double b, double rb) {
+  const double q0 = a * rb;
+  return fma(fma(-q0, b, a), rb, q0);
+}
 
 // Per-group scratch for the token reductions.
 struct GroupScratch {
-  float wmax[kGroupWarps];
-  float wsq[kGroupWarps];
-  double part[2][kGroupWarps];   // per candidate parity
-  int wcnt[kGroupWarps];
+  float wmax[4];
+  float wsq[4];
+  double part[2][4];     // per candidate parity
+  int wcnt[4];
   int ncand;
   int cand[kMaxCand];
 };
@@ -105,65 +117,83 @@ __device__ __forceinline__ bool wait(uint64_t* bar, uint32_t parity) {
 __device__ __forceinline__ void group_sync(int g) {
   asm volatile("bar.sync %0, %1;" :: "r"(1 + g), "n"(kGroupThreads) : "memory");
 }
-
-// H_96[m][k] = H_12[m/8][k/8] (-1)^popc((m%8) & (k%8)), negative?
-__device__ __forceinline__ bool h96_negative(int m, int k) {
-  return paley_negative(m >> 3, k >> 3) ^ (__popc((m & 7) & (k & 7)) & 1);
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               :: "r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
 }
 
-// Byte offset of 16-byte chunk c16 (0..15) of row a of a staged token: two
-// halves of 96 rows x 128 bytes (columns 64h .. 64h+63), 128-byte swizzle
-// (chunk c of row a at chunk position c ^ (a & 7)).
-__device__ __forceinline__ uint32_t b_chunk(int a, int c16) {
-  return (uint32_t)((c16 >> 3) * kHalfBytes + a * 128 + (((c16 & 7) ^ (a & 7)) << 4));
+// x 2^-896 as a double for the bf16 x in the top half of w: sign, exponent and
+// mantissa move into the double's high word as they are (an arithmetic shift
+// by 3 and a mask), so zero and subnormals map exactly too; integer pipes only.
+__device__ __forceinline__ double bf16_hi_scaled(uint32_t w) {
+  return __hiloint2double((int)((uint32_t)((int32_t)w >> 3) & 0x8FFFE000u), 0);
 }
+constexpr double kUnscale = 0x1p896;
 
-// Exact S_i (fp64) of a staged, sign-flipped token, computed by the
-// kGroupThreads threads of an epilogue group: thread tau takes the 16-byte
-// chunks tau, tau + kGroupThreads, ...; chunk ch holds x'[a*128 + c16*8 .. +7] (a = ch / 16, c16 =
-// ch % 16).  H[i][j] for i = o*128 + b, j = a*128 + c16*8 + e is H_96[o][a]
-// (-1)^(popc(b_hi & c16) + popc(b_lo & e)), b_hi = b / 8, b_lo = b % 8.
-// Values enter fp64 exactly (bf16 -> fp32 -> fp64 conversions).  Returns
+// Exact S_i (fp64) of a staged, sign-flipped token, i = (i12o, co, do),
+// computed by the kGroupThreads threads of an epilogue group: thread tau sums
+// the 96 terms with c = tau, held in the chunks k = i12 (k = 0..11) at byte
+// k*2048 + tau*16 of the stage (x'[k*1024 + tau*8 + d], d = 0..7).  The sign
+// of a term is H_12[i12o][k] H_128[co][tau] H_8[do][d]; bit k of row12 is
+// H_12[i12o][k] < 0.  Values enter fp64 exactly, scaled by 2^-896
+// (bf16_hi_scaled), and the partial sum is scaled back at the end.  Returns
 // this thread's partial sum.
-__device__ __forceinline__ double exact_partial(const uint8_t* tok, int i, int tau) {
-  const int o = i >> 7, bhi = (i >> 3) & 15, blo = i & 7;
+__device__ __forceinline__ double exact_partial(const uint8_t* tok, int i, uint32_t row12,
+                                                int tau) {
+  const int co = (i >> 3) & 127, dd = i & 7;
+  // row dd of H_8 as bits: bit d = popc(dd & d) & 1
+  const uint32_t h8 = (uint32_t)(0x963C5AF066CCAA00ull >> (8 * dd));
   uint32_t em[4];
 #pragma unroll
   for (int w = 0; w < 4; ++w)
-    em[w] = ((uint32_t)(__popc(blo & (2 * w)) & 1) << 15) |
-            ((uint32_t)(__popc(blo & (2 * w + 1)) & 1) << 31);
-  const uint32_t fc = (__popc(bhi & (tau & 15)) & 1) ? 0x80008000u : 0u;   // c16 = tau % 16
+    em[w] = (((h8 >> (2 * w)) & 1u) << 15) | (((h8 >> (2 * w + 1)) & 1u) << 31);
+  const uint32_t fc = (__popc(co & tau) & 1) ? 0x80008000u : 0u;
+  const uint8_t* p = tok + tau * 16;
   double acc[4] = {0.0, 0.0, 0.0, 0.0};
 #pragma unroll
-  for (int k = 0; k < kChunks / kGroupThreads; ++k) {
-    const int ch = tau + kGroupThreads * k;
-    const int a = ch >> 4, c16 = ch & 15;
-    const uint32_t flip = (h96_negative(o, a) ? 0x80008000u : 0u) ^ fc;
-    const uint4 v = *reinterpret_cast<const uint4*>(tok + b_chunk(a, c16));
+  for (int k = 0; k < 12; ++k) {
+    const uint4 v = *reinterpret_cast<const uint4*>(p + k * 2048);
+    const uint32_t flip = fc ^ ((0u - ((row12 >> k) & 1u)) & 0x80008000u);
     const uint32_t ww[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
       const uint32_t x2 = ww[w] ^ em[w] ^ flip;   // the two terms' signed bf16 bits
-      acc[w] += (double)__uint_as_float(x2 << 16);           // exact: bf16 -> fp32 -> fp64
-      acc[(w + 2) & 3] += (double)__uint_as_float(x2 & 0xffff0000u);
+      acc[w] += bf16_hi_scaled(x2 << 16);
+      acc[(w + 2) & 3] += bf16_hi_scaled(x2);
     }
   }
-  return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+  return ((acc[0] + acc[1]) + (acc[2] + acc[3])) * kUnscale;
 }
 
-// Six butterfly stages (H_64, natural order) on f[0..31] (f[p] holds
-// elements 2p, 2p + 1) in place.
-__device__ __forceinline__ void h64(float2 (&f)[32]) {
+// H_8 over d on f[0..3] (f[e] holds d = 2e, 2e + 1), natural order.
+__device__ __forceinline__ void h8(float2* f) {
 #pragma unroll
-  for (int p = 0; p < 32; ++p) {
-    const float a = f[p].x, b = f[p].y;
-    f[p] = make_float2(a + b, a - b);
+  for (int e = 0; e < 4; ++e) {
+    const float a = f[e].x, b = f[e].y;
+    f[e] = make_float2(a + b, a - b);
   }
+  bfly2(f[0], f[1]);
+  bfly2(f[2], f[3]);
+  bfly2(f[0], f[2]);
+  bfly2(f[1], f[3]);
+}
+
+// H_12 (Paley I, q = 11) over i12 on the twelve vectors f[0], f[4], ..., f[44]
+// (two independent transforms, one per f32x2 half), in place.
+__device__ __forceinline__ void h12(float2* f) {
+  float2 q[11], v[11];
 #pragma unroll
-  for (int hh = 1; hh < 32; hh <<= 1)
+  for (int k = 0; k < 11; ++k) {
+    q[k] = add2(f[4 * (1 + k)], f[4 * (1 + (k + 1) % 11)]);
+    v[k] = add2(f[4 * (1 + k)], f[4 * (1 + (k + 4) % 11)]);
+  }
+  const float2 t = add2(f[0], add2(add2(add2(add2(add2(q[0], q[2]), q[4]), q[6]), q[8]), f[44]));
+  const float2 two = make_float2(2.0f, 2.0f), negt = make_float2(-t.x, -t.y);
 #pragma unroll
-    for (int p = 0; p < 32; ++p)
-      if (!(p & hh)) bfly2(f[p], f[p | hh]);
+  for (int i = 0; i < 11; ++i)
+    f[4 * (1 + i)] = fma2(two, add2(add2(q[i], q[(i + 3) % 11]), v[(i + 5) % 11]), negt);
+  f[0] = t;
 }
 
 // Two's-complement INT4 nibble in the low 4 bits of the fp32 value
@@ -186,16 +216,16 @@ __device__ __forceinline__ uint32_t int4x8(const float2* f, float2 c2) {
 
 template <int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
-k_tc12288(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ signs, Params P) {
+k_tc12288(const int8_t* __restrict__ signs, Params P) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* sA = smem;                                    // 32 KB: A = H_96, zero-padded
+  uint8_t* sA = smem;                                    // 32 KB: A = H_128
   uint8_t* sB = smem + 32768;                            // kStages x 24 KB
-  uint4* smask = reinterpret_cast<uint4*>(sB + kStages * kStageBytes);   // kChunks
-  GroupScratch* gs = reinterpret_cast<GroupScratch*>(smask + kChunks);   // 2 groups x 2
-  uint64_t* bars = reinterpret_cast<uint64_t*>(gs + 4);
-  uint64_t* full = bars;                                 // TMA landed
+  GroupScratch* gs = reinterpret_cast<GroupScratch*>(sB + kStages * kStageBytes);   // 2 x 2
+  uint32_t* prow = reinterpret_cast<uint32_t*>(gs + 2 * kGroups);   // 12 rows of H_12 as bits
+  uint64_t* bars = reinterpret_cast<uint64_t*>(prow + 16);
+  uint64_t* full = bars;                                 // bulk copy landed
   uint64_t* ready = bars + kStages;                      // signs applied
   uint64_t* empty = bars + 2 * kStages;                  // MMAs and fix-ups done with the stage
   uint64_t* tfull = bars + 3 * kStages;                  // accumulator written (kAcc)
@@ -212,7 +242,7 @@ k_tc12288(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ s
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&ready[s], 32 * kSignWarps);
+      mbar_init(&ready[s], kSignLanes);
       mbar_init(&empty[s], kMode == kInt4 ? 2 : 1);   // MMA commit [+ epilogue]
     }
     for (int d = 0; d < kAcc; ++d) {
@@ -224,35 +254,25 @@ k_tc12288(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ s
     for (int64_t k = 0; k < prefilled; ++k) {
       const int64_t token = blockIdx.x + k * gridDim.x;
       mbar_expect_tx(&full[k], kStageBytes);
-      tma_load_2d(sB + k * kStageBytes, &tmap, 0, (int)(token * kRows), &full[k]);
-      tma_load_2d(sB + k * kStageBytes + kHalfBytes, &tmap, 64, (int)(token * kRows), &full[k]);
+      bulk_load(sB + k * kStageBytes, P.x + token * N, kStageBytes, &full[k]);
     }
   }
-  // A = H_96 zero-padded, one 16-byte chunk (8 columns) per step
+  // A = H_128, one 16-byte chunk (8 columns) per step
   for (int idx = threadIdx.x; idx < 128 * 16; idx += blockDim.x) {
     const int m = idx >> 4, k0 = (idx & 15) * 8;
     uint32_t w[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      uint32_t lo = 0, hi = 0;                        // zero padding
-      if (m < kRows && k0 + 2 * e < kRows) {
-        lo = h96_negative(m, k0 + 2 * e) ? 0xBF80u : 0x3F80u;       // -1 / +1
-        hi = h96_negative(m, k0 + 2 * e + 1) ? 0xBF80u : 0x3F80u;
-      }
+      const uint32_t lo = (__popc(m & (k0 + 2 * e)) & 1) ? 0xBF80u : 0x3F80u;   // -1 / +1
+      const uint32_t hi = (__popc(m & (k0 + 2 * e + 1)) & 1) ? 0xBF80u : 0x3F80u;
       w[e] = lo | (hi << 16);
     }
     *reinterpret_cast<uint4*>(sA + a_off(m, k0)) = make_uint4(w[0], w[1], w[2], w[3]);
   }
-  for (int i = threadIdx.x; i < kChunks; i += blockDim.x) {
-    uint4 m4 = make_uint4(0, 0, 0, 0);
-    if (signs) {
-      const uint2 sv = __ldg(reinterpret_cast<const uint2*>(signs) + i);
-      m4 = make_uint4(__byte_perm(sv.x, 0, 0x1404) & 0x80008000u,
-                      __byte_perm(sv.x, 0, 0x3424) & 0x80008000u,
-                      __byte_perm(sv.y, 0, 0x1404) & 0x80008000u,
-                      __byte_perm(sv.y, 0, 0x3424) & 0x80008000u);
-    }
-    smask[i] = m4;
+  if (threadIdx.x < 12) {
+    uint32_t bits = 0;
+    for (int c = 0; c < 12; ++c) bits |= (uint32_t)paley_negative(threadIdx.x, c) << c;
+    prow[threadIdx.x] = bits;
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
@@ -265,9 +285,8 @@ k_tc12288(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ s
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-
   if (warp == 0) {
-    // ================= TMA producer: two 96-row boxes per token
+    // ================= producer: one 24 KB bulk copy per token
     if (lane == 0) {
       int64_t issued = prefilled;
       for (int64_t k = prefilled; k < my_tiles; ++k) {
@@ -275,9 +294,7 @@ k_tc12288(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ s
         if (k >= kStages && !wait(&empty[s], (uint32_t)(k / kStages - 1) & 1)) break;
         const int64_t token = blockIdx.x + k * gridDim.x;
         mbar_expect_tx(&full[s], kStageBytes);
-        tma_load_2d(sB + s * kStageBytes, &tmap, 0, (int)(token * kRows), &full[s]);
-        tma_load_2d(sB + s * kStageBytes + kHalfBytes, &tmap, 64, (int)(token * kRows),
-                    &full[s]);
+        bulk_load(sB + s * kStageBytes, P.x + token * N, kStageBytes, &full[s]);
         issued = k + 1;
       }
       // no copy may still be in flight when the CTA exits
@@ -296,14 +313,14 @@ k_tc12288(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ s
         if (k >= kAcc && !wait(&tempty[d], (uint32_t)(k / kAcc - 1) & 1)) break;
         tc_fence_after();
         const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB + s * kStageBytes);
-        const uint32_t tmem_d = tmem_base + (uint32_t)(d * kCols);
+        const uint32_t tmem_d = tmem_base + (uint32_t)(d * 128);
 #pragma unroll
-        for (int ks = 0; ks < kRows / 16; ++ks) {
+        for (int ks = 0; ks < 8; ++ks) {
           // A: K-major, K step of 16 = 32 bytes inside a 128-byte swizzle row
           const uint64_t adesc = smem_desc(a0 + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, 2);
-          // B: MN-major 128-byte swizzle atoms of 64 columns (the two halves,
-          // kHalfBytes apart), 8-row groups 1 KB apart; K step of 16 rows = 2 KB
-          const uint64_t bdesc = smem_desc(b0 + ks * 2048, kHalfBytes, 1024, 2);
+          // B: MN-major, no swizzle: c octets 128 bytes apart (leading), i12
+          // blocks 2048 bytes apart (stride); a K step of 16 is two c octets
+          const uint64_t bdesc = smem_desc(b0 + ks * 256, 128, 2048, 0);
           mma_bf16(tmem_d, adesc, bdesc, idesc, ks > 0 ? 1u : 0u);
         }
         mma_commit(&empty[s]);
@@ -313,21 +330,21 @@ k_tc12288(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ s
       for (int64_t k = issued > kAcc ? issued - kAcc : 0; k < issued; ++k)
         wait(&tfull[k % kAcc], (uint32_t)(k / kAcc) & 1);
     }
-  } else if (is_sign_warp(warp)) {
-    // ================= sign flip: lane t0 of the sign warps takes the physical
-    // chunks t0 + 192 i (conflict-free), i = 0..7: half i / 4, row a = t0 / 8 +
-    // 24 (i % 4), slot t0 % 8, which holds logical chunk (t0 % 8) ^ (a % 8) of
-    // the half.  The lane's 8 sign masks stay in registers.
-    constexpr int kLanes = 32 * kSignWarps;
-    constexpr int kPer = kChunks / kLanes;
-    const int t0 = sign_index(warp) * 32 + lane;
-    uint4 msk[kPer];
-    {
-      const int cl = (t0 & 7) ^ ((t0 >> 3) & 7);
+  } else if (warp < 2 + kSignWarps) {
+    // ================= sign flip: lane t0 takes the chunks t0 + 64 i
+    // (consecutive lanes, consecutive 16-byte chunks); its masks stay in
+    // registers.
+    const int t0 = (warp - 2) * 32 + lane;
+    uint4 msk[kSignPer];
 #pragma unroll
-      for (int i = 0; i < kPer; ++i) {
-        const int a = (t0 >> 3) + (kLanes / 8) * (i % (kPer / 2));
-        msk[i] = smask[a * 16 + (i / (kPer / 2)) * 8 + cl];
+    for (int i = 0; i < kSignPer; ++i) {
+      msk[i] = make_uint4(0, 0, 0, 0);
+      if (signs) {
+        const uint2 sv = __ldg(reinterpret_cast<const uint2*>(signs) + t0 + kSignLanes * i);
+        msk[i] = make_uint4(__byte_perm(sv.x, 0, 0x1404) & 0x80008000u,
+                            __byte_perm(sv.x, 0, 0x3424) & 0x80008000u,
+                            __byte_perm(sv.y, 0, 0x1404) & 0x80008000u,
+                            __byte_perm(sv.y, 0, 0x3424) & 0x80008000u);
       }
     }
     for (int64_t k = 0; k < my_tiles; ++k) {
@@ -336,13 +353,13 @@ k_tc12288(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ s
       if (signs) {
         uint4* st = reinterpret_cast<uint4*>(sB + s * kStageBytes) + t0;
 #pragma unroll
-        for (int i = 0; i < kPer; ++i) {
-          uint4 w = st[kLanes * i];
+        for (int i = 0; i < kSignPer; ++i) {
+          uint4 w = st[kSignLanes * i];
           w.x ^= msk[i].x;
           w.y ^= msk[i].y;
           w.z ^= msk[i].z;
           w.w ^= msk[i].w;
-          st[kLanes * i] = w;
+          st[kSignLanes * i] = w;
         }
         fence_async_smem();
       }
@@ -350,120 +367,116 @@ k_tc12288(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ s
       mbar_arrive(&ready[s]);
     }
   } else {
-    // ================= epilogue: group g of warps 4+8g .. 11+8g.  Warp w
-    // reads TMEM lane quarter q = w % 4 (rows o = 32 q + lane); the first four
-    // warps of a group take output half oh = 0, the other four oh = 1.  The
-    // accumulator row o holds D0 (columns 0-63, beta6 = 0) and D1 (64-127);
-    // the beta6 stage gives S[o][oh][.] = D0 + D1 (oh = 0) or D0 - D1, then
-    // H_64 over the 64 low columns: outputs o*128 + oh*64 .. +63.
-    const int g = (warp - 4) >> 3;
-    const int q = warp & 3;                   // TMEM lane quarter (0..2)
-    const int oh = (warp >> 2) & 1 ? 0 : 1;   // output half (beta6 of the output)
-    const int o = q * 32 + lane;              // accumulator row
-    const int wg = oh * 3 + q;                // warp within the group
-    const int tau = wg * 32 + lane;           // thread within the group
-    const bool rowv = true;
-    for (int64_t k = g; k < my_tiles; k += 2) {
-      const int d = (int)(k % kAcc);
-      const int st = (int)(k % kStages);
-      const int64_t token = blockIdx.x + k * gridDim.x;
+    // ================= epilogue: group g of warps 4 + 4g .. 7 + 4g; warp w
+    // reads TMEM lane quarter q = w % 4, lane co = 32 q + lane.
+    const int g = (warp - 4) >> 2;
+    const int q = warp & 3;
+    const int co = q * 32 + lane;             // also the thread's index in the group
+    const int ntiles = (int)my_tiles;         // tokens < 2^31
+    for (int k = g; k < ntiles; k += kGroups) {
+      const int d = k % kAcc;
+      const int st = k % kStages;
+      const int64_t token = blockIdx.x + (int64_t)k * gridDim.x;
       // scratch alternates between the group's consecutive tokens, so a token
       // never overwrites one that a slower warp may still be reading
-      GroupScratch& S = gs[2 * g + ((k >> 1) & 1)];
+      GroupScratch& S = gs[2 * g + ((k / kGroups) & 1)];
       // A timed-out wait does not leave the loop: the failure is recorded and
       // the token's outputs are not written.
       const bool ok = wait(&tfull[d], (uint32_t)(k / kAcc) & 1);
       tc_fence_after();
-      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(d * kCols);
-      float2 f[32];
-      if (rowv) {
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(d * 128);
+      float2 f[48];                           // f[4 i12 + e] holds d = 2e, 2e + 1
+      {
+        uint32_t r[3][32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r0[16], r1[16];
-          tmem_ld16(taddr + c * 16, r0);
-          tmem_ld16(taddr + 64 + c * 16, r1);
-          tmem_wait_ld();
+        for (int c = 0; c < 3; ++c) tmem_ld32(taddr + c * 32, r[c]);
+        tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float a0 = __uint_as_float(r0[2 * e]), a1 = __uint_as_float(r0[2 * e + 1]);
-            const float b0 = __uint_as_float(r1[2 * e]), b1 = __uint_as_float(r1[2 * e + 1]);
-            f[8 * c + e] = oh ? make_float2(a0 - b0, a1 - b1) : make_float2(a0 + b0, a1 + b1);
-          }
-        }
-      } else {
-#pragma unroll
-        for (int p = 0; p < 32; ++p) f[p] = make_float2(0.0f, 0.0f);
-      }
-      h64(f);
-
-      if (kMode == kRot) {
-        tc_fence_before();
-        mbar_arrive(&tempty[d]);
-        if (ok && rowv) {
-          const float inv = (float)(1.0 / P.sqrt_n);
-          float4* dst = reinterpret_cast<float4*>(P.out + token * N + o * 128 + oh * 64);
+        for (int c = 0; c < 3; ++c)
 #pragma unroll
           for (int p = 0; p < 16; ++p)
-            dst[p] = make_float4(f[2 * p].x * inv, f[2 * p].y * inv, f[2 * p + 1].x * inv,
-                                 f[2 * p + 1].y * inv);
+            f[16 * c + p] =
+                make_float2(__uint_as_float(r[c][2 * p]), __uint_as_float(r[c][2 * p + 1]));
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[d]);                // the values live in registers from here on
+#pragma unroll
+      for (int i12 = 0; i12 < 12; ++i12) h8(f + 4 * i12);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) h12(f + e);
+
+      if (kMode == kRot) {
+        if (ok) {
+          const float inv = (float)(1.0 / P.sqrt_n);
+          float* dst = P.out + token * N + co * 8;
+#pragma unroll
+          for (int i12 = 0; i12 < 12; ++i12) {
+            const float2* h = f + 4 * i12;
+            reinterpret_cast<float4*>(dst + i12 * 1024)[0] =
+                make_float4(h[0].x * inv, h[0].y * inv, h[1].x * inv, h[1].y * inv);
+            reinterpret_cast<float4*>(dst + i12 * 1024)[1] =
+                make_float4(h[2].x * inv, h[2].y * inv, h[3].x * inv, h[3].y * inv);
+          }
         }
         continue;
       }
 
       // ---- token maximum and ||S_hat||_2^2 over the group
-      float mx = 0.0f, sq = 0.0f;
+      // four independent chains each
+      float mj[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      float2 sj[4] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f),
+                      make_float2(0.0f, 0.0f)};
 #pragma unroll
-      for (int p = 0; p < 32; ++p) {
-        mx = fmax3(mx, fabsf(f[p].x), fabsf(f[p].y));
-        sq = fmaf(f[p].x, f[p].x, fmaf(f[p].y, f[p].y, sq));
+      for (int p = 0; p < 48; ++p) {
+        mj[p & 3] = fmax3(mj[p & 3], fabsf(f[p].x), fabsf(f[p].y));
+        sj[p & 3] = fma2(f[p], f[p], sj[p & 3]);
       }
+      float mx = fmaxf(fmaxf(mj[0], mj[1]), fmaxf(mj[2], mj[3]));
+      const float2 sq2 = add2(add2(sj[0], sj[1]), add2(sj[2], sj[3]));
+      float sq = sq2.x + sq2.y;
       const float own_mx = mx;
-      mx = warp_max(mx);
+      mx = __uint_as_float(redux_max(__float_as_uint(mx)));   // non-negative: integer order
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
       if (lane == 0) {
-        S.wmax[wg] = mx;
-        S.wsq[wg] = sq;
+        S.wmax[q] = mx;
+        S.wsq[q] = sq;
       }
-      if (tau == 0) S.ncand = 0;
-      group_sync(g);                           // also: every thread has read D0 and D1
+      if (co == 0) S.ncand = 0;
+      group_sync(g);
       float M = 0.0f, Q = 0.0f;
 #pragma unroll
-      for (int w = 0; w < kGroupWarps; ++w) {
+      for (int w = 0; w < 4; ++w) {
         M = fmaxf(M, S.wmax[w]);
         Q += S.wsq[w];
       }
       const bool finite = isfinite(M) && isfinite(Q);
-      // E rounded up (fp32 sums of 12288 squares err by far less than 2^-10)
-      const float E = __fmul_ru((float)kBoundC, __fsqrt_ru(__fmul_ru(Q, 1.0f + 0x1p-10f)));
+      // E rounded up (fp32 sums of 12288 squares err by far less than 2^-10; a
+      // correctly rounded square root is within 2^-24 of the true one)
+      const float E = __fmul_ru(__fmul_ru((float)kBoundC, 1.0f + 0x1p-22f),
+                                sqrtf(__fmul_ru(Q, 1.0f + 0x1p-10f)));
       const float thr = __fsub_rd(M, __fmul_ru(2.0f, E));
       // ---- candidates: every output within 2E of the maximum
-      uint32_t cm[2] = {0u, 0u};
-      if (rowv && finite && M > 0.0f && own_mx >= thr) {
+      uint32_t cm[3] = {0u, 0u, 0u};
+      if (finite && M > 0.0f && own_mx >= thr) {
 #pragma unroll
-        for (int p = 0; p < 32; ++p) {
+        for (int p = 0; p < 48; ++p) {
           if (fabsf(f[p].x) >= thr) cm[p >> 4] |= 1u << (2 * (p & 15));
           if (fabsf(f[p].y) >= thr) cm[p >> 4] |= 1u << (2 * (p & 15) + 1);
         }
       }
-      // park S_hat in this thread's half of the accumulator row while the
-      // registers serve the fix-ups (both halves were read before the sync)
-      if (rowv) {
-#pragma unroll
-        for (int c = 0; c < 2; ++c)
-          tmem_st32(taddr + oh * 64 + c * 32, *reinterpret_cast<const uint32_t(*)[32]>(
-                                                  reinterpret_cast<const uint32_t*>(f) + 32 * c));
-      }
-      const int myc = __popc(cm[0]) + __popc(cm[1]);
+      // value 2p + h of this thread is output (p / 4) * 1024 + co * 8 + (p % 4) * 2 + h
+      const int myc = __popc(cm[0]) + __popc(cm[1]) + __popc(cm[2]);
       if (myc > 0) {
         int slot = atomicAdd(&S.ncand, myc);
 #pragma unroll
-        for (int w = 0; w < 2; ++w) {
+        for (int w = 0; w < 3; ++w) {
           uint32_t bits = cm[w];
           while (bits) {
             const int b = __ffs(bits) - 1;
             bits &= bits - 1;
-            if (slot < kMaxCand) S.cand[slot] = o * 128 + oh * 64 + w * 32 + b;
+            const int v = 32 * w + b, p = v >> 1;
+            if (slot < kMaxCand) S.cand[slot] = (p >> 2) * 1024 + co * 8 + (p & 3) * 2 + (v & 1);
             ++slot;
           }
         }
@@ -474,15 +487,15 @@ k_tc12288(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ s
       // ---- exact maximum over the candidates
       double best = 0.0;
       const uint8_t* tok = sB + st * kStageBytes;   // held until the fix-ups are done
+      auto exact_at = [&](int ci) { return exact_partial(tok, ci, prow[ci >> 10], co); };
       if (total > 0) wait(&ready[st], (uint32_t)(k / kStages) & 1);   // sign flips visible
       if (total <= kMaxCand) {
         for (int c = 0; c < total; ++c) {
-          double part = warp_sum_d(exact_partial(tok, S.cand[c], tau));
-          if (lane == 0) S.part[c & 1][wg] = part;
+          double part = warp_sum_d(exact_at(S.cand[c]));
+          if (lane == 0) S.part[c & 1][q] = part;
           group_sync(g);
-          double sum = 0.0;
-#pragma unroll
-          for (int w = 0; w < kGroupWarps; ++w) sum += S.part[c & 1][w];
+          const double sum = (S.part[c & 1][0] + S.part[c & 1][1]) +
+                             (S.part[c & 1][2] + S.part[c & 1][3]);
           best = fmax(best, fabs(sum));
         }
       } else {
@@ -493,24 +506,25 @@ k_tc12288(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ s
           const int v = __shfl_up_sync(0xffffffffu, incl, off);
           if (lane >= off) incl += v;
         }
-        if (lane == 31) S.wcnt[wg] = incl;
+        if (lane == 31) S.wcnt[q] = incl;
         group_sync(g);
         int base = 0;
 #pragma unroll
-        for (int w = 0; w < kGroupWarps; ++w) base += (w < wg) ? S.wcnt[w] : 0;
+        for (int w = 0; w < 4; ++w) base += (w < q) ? S.wcnt[w] : 0;
         const int rank0 = base + incl - myc;
         for (int r0 = 0; r0 < total; r0 += kMaxCand) {
           group_sync(g);                        // the previous round's reads are done
           if (myc > 0 && rank0 < r0 + kMaxCand && rank0 + myc > r0) {
             int rk = rank0;
 #pragma unroll
-            for (int w = 0; w < 2; ++w) {
+            for (int w = 0; w < 3; ++w) {
               uint32_t bits = cm[w];
               while (bits) {
                 const int b = __ffs(bits) - 1;
                 bits &= bits - 1;
+                const int v = 32 * w + b, p = v >> 1;
                 if (rk >= r0 && rk < r0 + kMaxCand)
-                  S.cand[rk - r0] = o * 128 + oh * 64 + w * 32 + b;
+                  S.cand[rk - r0] = (p >> 2) * 1024 + co * 8 + (p & 3) * 2 + (v & 1);
                 ++rk;
               }
             }
@@ -518,42 +532,34 @@ k_tc12288(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ s
           group_sync(g);
           const int nc = min(kMaxCand, total - r0);
           for (int c = 0; c < nc; ++c) {
-            double part = warp_sum_d(exact_partial(tok, S.cand[c], tau));
-            if (lane == 0) S.part[c & 1][wg] = part;
+            double part = warp_sum_d(exact_at(S.cand[c]));
+            if (lane == 0) S.part[c & 1][q] = part;
             group_sync(g);
-            double sum = 0.0;
-#pragma unroll
-            for (int w = 0; w < kGroupWarps; ++w) sum += S.part[c & 1][w];
+            const double sum = (S.part[c & 1][0] + S.part[c & 1][1]) +
+                               (S.part[c & 1][2] + S.part[c & 1][3]);
             best = fmax(best, fabs(sum));
           }
         }
       }
-      if (tau == 0) mbar_arrive(&empty[st]);   // every read of the stage is behind a group sync
+      if (co == 0) mbar_arrive(&empty[st]);   // every read of the stage is behind a group sync
 
-      // ---- scale and codes: 32 bytes per row thread.  A row holding an
+      // ---- scale and codes: one 32-bit word per i12.  A row holding an
       // infinity or NaN gets the scale of its computed maximum (not exact).
-      if (!finite) best = (double)M;
-      const float scale = (M > 0.0f || !finite) ? __double2float_rn((best / P.sqrt_n) / 7.0)
-                                                : 0.0f;
-      if (rowv) {
-        tmem_wait_st();
-        const float cq = scale > 0.0f ? __double2float_rn(1.0 / (P.sqrt_n * (double)scale)) : 0.0f;
+      float scale = 0.0f;
+      if (!finite)
+        scale = __double2float_rn(((double)M / P.sqrt_n) / 7.0);
+      else if (M > 0.0f)
+        scale = __double2float_rn(div_rn(div_rn(best, P.sqrt_n, P.rcp_sqrt_n), 7.0, 1.0 / 7.0));
+      if (ok) {
+        // 1 / (sqrt(n) scale) in fp32 (an error of a few ulp moves only codes
+        // within far less than 1e-5 of a rounding boundary)
+        const float cq = scale > 0.0f ? __frcp_rn((float)P.sqrt_n * scale) : 0.0f;
         const float2 c2 = make_float2(cq, cq);
-        uint4* dst = reinterpret_cast<uint4*>(P.codes + token * (N / 2) + o * 64 + oh * 32);
+        uint32_t* dst = reinterpret_cast<uint32_t*>(P.codes + token * (N / 2)) + co;
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          float2 h[16];
-          tmem_ld32(taddr + oh * 64 + c * 32,
-                    *reinterpret_cast<uint32_t(*)[32]>(reinterpret_cast<uint32_t*>(h)));
-          tmem_wait_ld();
-          if (ok)
-            dst[c] = make_uint4(int4x8(h, c2), int4x8(h + 4, c2), int4x8(h + 8, c2),
-                                int4x8(h + 12, c2));
-        }
+        for (int i12 = 0; i12 < 12; ++i12) dst[i12 * 128] = int4x8(f + 4 * i12, c2);
+        if (co == 0) P.scales[token] = scale;
       }
-      tc_fence_before();
-      mbar_arrive(&tempty[d]);
-      if (ok && tau == 0) P.scales[token] = scale;
     }
   }
 
@@ -572,17 +578,14 @@ k_tc12288(const __grid_constant__ CUtensorMap tmap, const int8_t* __restrict__ s
 namespace {
 
 constexpr size_t kTcpSmem = 1024 + 32768 + tcp::kStages * tcp::kStageBytes +
-                            tcp::kChunks * 16 + 4 * sizeof(tcp::GroupScratch) + 256;
+                            2 * tcp::kGroups * sizeof(tcp::GroupScratch) + 64 + 256;
 
 template <int kMode>
 cudaError_t launch_tcp(const void* x, const int8_t* signs, tcp::Params& P, const Geometry& g,
                        cudaStream_t s) {
-  CUtensorMap map;
-  // [tokens * 96, 128] view: rows of 256 bytes, 64 x 96 boxes (half a token)
-  if (!encode_tmap_bf16_2d(&map, x, tcp::kCols, (uint64_t)P.tokens * tcp::kRows, 64,
-                           tcp::kRows, CU_TENSOR_MAP_SWIZZLE_128B))
-    return cudaErrorNotSupported;
+  P.x = static_cast<const uint16_t*>(x);
   P.sqrt_n = g.sqrt_b;
+  P.rcp_sqrt_n = 1.0 / g.sqrt_b;
   auto k = tcp::k_tc12288<kMode>;
   cudaFuncSetAttribute((const void*)k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        (int)kTcpSmem);
@@ -590,16 +593,17 @@ cudaError_t launch_tcp(const void* x, const int8_t* signs, tcp::Params& P, const
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t grid = P.tokens < sms ? P.tokens : sms;
-  k<<<(int)grid, tcp::kThreads, kTcpSmem, s>>>(map, signs, P);
+  k<<<(int)grid, tcp::kThreads, kTcpSmem, s>>>(signs, P);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 bool tcp_supported(const Geometry& g, int dtype, const void* x, int64_t tokens) {
-  // TMA: 16-byte aligned base, int32 row coordinates (tokens * 96)
+  // bulk copies: a 16-byte aligned base (each row is 24 KB, so every row is
+  // aligned); 32-bit token counters in the epilogue
   return dtype == 1 && g.paley && g.b == g.n && g.n == tcp::N &&
-         (reinterpret_cast<uintptr_t>(x) & 15) == 0 && tokens < (int64_t(1) << 24);
+         (reinterpret_cast<uintptr_t>(x) & 15) == 0 && tokens < (int64_t(1) << 31);
 }
 
 cudaError_t launch_tcp_int4(const void* x, int64_t tokens, const Geometry& g,
