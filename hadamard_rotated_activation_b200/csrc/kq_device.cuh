@@ -69,6 +69,16 @@ __device__ __forceinline__ bool paley_negative(int a, int c) {
   return (w >> (k & 31)) & 1u;
 }
 
+// a / b correctly rounded for finite a and a constant b, from rb = RN(1 / b):
+// q0 = RN(a rb) is within an ulp, its residual a - q0 b is exact under an
+// FMA, and one correction step gives the rounded quotient (Markstein's
+// theorem for fused multiply-add); a short dependent chain instead of a
+// division routine.
+__device__ __forceinline__ double div_rn(double a, double b, double rb) {
+  const double q0 = a * rb;
+  return fma(fma(-q0, b, a), rb, q0);
+}
+
 // ------------------------------------------------------------ KV-cache rows
 // Output unit of input unit u (kpr units of 128 per row) when rows go to the
 // cache rows a slot mapping names: slot[u / kpr] * kpr + u % kpr, or -1 when

@@ -401,8 +401,12 @@ k_tcb128_asym(const __grid_constant__ CUtensorMap tmap, Params P) {
         double smax, smin;
         tile_exact_minmax(stile, q * 32 + src, smax, smin);
         if (lane == src) {
-          const double ymx = smax / 11.313708498984761, ymn = smin / 11.313708498984761;
-          s16 = f64_to_f16_bits((ymx - ymn) / 15.0);
+          constexpr double kSqrt128 = 11.313708498984761;   // IEEE sqrt(128)
+          const bool fin = isfinite(smax) && isfinite(smin);
+          const double ymx = fin ? div_rn(smax, kSqrt128, 1.0 / kSqrt128) : smax / kSqrt128;
+          const double ymn = fin ? div_rn(smin, kSqrt128, 1.0 / kSqrt128) : smin / kSqrt128;
+          const double rng = ymx - ymn;
+          s16 = f64_to_f16_bits(isfinite(rng) ? div_rn(rng, 15.0, 1.0 / 15.0) : rng / 15.0);
           const double sd = f16_bits_to_f64((uint16_t)s16);
           zf = sd > 0.0 ? (float)rint(-ymn / sd) : 0.0f;
         }

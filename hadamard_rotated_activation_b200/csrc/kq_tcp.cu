@@ -92,14 +92,6 @@ struct Params {
   double rcp_sqrt_n;     // fp64 1 / sqrt_n, correctly rounded
 };
 
-// a / b correctly rounded for finite a, from rb = RN(1 / b): q0 = RN(a rb) is
-// within an ulp, its residual a - q0 b is exact under an FMA, and one
-// correction step gives the rounded quotient (Markstein's theorem for fused
-// multiply-add); a short dependent chain instead of a division routine.
-__device__ __forceinline__ double div_rn(double a, double b, double rb) {
-  const double q0 = a * rb;
-  return fma(fma(-q0, b, a), rb, q0);
-}
 
 // Per-group scratch for the token reductions.
 struct GroupScratch {
