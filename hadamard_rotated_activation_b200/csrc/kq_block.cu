@@ -1,15 +1,16 @@
-// Thread-per-block kernels for 128-wide Hadamard blocks (block = 128).
+// SIMT kernels for 128-wide Hadamard blocks (block = 128).
 //
 // "Block-Hadamard-128" (NVFP4 thread, discrete_descent's note) and the
 // per-head 128-point Hadamard of the KV cache (QuaRot reviews, final comments)
-// apply an independent H_128 to every 128 consecutive columns.  Here one
-// thread owns one (row, block) unit: its 128 inputs arrive by sixteen 16-byte
-// loads straight into registers, the sign flips are XORs on the bf16 sign
-// bits, and the seven butterfly stages run in registers (stage 0 in scalar
-// fp32, stages 1..6 on packed f32x2 pairs).  The 16-element NVFP4 blocks and
-// the 128-element INT4 groups lie inside the thread, so extrema, scales,
-// rounding and nibble packing need no communication.  There is no shared
-// memory and no barrier.
+// apply an independent H_128 to every 128 consecutive columns.
+//   * Asymmetric INT4: one thread owns one (row, block) unit: its 128 inputs
+//     arrive from a per-warp shared-memory stage, the sign flips are XORs on
+//     the bf16 sign bits, and the seven butterfly stages run in registers
+//     (stage 0 in scalar fp32, stages 1..6 on packed f32x2 pairs).  The
+//     128-element group lies inside the thread, so extrema, scale, zero
+//     point, rounding and nibble packing need no communication.
+//   * NVFP4: four lanes share a unit (five stages in registers, two across
+//     the quad by shuffles); each lane then owns two whole 16-blocks.
 //
 // Exact scales.  The fp32 transform of one 128-block is within
 // E = gamma_7 sqrt(128) max|S_hat| of the exact sums (see error_bound in
@@ -208,15 +209,59 @@ __device__ __forceinline__ float e4m3_recip(uint32_t c) {
   return ldexpf(r, 7 - (int)e);
 }
 
-// ---------------------------------------------------------------- NVFP4
+// ------------------------------------------------ NVFP4, four lanes a block
+// Four lanes (a quad) share one 128-block: lane j of the quad loads the 64
+// contiguous bytes of elements 32j .. 32j+31 (a warp reads 2 KB contiguous),
+// runs the five in-lane butterfly stages (bit 0 in scalar fp32, bits 1-4 on
+// f32x2 pairs) and the two stages across the quad (bits 5 and 6, shuffles),
+// and then holds the outputs 32j .. 32j+31: its two NVFP4 16-blocks.  Same
+// seven fp32 stages as a thread-per-block transform, so the same bound
+// E = e_coef max|S_hat| over the block.  A quad per block gives four times the
+// warps of a thread per block, which the short c2-sized inputs need (12.5
+// against 14.4 us on 2048 x 4096; 55.2 against 56.0 us on 16384 x 4096).
+constexpr int kQThreads = 256;
+constexpr int kQLanes = 4;
+
+// Exact S of element e (0..127) of 128-block u, computed by the whole warp in
+// fp64 from global memory (lane l sums inputs 4l .. 4l+3, with the staged sign
+// masks of column block k); every lane gets the result.
+__device__ __noinline__ double warp_exact_S_global(const uint16_t* __restrict__ x,
+                                                   const uint4* smask, int64_t u, int k, int e) {
+  const int lane = threadIdx.x & 31;
+  const uint2 w = __ldg(reinterpret_cast<const uint2*>(x + u * B) + lane);
+  uint32_t ma = 0, mb = 0;
+  if (smask) {
+    const uint4 m = smask[k * 16 + ((lane >> 1) ^ (k & 15))];
+    ma = (lane & 1) ? m.z : m.x;
+    mb = (lane & 1) ? m.w : m.y;
+  }
+  const uint32_t pr[2] = {w.x ^ ma, w.y ^ mb};
+  double acc = 0.0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int j = 4 * lane + q;
+    const uint32_t bits = (q & 1) ? (pr[q >> 1] & 0xffff0000u) : (pr[q >> 1] << 16);
+    const double xv = (double)__uint_as_float(bits);
+    acc += (__popc(e & j) & 1) ? -xv : xv;
+  }
+  return warp_sum_d(acc);
+}
+
 // kMode 0: quantize with the static/dynamic tensor scale.
 // kMode 1: dynamic-scale statistics (row max and bound), no outputs.
-template <int kMode>
-__global__ void __launch_bounds__(kThreads, 3)
-k_blk128_nvfp4(Params P) {
-  const int lane = threadIdx.x & 31;
+// kLanes lanes share a block: each holds kEpl = 128 / kLanes consecutive
+// elements, runs log2(kEpl) butterfly stages in registers and log2(kLanes)
+// across its lane group, and owns kEpl / 16 NVFP4 blocks of the outputs.
+template <int kMode, int kLanes>
+__global__ void __launch_bounds__(kQThreads, 3)
+k_blk128_nvfp4_q(Params P) {
+  constexpr int kEpl = B / kLanes;          // elements a lane
+  constexpr int kPpl = kEpl / 2;            // f32x2 pairs a lane
+  constexpr int kCpl = kEpl / 8;            // 16-byte chunks a lane
+  constexpr int kBpl = kEpl / 16;           // NVFP4 blocks a lane
+  constexpr int kUpw = 32 / kLanes;         // blocks a warp per step
+  const int lane = threadIdx.x & 31, qj = lane & (kLanes - 1);
   float t = 0.0f, c6 = 0.0f, inv_bt = 0.0f;
-  const float sqrt_b = 11.313708498984761f;  // sqrt(128), only in fp32 factors
   if (kMode == 0) {
     if (P.ws) {
       const double g = __longlong_as_double((long long)P.ws->gmax_bits);
@@ -225,48 +270,70 @@ k_blk128_nvfp4(Params P) {
     } else {
       t = *P.tensor_scale;
     }
-    // r = max|S| / (sqrt(b) 6 t); c6 rounded down/up bracket handled by margins
     c6 = (t > 0.0f) ? (float)(1.0 / (11.313708498984761 * 6.0 * (double)t)) : 0.0f;
     inv_bt = (t > 0.0f) ? (float)(1.0 / (11.313708498984761 * (double)t)) : 0.0f;
   }
-  (void)sqrt_b;
   extern __shared__ __align__(16) uint4 smem4[];
-  uint4* stages = smem4 + (threadIdx.x >> 5) * 1024;      // two 8 KB stages per warp
-  uint4* smask = P.signs ? smem4 + (blockDim.x >> 5) * 1024 : nullptr;
-  // 1 / value of E4M3 codes 1..126 (0 takes the sign-only path, 127 is NaN)
-  float* rcp = reinterpret_cast<float*>(smem4 + (blockDim.x >> 5) * 1024 +
-                                        (P.signs ? P.n / 8 : 0));
+  uint4* smask = P.signs ? smem4 : nullptr;
+  float* rcp = reinterpret_cast<float*>(smem4 + (P.signs ? P.n / 8 : 0));
   if (smask) stage_signs(P.signs, P.n, smask);
   if (kMode == 0)
     for (int i = threadIdx.x; i < 128; i += blockDim.x)
       rcp[i] = (i >= 1 && i <= 126) ? e4m3_recip((uint32_t)i) : 0.0f;
   __syncthreads();
-  const int kpr = P.n / B;                  // column blocks per row (power of two)
+  const int kpr = P.n / B;
   const int kpr_log2 = __ffs(kpr) - 1;
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  // uniform trip count across the warp so warp-cooperative steps are safe
-  const int64_t base0 = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31);
-  if (base0 < P.units) prefetch_units(P.x, base0, P.units, stages);
-  int it = 0;
-  for (int64_t ub = base0; ub < P.units; ub += stride, ++it) {
-    const int64_t u = ub + lane;
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  // uniform trip count across the warp
+  for (int64_t ub = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * kUpw;
+       ub < P.units; ub += nwarps * kUpw) {
+    const int64_t u = ub + lane / kLanes;
     const bool active = u < P.units;
-    float2 v[64];
-    const int64_t row = active ? (u >> kpr_log2) : 0;
-    uint4* stage = stages + (it & 1) * 512;
-    __syncwarp();
-    const bool more = ub + stride < P.units;
-    if (more) prefetch_units(P.x, ub + stride, P.units, stages + ((it + 1) & 1) * 512);
-    wait_prefetch(more);
-    load_transform(stage, lane, smask, (int)(u & (kpr - 1)), v);
-    if (!active) {
+    const int k = (int)(u & (kpr - 1));
+    uint4 w[kCpl];
 #pragma unroll
-      for (int p = 0; p < 64; ++p) v[p] = make_float2(0.f, 0.f);
+    for (int c = 0; c < kCpl; ++c)
+      w[c] = active ? __ldg(reinterpret_cast<const uint4*>(P.x + u * B + qj * kEpl) + c)
+                    : make_uint4(0, 0, 0, 0);
+    float2 v[kPpl];
+#pragma unroll
+    for (int c = 0; c < kCpl; ++c) {
+      uint32_t ww[4] = {w[c].x, w[c].y, w[c].z, w[c].w};
+      if (smask) {
+        const uint4 m = smask[k * 16 + ((qj * kCpl + c) ^ (k & 15))];
+        ww[0] ^= m.x;
+        ww[1] ^= m.y;
+        ww[2] ^= m.z;
+        ww[3] ^= m.w;
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float lo = __uint_as_float(ww[q] << 16);
+        const float hi = __uint_as_float(ww[q] & 0xffff0000u);
+        v[4 * c + q] = make_float2(lo + hi, lo - hi);   // stage on bit 0
+      }
     }
-    // per 16-block maxima
-    float bm[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int h = 1; h < kPpl; h <<= 1)
+#pragma unroll
+      for (int p = 0; p < kPpl; ++p)
+        if (!(p & h)) bfly2(v[p], v[p | h]);
+    // the high index bits: across the lane group (the lane with the bit set
+    // keeps a - b)
+#pragma unroll
+    for (int o = 1; o < kLanes; o <<= 1) {
+      const float2 sg = (qj & o) ? make_float2(-1.0f, -1.0f) : make_float2(1.0f, 1.0f);
+#pragma unroll
+      for (int p = 0; p < kPpl; ++p) {
+        const float2 pv = make_float2(__shfl_xor_sync(0xffffffffu, v[p].x, o),
+                                      __shfl_xor_sync(0xffffffffu, v[p].y, o));
+        v[p] = fma2(v[p], sg, pv);
+      }
+    }
+    // the lane's blocks: outputs kEpl qj + 16 j .. +15
+    float bm[kBpl];
+#pragma unroll
+    for (int j = 0; j < kBpl; ++j) {
       float m = 0.0f;
 #pragma unroll
       for (int p = 8 * j; p < 8 * j + 8; ++p) m = fmax3(m, fabsf(v[p].x), fabsf(v[p].y));
@@ -274,11 +341,14 @@ k_blk128_nvfp4(Params P) {
     }
     float mh = bm[0];
 #pragma unroll
-    for (int j = 1; j < 8; ++j) mh = fmaxf(mh, bm[j]);
+    for (int j = 1; j < kBpl; ++j) mh = fmaxf(mh, bm[j]);
+#pragma unroll
+    for (int o = 1; o < kLanes; o <<= 1) mh = fmaxf(mh, __shfl_xor_sync(0xffffffffu, mh, o));
     const float E = __fmul_ru(P.e_coef, mh);
+    const int64_t row = active ? (u >> kpr_log2) : 0;
 
     if (kMode == 1) {
-      if (active) {
+      if (active && qj == 0) {
         const float lower = fmaxf(__fsub_rd(mh, E), 0.0f);
         atomicMax(reinterpret_cast<unsigned int*>(&P.ws->rows[row].x), __float_as_uint(mh));
         atomicMax(reinterpret_cast<unsigned int*>(&P.ws->rows[row].y), __float_as_uint(E));
@@ -287,39 +357,39 @@ k_blk128_nvfp4(Params P) {
       continue;
     }
 
-    // E4M3 block scales from the interval [m - E, m + E] (scaled by c6 with a
-    // relative margin covering every fp32 rounding on the way); sc holds the
-    // eight codes as bytes
-    uint32_t sc[2] = {0, 0};
-    uint32_t undecided = 0;
+    // E4M3 block scales from [m - E, m + E] (scaled by c6 with a relative
+    // margin covering every fp32 rounding on the way)
+    uint32_t sc = 0, undecided = 0;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < kBpl; ++j) {
       const float lo = fmaxf(bm[j] - E, 0.0f) * c6 * (1.0f - 0x1p-20f);
       const float hi = (bm[j] + E) * c6 * (1.0f + 0x1p-20f);
       const uint32_t cc = e4m3_pair(lo, hi);
-      sc[j >> 2] |= (cc & 0xffu) << (8 * (j & 3));
+      sc |= (cc & 0xffu) << (8 * j);
       if ((cc & 0xffu) != (cc >> 8)) undecided |= 1u << j;
     }
-    if (t <= 0.0f) undecided = 0;
+    if (t <= 0.0f || !active) undecided = 0;
     // warp-cooperative exact fix-up of undecided block scales
-    unsigned todo = __ballot_sync(0xffffffffu, active && undecided != 0);
+    unsigned todo = __ballot_sync(0xffffffffu, undecided != 0);
     while (todo) {
       const int src = __ffs(todo) - 1;
       todo &= todo - 1;
       const uint32_t und = __shfl_sync(0xffffffffu, undecided, src);
-      const int kk = (int)((ub + src) & (kpr - 1));
-      for (int j = 0; j < 8; ++j) {
+      const int64_t usrc = __shfl_sync(0xffffffffu, u, src);
+      const int ksrc = __shfl_sync(0xffffffffu, k, src);
+#pragma unroll 1
+      for (int j = 0; j < kBpl; ++j) {
         if (!((und >> j) & 1u)) continue;
-        // candidates: |S_hat| >= bm[j] - 2E inside block j of thread src
+        // candidates: |S_hat| >= bm[j] - 2E inside block j of lane src
         uint32_t cand = 0;
         if (lane == src) {
-          float thr = 0.0f, bmj = 0.0f;
+          float bmj = bm[0];
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
+          for (int q = 1; q < kBpl; ++q)
             if (q == j) bmj = bm[q];
-          thr = bmj - 2.0f * E;
+          const float thr = bmj - 2.0f * E;
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
+          for (int q = 0; q < kBpl; ++q) {
             if (q != j) continue;
 #pragma unroll
             for (int p = 0; p < 8; ++p) {
@@ -330,68 +400,65 @@ k_blk128_nvfp4(Params P) {
           }
         }
         cand = __shfl_sync(0xffffffffu, cand, src);
+        const int e0 = kEpl * (src & (kLanes - 1)) + 16 * j;
         double best = 0.0;
         while (cand) {
           const int e = __ffs(cand) - 1;
           cand &= cand - 1;
-          best = fmax(best, fabs(warp_exact_S(stage, smask, src, kk, 16 * j + e)));
+          best = fmax(best, fabs(warp_exact_S_global(P.x, smask, usrc, ksrc, e0 + e)));
         }
         const double y = best / 11.313708498984761;
         const float r = __double2float_rn(y / (6.0 * (double)t));
         const uint32_t code = e4m3_pair(r, r) & 0xffu;
-        if (lane == src) {
-          const int w = j >> 2, sh = 8 * (j & 3);
-          sc[w] = (sc[w] & ~(0xffu << sh)) | (code << sh);
-        }
+        if (lane == src) sc = (sc & ~(0xffu << (8 * j))) | (code << (8 * j));
       }
     }
-    // codes, two 16-blocks (one 16-byte chunk) at a time, straight to global
-    uint4* dst = reinterpret_cast<uint4*>(P.codes + u * (B / 2));
+    // codes: the lane's kEpl outputs are kEpl / 2 bytes
+    uint32_t words[2 * kBpl];
     const float2 zero2 = make_float2(0.0f, 0.0f);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      uint32_t words[4];
+    for (int j = 0; j < kBpl; ++j) {
+      const uint32_t code = (sc >> (8 * j)) & 0xffu;
+      if (code != 0 && t > 0.0f) {
+        const float c = inv_bt * rcp[code];
+        const float2 c2 = make_float2(c, c);
+        float q[16];
 #pragma unroll
-      for (int jj = 0; jj < 2; ++jj) {
-        const int j = 2 * k + jj;
-        const uint32_t code = (sc[j >> 2] >> (8 * (j & 3))) & 0xffu;
-        if (code != 0 && t > 0.0f) {
-          const float c = inv_bt * rcp[code];
-          const float2 c2 = make_float2(c, c);
-          float q[16];
-#pragma unroll
-          for (int p = 0; p < 8; ++p) {
-            const float2 a = fma2(v[8 * j + p], c2, zero2);   // + 0 turns -0 into +0
-            q[2 * p] = a.x;
-            q[2 * p + 1] = a.y;
-          }
-          words[2 * jj] = e2m1x8_hw(q);
-          words[2 * jj + 1] = e2m1x8_hw(q + 8);
-        } else {
-          uint32_t w0 = 0, w1 = 0;
-#pragma unroll
-          for (int p = 0; p < 4; ++p) {
-            w0 |= (v[8 * j + p].x < 0.0f ? 8u : 0u) << (8 * p);
-            w0 |= (v[8 * j + p].y < 0.0f ? 8u : 0u) << (8 * p + 4);
-            w1 |= (v[8 * j + 4 + p].x < 0.0f ? 8u : 0u) << (8 * p);
-            w1 |= (v[8 * j + 4 + p].y < 0.0f ? 8u : 0u) << (8 * p + 4);
-          }
-          words[2 * jj] = w0;
-          words[2 * jj + 1] = w1;
+        for (int p = 0; p < 8; ++p) {
+          const float2 a = fma2(v[8 * j + p], c2, zero2);   // + 0 turns -0 into +0
+          q[2 * p] = a.x;
+          q[2 * p + 1] = a.y;
         }
+        words[2 * j] = e2m1x8_hw(q);
+        words[2 * j + 1] = e2m1x8_hw(q + 8);
+      } else {
+        uint32_t w0 = 0, w1 = 0;
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          w0 |= (v[8 * j + p].x < 0.0f ? 8u : 0u) << (8 * p);
+          w0 |= (v[8 * j + p].y < 0.0f ? 8u : 0u) << (8 * p + 4);
+          w1 |= (v[8 * j + 4 + p].x < 0.0f ? 8u : 0u) << (8 * p);
+          w1 |= (v[8 * j + 4 + p].y < 0.0f ? 8u : 0u) << (8 * p + 4);
+        }
+        words[2 * j] = w0;
+        words[2 * j + 1] = w1;
       }
-      if (active) dst[k] = make_uint4(words[0], words[1], words[2], words[3]);
     }
     if (active) {
-      if (P.sf_kc4 == 0) {
-        *reinterpret_cast<uint2*>(P.scales8 + u * (B / 16)) = make_uint2(sc[0], sc[1]);
-      } else {
-        // blocks 8 kk .. 8 kk + 7 of the row: two words of the tensor-core layout
-        const int c0 = (int)(u & (kpr - 1)) * (B / 16);
-        *reinterpret_cast<uint32_t*>(P.scales8 + sf_offset(row, c0, P.n / 16, P.sf_kc4)) = sc[0];
-        *reinterpret_cast<uint32_t*>(P.scales8 + sf_offset(row, c0 + 4, P.n / 16, P.sf_kc4)) =
-            sc[1];
-      }
+      uint8_t* cdst = P.codes + u * (B / 2) + qj * (kEpl / 2);
+      if (kBpl == 2)
+        *reinterpret_cast<uint4*>(cdst) = make_uint4(words[0], words[1], words[2], words[3]);
+      else
+        *reinterpret_cast<uint2*>(cdst) = make_uint2(words[0], words[1]);
+      // the lane's blocks start at an index that is a multiple of kBpl: they are
+      // consecutive bytes in either layout
+      const int c0 = k * (B / 16) + kBpl * qj;
+      const int64_t off = P.sf_kc4 == 0 ? u * (B / 16) + kBpl * qj
+                                        : sf_offset(row, c0, P.n / 16, P.sf_kc4);
+      if (kBpl == 2)
+        *reinterpret_cast<uint16_t*>(P.scales8 + off) = (uint16_t)sc;
+      else
+        P.scales8[off] = (uint8_t)sc;
     }
   }
 }
@@ -561,6 +628,20 @@ bool blk128_supported(const Geometry& g, int dtype) {
   return dtype == 1 && g.b == 128 && !g.paley && g.n % 128 == 0 && (kpr & (kpr - 1)) == 0;
 }
 
+int qblk_grid(const void* kernel, int64_t units, size_t smem) {
+  int dev = 0, sms = 0, per_sm = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (smem > 48 * 1024)
+    cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, blk::kQThreads, smem);
+  if (per_sm < 1) per_sm = 1;
+  const int64_t per_cta = (blk::kQThreads / 32) * (32 / blk::kQLanes);   // blocks per step
+  const int64_t need = (units + per_cta - 1) / per_cta;
+  const int64_t cap = (int64_t)sms * per_sm;
+  return (int)(need < cap ? need : cap);
+}
+
 cudaError_t launch_blk128_nvfp4(const void* x, int64_t tokens, const Geometry& g,
                                 const int8_t* signs, uint8_t* codes, uint8_t* bscales,
                                 float* tensor_scale, NvWorkspace* ws, cudaStream_t s) {
@@ -575,15 +656,15 @@ cudaError_t launch_blk128_nvfp4(const void* x, int64_t tokens, const Geometry& g
   P.n = g.n;
   P.e_coef = e_coef_128();
   P.sf_kc4 = g.sf_kc4;
+  const size_t smq = (signs ? (size_t)g.n / 8 * 16 : 0) + 128 * 4;
   if (ws) {
     const int ph = g.dyn ? g.dyn : 7;
     if (ph & 1) {
       cudaError_t e =
           cudaMemsetAsync(ws, 0, kNvWorkspaceHeader + (size_t)tokens * sizeof(float2), s);
       if (e != cudaSuccess) return e;
-      auto k1 = blk::k_blk128_nvfp4<1>;
-      const size_t sm1 = blk_smem(g.n, signs != nullptr);
-      k1<<<blk_grid((const void*)k1, P.units, sm1), blk::kThreads, sm1, s>>>(P);
+      auto k1 = blk::k_blk128_nvfp4_q<1, blk::kQLanes>;
+      k1<<<qblk_grid((const void*)k1, P.units, smq), blk::kQThreads, smq, s>>>(P);
       e = cudaGetLastError();
       if (e != cudaSuccess) return e;
     }
@@ -593,9 +674,8 @@ cudaError_t launch_blk128_nvfp4(const void* x, int64_t tokens, const Geometry& g
     }
     if (!(ph & 4)) return cudaSuccess;
   }
-  auto k0 = blk::k_blk128_nvfp4<0>;
-  const size_t sm0 = blk_smem(g.n, signs != nullptr);
-  k0<<<blk_grid((const void*)k0, P.units, sm0), blk::kThreads, sm0, s>>>(P);
+  auto k0 = blk::k_blk128_nvfp4_q<0, blk::kQLanes>;
+  k0<<<qblk_grid((const void*)k0, P.units, smq), blk::kQThreads, smq, s>>>(P);
   return cudaGetLastError();
 }
 
