@@ -115,7 +115,8 @@ def test_guards_int4_asym(dim, tokens, signs):
 
 NV_SHAPES = [
     (4096, 0, 37),               # 4096-wide tensor-core kernel (statistics pass too)
-    (4096, 128, 37),             # block-128 thread-per-block kernel
+    (4096, 128, 37),             # block-128 kernel, four lanes per block
+    (128, 128, 37),              # the same with a ragged last step (37 blocks)
     (2048, 0, 37),               # warp per row
     (12288, 0, 7),               # row per CTA
 ]

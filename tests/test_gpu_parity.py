@@ -155,6 +155,21 @@ def test_nvfp4_small_dynamic_and_static(key, tokens):
     assert np.array_equal(deq.view(np.uint32), want.view(np.uint32))
 
 
+@pytest.mark.parametrize("dim,tokens", [(128, 37), (256, 41), (512, 3)])
+def test_nvfp4_block128_ragged_lane_groups(dim, tokens):
+    """Block-128 NVFP4 with a block count that is not a multiple of a warp's
+    eight blocks (four lanes per block): the idle lanes of the last step write
+    nothing and the active ones stay exact, in both tensor-scale modes."""
+    w = wl.Workload("c2", tokens, dim, wl.BF16, 128, True, wl.NVFP4, 13)
+    inp = wl.make_inputs(w)
+    y = oracle.rht(inp.values, inp.signs, 128)
+    codes, bs, ts = P.gpu_nvfp4(inp)
+    P.check_nvfp4(codes, bs, ts, y)
+    t = np.float32(ts * 0.5)
+    c2, b2, _ = P.gpu_nvfp4(inp, tensor_scale=t)
+    P.check_nvfp4(c2, b2, t, y, tensor_scale=t)
+
+
 @pytest.mark.parametrize("key,tokens", [("c2", 2500), ("c4", 2500)])
 def test_nvfp4_dynamic_every_row_a_candidate(key, tokens):
     """Identical rows all reach the global lower bound, so the dynamic global
