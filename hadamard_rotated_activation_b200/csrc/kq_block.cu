@@ -17,6 +17,12 @@
 // kq_device.cuh).  A scale is decided from the fp32 values when both ends of
 // its interval round to the same stored value; the rare undecided ones are
 // recomputed by the whole warp as exact fp64 dot products with the input.
+//
+// Dynamic NVFP4 tensor scale: a statistics pass (row maxima and bounds), then
+// the quantisation pass, which on up to kFusedExactRows rows finds the exact
+// global maximum itself (each CTA screens every row's statistics and
+// transforms the candidate rows in fp64) and is launched as a programmatic
+// dependent of the statistics pass.
 #include <cfloat>
 #include <climits>
 #include <cstdint>
@@ -45,6 +51,7 @@ struct Params {
   int n;
   float e_coef;                 // E = e_coef * max|S_hat| (rounded up)
   int sf_kc4;                   // NVFP4 scale layout (Geometry::sf_kc4)
+  int fuse_exact;               // NVFP4 dynamic quantisation: compute the exact maximum first
 };
 
 __device__ __forceinline__ int stage_chunk(int unit, int c);
@@ -247,11 +254,145 @@ __device__ __noinline__ double warp_exact_S_global(const uint16_t* __restrict__ 
   return warp_sum_d(acc);
 }
 
+// max |S| over the outputs of up to four 128-blocks at once, in fp64: eight
+// lanes a block (lanes 8i .. 8i+7 take block u_i of column block k_i, or
+// nothing if u_i < 0); lane j of the eight holds inputs 16j .. 16j+15 (signs
+// applied, exact in fp64), runs index bits 0 .. 3 as butterflies in the lane
+// and bits 4 .. 6 across the eight.  Every lane gets the maximum over the
+// four blocks.
+__device__ __noinline__ double warp_blocks_absmax_f64(const uint16_t* __restrict__ x,
+                                                      const uint4* smask, int64_t u, int k) {
+  const int lane = threadIdx.x & 31, j = lane & 7;
+  double v[16];
+  if (u >= 0) {
+    const uint4* src = reinterpret_cast<const uint4*>(x + u * B) + 2 * j;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint4 w = __ldg(src + h);
+      uint4 m = make_uint4(0, 0, 0, 0);
+      if (smask) m = smask[k * 16 + ((2 * j + h) ^ (k & 15))];
+      const uint32_t ww[4] = {w.x ^ m.x, w.y ^ m.y, w.z ^ m.z, w.w ^ m.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        v[8 * h + 2 * q] = (double)__uint_as_float(ww[q] << 16);
+        v[8 * h + 2 * q + 1] = (double)__uint_as_float(ww[q] & 0xffff0000u);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) v[e] = 0.0;
+  }
+#pragma unroll
+  for (int st = 1; st < 16; st <<= 1)
+#pragma unroll
+    for (int e = 0; e < 16; ++e)
+      if (!(e & st)) {
+        const double a = v[e], b = v[e | st];
+        v[e] = a + b;
+        v[e | st] = a - b;
+      }
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1)
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const double p = __shfl_xor_sync(0xffffffffu, v[e], o);
+      v[e] = (lane & o) ? p - v[e] : v[e] + p;
+    }
+  double m = 0.0;
+#pragma unroll
+  for (int e = 0; e < 16; ++e) m = fmax(m, fabs(v[e]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, o));
+  return m;
+}
+
+// The exact maximum of the dynamic tensor scale, computed by one whole CTA
+// from the row statistics of the workspace: rows whose bound reaches the
+// global lower bound are candidates, and every 128-block of a candidate row
+// is transformed in fp64 (eight lanes a block, four blocks a warp).  A row
+// whose computed maximum is zero has E = 0 and is exactly zero.  The row
+// statistics are read eight rows a thread at a time into one candidate list;
+// if more rows qualify than the list holds (many rows tied), each warp screens
+// and finishes rows on its own instead, which costs one fp64 transform per
+// tied row.  Every thread of the CTA must call it; all get max |S| (fp64,
+// unnormalised).
+constexpr int kTailCand = 512;
+__device__ __forceinline__ bool tail_candidate(float2 st, float L) {
+  return st.x > 0.0f && (double)st.x + (double)st.y >= (double)L;
+}
+__device__ __noinline__ double cta_exact_max(const uint16_t* __restrict__ x, const NvWorkspace* ws,
+                                             int64_t units, const uint4* smask, int kpr_log2) {
+  __shared__ int64_t s_cand[kTailCand];
+  __shared__ int s_nc;
+  __shared__ double s_m[kQThreads / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const float L = __uint_as_float(__ldcg(&ws->lower_bits));
+  const int64_t tokens = units >> kpr_log2;
+  const int kpr = 1 << kpr_log2;
+  if (threadIdx.x == 0) s_nc = 0;
+  __syncthreads();
+  for (int64_t base = 0; base < tokens; base += 8 * (int64_t)blockDim.x) {
+    float2 st[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int64_t r = base + i * (int64_t)blockDim.x + threadIdx.x;
+      st[i] = r < tokens ? __ldcg(&ws->rows[r]) : make_float2(0.0f, 0.0f);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if (tail_candidate(st[i], L)) {
+        const int slot = atomicAdd(&s_nc, 1);
+        if (slot < kTailCand) s_cand[slot] = base + i * (int64_t)blockDim.x + threadIdx.x;
+      }
+  }
+  __syncthreads();
+  const int nc = s_nc;
+  double m = 0.0;
+  if (nc <= kTailCand) {
+    // (row, block) pairs, four a warp at a time
+    const int npairs = nc << kpr_log2;
+    for (int p0 = 4 * warp; p0 < npairs; p0 += 4 * nw) {
+      const int p = p0 + (lane >> 3);
+      const int kb = p & (kpr - 1);
+      const int64_t u = p < npairs ? (s_cand[p >> kpr_log2] << kpr_log2) + kb : -1;
+      m = fmax(m, warp_blocks_absmax_f64(x, smask, u, kb));
+    }
+  } else {
+    for (int64_t r0 = (int64_t)warp * 32; r0 < tokens; r0 += (int64_t)nw * 32) {
+      const int64_t r = r0 + lane;
+      const bool c = r < tokens && tail_candidate(__ldcg(&ws->rows[r]), L);
+      unsigned todo = __ballot_sync(0xffffffffu, c);
+      while (todo) {
+        const int src = __ffs(todo) - 1;
+        todo &= todo - 1;
+        for (int kb0 = 0; kb0 < kpr; kb0 += 4) {
+          const int kb = kb0 + (lane >> 3);
+          const int64_t u = kb < kpr ? ((r0 + src) << kpr_log2) + kb : -1;
+          m = fmax(m, warp_blocks_absmax_f64(x, smask, u, kb));
+        }
+      }
+    }
+  }
+  if (lane == 0) s_m[warp] = m;
+  __syncthreads();
+  double t = s_m[0];
+  for (int w = 1; w < nw; ++w) t = fmax(t, s_m[w]);
+  return t;
+}
+
+// Inputs of the largest row count whose quantisation pass computes the exact
+// maximum itself (every CTA reads all row statistics in its prologue); larger
+// inputs run the exact-maximum step as a launch of its own.
+constexpr int64_t kFusedExactRows = 8192;
+
 // kMode 0: quantize with the static/dynamic tensor scale.
 // kMode 1: dynamic-scale statistics (row max and bound), no outputs.
-// kLanes lanes share a block: each holds kEpl = 128 / kLanes consecutive
-// elements, runs log2(kEpl) butterfly stages in registers and log2(kLanes)
-// across its lane group, and owns kEpl / 16 NVFP4 blocks of the outputs.
+// Four lanes share a block: each holds 32 consecutive elements, runs five
+// butterfly stages in registers and two across its quad, and owns two NVFP4
+// blocks of the outputs.  Dynamic quantisation takes t from the workspace's
+// exact maximum, or (P.fuse_exact) computes that maximum itself first; it
+// waits for the statistics launch (programmatic dependent launch) only after
+// the signs are staged and its first inputs are on their way into L2.
 template <int kMode, int kLanes>
 __global__ void __launch_bounds__(kQThreads, 3)
 k_blk128_nvfp4_q(Params P) {
@@ -261,21 +402,17 @@ k_blk128_nvfp4_q(Params P) {
   constexpr int kBpl = kEpl / 16;           // NVFP4 blocks a lane
   constexpr int kUpw = 32 / kLanes;         // blocks a warp per step
   const int lane = threadIdx.x & 31, qj = lane & (kLanes - 1);
-  float t = 0.0f, c6 = 0.0f, inv_bt = 0.0f;
-  if (kMode == 0) {
-    if (P.ws) {
-      const double g = __longlong_as_double((long long)P.ws->gmax_bits);
-      t = __double2float_rn((g / 11.313708498984761) / 2688.0);
-      if (blockIdx.x == 0 && threadIdx.x == 0) *P.tensor_scale = t;
-    } else {
-      t = *P.tensor_scale;
-    }
-    c6 = (t > 0.0f) ? (float)(1.0 / (11.313708498984761 * 6.0 * (double)t)) : 0.0f;
-    inv_bt = (t > 0.0f) ? (float)(1.0 / (11.313708498984761 * (double)t)) : 0.0f;
-  }
   extern __shared__ __align__(16) uint4 smem4[];
   uint4* smask = P.signs ? smem4 : nullptr;
   float* rcp = reinterpret_cast<float*>(smem4 + (P.signs ? P.n / 8 : 0));
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  const int64_t ub0 = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * kUpw;
+  if (kMode == 1) {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  } else if (ub0 + lane / kLanes < P.units) {
+    // the first step's 64 bytes of this lane, into L2 while the prologue runs
+    asm volatile("prefetch.global.L2 [%0];" :: "l"(P.x + (ub0 + lane / kLanes) * B + qj * kEpl));
+  }
   if (smask) stage_signs(P.signs, P.n, smask);
   if (kMode == 0)
     for (int i = threadIdx.x; i < 128; i += blockDim.x)
@@ -283,10 +420,29 @@ k_blk128_nvfp4_q(Params P) {
   __syncthreads();
   const int kpr = P.n / B;
   const int kpr_log2 = __ffs(kpr) - 1;
-  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  float t = 0.0f, c6 = 0.0f, inv_bt = 0.0f;
+  if (kMode == 0) {
+    // the statistics launch (if any) is complete past this point
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (P.ws) {
+      const double g = P.fuse_exact ? cta_exact_max(P.x, P.ws, P.units, smask, kpr_log2)
+                                    : __longlong_as_double((long long)__ldcg(&P.ws->gmax_bits));
+      t = __double2float_rn((g / 11.313708498984761) / 2688.0);
+      if (blockIdx.x == 0 && threadIdx.x == 0) {
+        *P.tensor_scale = t;
+        if (P.fuse_exact) P.ws->gmax_bits = (unsigned long long)__double_as_longlong(g);
+      }
+    } else {
+      t = *P.tensor_scale;
+    }
+    c6 = (t > 0.0f) ? (float)(1.0 / (11.313708498984761 * 6.0 * (double)t)) : 0.0f;
+    inv_bt = (t > 0.0f) ? (float)(1.0 / (11.313708498984761 * (double)t)) : 0.0f;
+  }
+  // lanes whose blocks share a row in one step (a power of two <= 32)
+  const int seg = kLanes * kpr < 32 ? kLanes * kpr : 32;
+  float lower = 0.0f;   // statistics: this lane's largest lower bound
   // uniform trip count across the warp
-  for (int64_t ub = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * kUpw;
-       ub < P.units; ub += nwarps * kUpw) {
+  for (int64_t ub = ub0; ub < P.units; ub += nwarps * kUpw) {
     const int64_t u = ub + lane / kLanes;
     const bool active = u < P.units;
     const int k = (int)(u & (kpr - 1));
@@ -348,15 +504,20 @@ k_blk128_nvfp4_q(Params P) {
     const int64_t row = active ? (u >> kpr_log2) : 0;
 
     if (kMode == 1) {
-      if (active && qj == 0) {
-        const float lower = fmaxf(__fsub_rd(mh, E), 0.0f);
-        atomicMax(reinterpret_cast<unsigned int*>(&P.ws->rows[row].x), __float_as_uint(mh));
-        atomicMax(reinterpret_cast<unsigned int*>(&P.ws->rows[row].y), __float_as_uint(E));
-        atomicMax(&P.ws->lower_bits, __float_as_uint(lower));
+      // one atomic pair a row and step (the row's E is e_coef times its
+      // maximum, rounded up, like every block's); one lower-bound atomic a warp
+      if (active) lower = fmaxf(lower, __fsub_rd(mh, E));
+      float rm = mh;
+#pragma unroll
+      for (int o = kLanes; o < 32; o <<= 1)
+        if (o < seg) rm = fmaxf(rm, __shfl_xor_sync(0xffffffffu, rm, o));
+      if (active && (lane & (seg - 1)) == 0) {
+        atomicMax(reinterpret_cast<unsigned int*>(&P.ws->rows[row].x), __float_as_uint(rm));
+        atomicMax(reinterpret_cast<unsigned int*>(&P.ws->rows[row].y),
+                  __float_as_uint(__fmul_ru(P.e_coef, rm)));
       }
       continue;
     }
-
     // E4M3 block scales from [m - E, m + E] (scaled by c6 with a relative
     // margin covering every fp32 rounding on the way)
     uint32_t sc = 0, undecided = 0;
@@ -460,6 +621,11 @@ k_blk128_nvfp4_q(Params P) {
       else
         P.scales8[off] = (uint8_t)sc;
     }
+  }
+  if (kMode == 1) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) lower = fmaxf(lower, __shfl_xor_sync(0xffffffffu, lower, o));
+    if (lane == 0 && lower > 0.0f) atomicMax(&P.ws->lower_bits, __float_as_uint(lower));
   }
 }
 
@@ -657,26 +823,48 @@ cudaError_t launch_blk128_nvfp4(const void* x, int64_t tokens, const Geometry& g
   P.e_coef = e_coef_128();
   P.sf_kc4 = g.sf_kc4;
   const size_t smq = (signs ? (size_t)g.n / 8 * 16 : 0) + 128 * 4;
-  if (ws) {
-    const int ph = g.dyn ? g.dyn : 7;
-    if (ph & 1) {
-      cudaError_t e =
-          cudaMemsetAsync(ws, 0, kNvWorkspaceHeader + (size_t)tokens * sizeof(float2), s);
-      if (e != cudaSuccess) return e;
-      auto k1 = blk::k_blk128_nvfp4_q<1, blk::kQLanes>;
-      k1<<<qblk_grid((const void*)k1, P.units, smq), blk::kQThreads, smq, s>>>(P);
-      e = cudaGetLastError();
-      if (e != cudaSuccess) return e;
-    }
-    if (ph & 2) {
-      cudaError_t e = launch_nvfp4_global(x, 1, tokens, g, signs, ws, s);
-      if (e != cudaSuccess) return e;
-    }
-    if (!(ph & 4)) return cudaSuccess;
-  }
   auto k0 = blk::k_blk128_nvfp4_q<0, blk::kQLanes>;
-  k0<<<qblk_grid((const void*)k0, P.units, smq), blk::kQThreads, smq, s>>>(P);
-  return cudaGetLastError();
+  const int grid0 = qblk_grid((const void*)k0, P.units, smq);
+  if (!ws) {
+    k0<<<grid0, blk::kQThreads, smq, s>>>(P);
+    return cudaGetLastError();
+  }
+  const int ph = g.dyn ? g.dyn : 7;
+  // the whole dynamic call on a modest row count: statistics, then the
+  // quantisation pass computing the exact maximum itself, launched as a
+  // programmatic dependent of the statistics (it reads only the input before
+  // waiting for them)
+  const bool fused = ph == 7 && tokens <= blk::kFusedExactRows;
+  if (ph & 1) {
+    cudaError_t e =
+        cudaMemsetAsync(ws, 0, kNvWorkspaceHeader + (size_t)tokens * sizeof(float2), s);
+    if (e != cudaSuccess) return e;
+    auto k1 = blk::k_blk128_nvfp4_q<1, blk::kQLanes>;
+    k1<<<qblk_grid((const void*)k1, P.units, smq), blk::kQThreads, smq, s>>>(P);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if ((ph & 2) && !fused) {
+    cudaError_t e = launch_nvfp4_global(x, 1, tokens, g, signs, ws, s);
+    if (e != cudaSuccess) return e;
+  }
+  if (!(ph & 4)) return cudaSuccess;
+  if (!fused) {
+    k0<<<grid0, blk::kQThreads, smq, s>>>(P);
+    return cudaGetLastError();
+  }
+  P.fuse_exact = 1;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)grid0);
+  cfg.blockDim = dim3(blk::kQThreads);
+  cfg.dynamicSmemBytes = smq;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k0, P);
 }
 
 cudaError_t launch_blk128_asym(const void* x, int64_t tokens, const Geometry& g,

@@ -170,6 +170,34 @@ def test_nvfp4_block128_ragged_lane_groups(dim, tokens):
     P.check_nvfp4(c2, b2, t, y, tensor_scale=t)
 
 
+@pytest.mark.parametrize("tokens", [600, 5])
+def test_nvfp4_block128_dynamic_tied_rows(tokens):
+    """Dynamic tensor scale when every row ties for the maximum (one row
+    repeated): all rows are candidates of the exact-maximum step, at 600 more
+    than its candidate list holds."""
+    w = wl.Workload("c2", tokens, 256, wl.BF16, 128, True, wl.NVFP4, 21)
+    inp = wl.make_inputs(w)
+    inp = wl.Inputs(w, np.repeat(inp.values[:1], tokens, axis=0),
+                    np.repeat(inp.stored[:1], tokens, axis=0), inp.signs)
+    y = oracle.rht(inp.values, inp.signs, 128)
+    codes, bs, ts = P.gpu_nvfp4(inp)
+    assert ts == oracle.nvfp4_tensor_scale(y)
+    P.check_nvfp4(codes, bs, ts, y)
+
+
+def test_nvfp4_block128_dynamic_many_rows():
+    """Dynamic block-128 NVFP4 on more rows than the quantisation pass screens
+    for the exact maximum itself (the exact step then runs as a launch of its
+    own), and on exactly that many rows."""
+    for tokens in (8193, 8192):
+        w = wl.Workload("c2", tokens, 256, wl.BF16, 128, True, wl.NVFP4, 23)
+        inp = wl.make_inputs(w)
+        y = oracle.rht(inp.values, inp.signs, 128)
+        codes, bs, ts = P.gpu_nvfp4(inp)
+        assert ts == oracle.nvfp4_tensor_scale(y)
+        P.check_nvfp4(codes, bs, ts, y)
+
+
 @pytest.mark.parametrize("key,tokens", [("c2", 2500), ("c4", 2500)])
 def test_nvfp4_dynamic_every_row_a_candidate(key, tokens):
     """Identical rows all reach the global lower bound, so the dynamic global
