@@ -380,6 +380,16 @@ __device__ __noinline__ double cta_exact_max(const uint16_t* __restrict__ x, con
   return t;
 }
 
+// The 64 input bytes of lane qj of block u (zeros past the last block).
+template <int kCpl>
+__device__ __forceinline__ void load_step(const uint16_t* __restrict__ x, int64_t u, int64_t units,
+                                          int qj, uint4 (&w)[kCpl]) {
+#pragma unroll
+  for (int c = 0; c < kCpl; ++c)
+    w[c] = u < units ? __ldg(reinterpret_cast<const uint4*>(x + u * B + qj * (kCpl * 8)) + c)
+                     : make_uint4(0, 0, 0, 0);
+}
+
 // Inputs of the largest row count whose quantisation pass computes the exact
 // maximum itself (every CTA reads all row statistics in its prologue); larger
 // inputs run the exact-maximum step as a launch of its own.
@@ -394,7 +404,7 @@ constexpr int64_t kFusedExactRows = 8192;
 // waits for the statistics launch (programmatic dependent launch) only after
 // the signs are staged and its first inputs are on their way into L2.
 template <int kMode, int kLanes>
-__global__ void __launch_bounds__(kQThreads, 3)
+__global__ void __launch_bounds__(kQThreads, kLanes >= 4 ? 3 : 2)
 k_blk128_nvfp4_q(Params P) {
   constexpr int kEpl = B / kLanes;          // elements a lane
   constexpr int kPpl = kEpl / 2;            // f32x2 pairs a lane
@@ -407,12 +417,11 @@ k_blk128_nvfp4_q(Params P) {
   float* rcp = reinterpret_cast<float*>(smem4 + (P.signs ? P.n / 8 : 0));
   const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
   const int64_t ub0 = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * kUpw;
-  if (kMode == 1) {
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  } else if (ub0 + lane / kLanes < P.units) {
-    // the first step's 64 bytes of this lane, into L2 while the prologue runs
-    asm volatile("prefetch.global.L2 [%0];" :: "l"(P.x + (ub0 + lane / kLanes) * B + qj * kEpl));
-  }
+  if (kMode == 1) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // the lane's inputs of the first step are loaded before the prologue (sign
+  // table, tensor scale), the next step's at the end of each step
+  uint4 w[kCpl];
+  load_step(P.x, ub0 + lane / kLanes, P.units, qj, w);
   if (smask) stage_signs(P.signs, P.n, smask);
   if (kMode == 0)
     for (int i = threadIdx.x; i < 128; i += blockDim.x)
@@ -446,11 +455,6 @@ k_blk128_nvfp4_q(Params P) {
     const int64_t u = ub + lane / kLanes;
     const bool active = u < P.units;
     const int k = (int)(u & (kpr - 1));
-    uint4 w[kCpl];
-#pragma unroll
-    for (int c = 0; c < kCpl; ++c)
-      w[c] = active ? __ldg(reinterpret_cast<const uint4*>(P.x + u * B + qj * kEpl) + c)
-                    : make_uint4(0, 0, 0, 0);
     float2 v[kPpl];
 #pragma unroll
     for (int c = 0; c < kCpl; ++c) {
@@ -469,6 +473,10 @@ k_blk128_nvfp4_q(Params P) {
         v[4 * c + q] = make_float2(lo + hi, lo - hi);   // stage on bit 0
       }
     }
+    // the next step's inputs: here in the statistics pass (they load during
+    // the butterflies), after the stores in the quantisation pass (whose
+    // registers are all in use until then)
+    if (kMode == 1) load_step(P.x, u + nwarps * kUpw, P.units, qj, w);
 #pragma unroll
     for (int h = 1; h < kPpl; h <<= 1)
 #pragma unroll
@@ -607,20 +615,24 @@ k_blk128_nvfp4_q(Params P) {
     }
     if (active) {
       uint8_t* cdst = P.codes + u * (B / 2) + qj * (kEpl / 2);
-      if (kBpl == 2)
-        *reinterpret_cast<uint4*>(cdst) = make_uint4(words[0], words[1], words[2], words[3]);
-      else
-        *reinterpret_cast<uint2*>(cdst) = make_uint2(words[0], words[1]);
+#pragma unroll
+      for (int h = 0; h < kBpl / 2; ++h)
+        reinterpret_cast<uint4*>(cdst)[h] =
+            make_uint4(words[4 * h], words[4 * h + 1], words[4 * h + 2], words[4 * h + 3]);
+      if (kBpl == 1) *reinterpret_cast<uint2*>(cdst) = make_uint2(words[0], words[1]);
       // the lane's blocks start at an index that is a multiple of kBpl: they are
       // consecutive bytes in either layout
       const int c0 = k * (B / 16) + kBpl * qj;
       const int64_t off = P.sf_kc4 == 0 ? u * (B / 16) + kBpl * qj
                                         : sf_offset(row, c0, P.n / 16, P.sf_kc4);
-      if (kBpl == 2)
+      if (kBpl == 4)
+        *reinterpret_cast<uint32_t*>(P.scales8 + off) = sc;
+      else if (kBpl == 2)
         *reinterpret_cast<uint16_t*>(P.scales8 + off) = (uint16_t)sc;
       else
         P.scales8[off] = (uint8_t)sc;
     }
+    load_step(P.x, u + nwarps * kUpw, P.units, qj, w);
   }
   if (kMode == 1) {
 #pragma unroll
