@@ -227,7 +227,9 @@ __device__ __forceinline__ float e4m3_recip(uint32_t c) {
 // warps of a thread per block, which the short c2-sized inputs need (12.5
 // against 14.4 us on 2048 x 4096; 55.2 against 56.0 us on 16384 x 4096).
 constexpr int kQThreads = 256;
-constexpr int kQLanes = 4;
+constexpr int kQLanes = 4;        // quantisation pass
+constexpr int kQLanesStats = 8;   // statistics pass of the dynamic tensor scale, and the
+                                  // quantisation pass that computes the exact maximum
 
 // Exact S of element e (0..127) of 128-block u, computed by the whole warp in
 // fp64 from global memory (lane l sums inputs 4l .. 4l+3, with the staged sign
@@ -806,7 +808,7 @@ bool blk128_supported(const Geometry& g, int dtype) {
   return dtype == 1 && g.b == 128 && !g.paley && g.n % 128 == 0 && (kpr & (kpr - 1)) == 0;
 }
 
-int qblk_grid(const void* kernel, int64_t units, size_t smem) {
+int qblk_grid(const void* kernel, int64_t units, size_t smem, int lanes) {
   int dev = 0, sms = 0, per_sm = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -814,7 +816,7 @@ int qblk_grid(const void* kernel, int64_t units, size_t smem) {
     cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, blk::kQThreads, smem);
   if (per_sm < 1) per_sm = 1;
-  const int64_t per_cta = (blk::kQThreads / 32) * (32 / blk::kQLanes);   // blocks per step
+  const int64_t per_cta = (blk::kQThreads / 32) * (32 / lanes);   // blocks per step
   const int64_t need = (units + per_cta - 1) / per_cta;
   const int64_t cap = (int64_t)sms * per_sm;
   return (int)(need < cap ? need : cap);
@@ -836,7 +838,7 @@ cudaError_t launch_blk128_nvfp4(const void* x, int64_t tokens, const Geometry& g
   P.sf_kc4 = g.sf_kc4;
   const size_t smq = (signs ? (size_t)g.n / 8 * 16 : 0) + 128 * 4;
   auto k0 = blk::k_blk128_nvfp4_q<0, blk::kQLanes>;
-  const int grid0 = qblk_grid((const void*)k0, P.units, smq);
+  const int grid0 = qblk_grid((const void*)k0, P.units, smq, blk::kQLanes);
   if (!ws) {
     k0<<<grid0, blk::kQThreads, smq, s>>>(P);
     return cudaGetLastError();
@@ -851,8 +853,8 @@ cudaError_t launch_blk128_nvfp4(const void* x, int64_t tokens, const Geometry& g
     cudaError_t e =
         cudaMemsetAsync(ws, 0, kNvWorkspaceHeader + (size_t)tokens * sizeof(float2), s);
     if (e != cudaSuccess) return e;
-    auto k1 = blk::k_blk128_nvfp4_q<1, blk::kQLanes>;
-    k1<<<qblk_grid((const void*)k1, P.units, smq), blk::kQThreads, smq, s>>>(P);
+    auto k1 = blk::k_blk128_nvfp4_q<1, blk::kQLanesStats>;
+    k1<<<qblk_grid((const void*)k1, P.units, smq, blk::kQLanesStats), blk::kQThreads, smq, s>>>(P);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -866,8 +868,9 @@ cudaError_t launch_blk128_nvfp4(const void* x, int64_t tokens, const Geometry& g
     return cudaGetLastError();
   }
   P.fuse_exact = 1;
+  auto kf = blk::k_blk128_nvfp4_q<0, blk::kQLanesStats>;
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3((unsigned)grid0);
+  cfg.gridDim = dim3((unsigned)qblk_grid((const void*)kf, P.units, smq, blk::kQLanesStats));
   cfg.blockDim = dim3(blk::kQThreads);
   cfg.dynamicSmemBytes = smq;
   cfg.stream = s;
@@ -876,7 +879,7 @@ cudaError_t launch_blk128_nvfp4(const void* x, int64_t tokens, const Geometry& g
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k0, P);
+  return cudaLaunchKernelEx(&cfg, kf, P);
 }
 
 cudaError_t launch_blk128_asym(const void* x, int64_t tokens, const Geometry& g,
