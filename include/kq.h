@@ -194,7 +194,7 @@ KQ_API kq_status kq_rht_quant_int4_kv(const void* x, int dtype, int64_t tokens,
  * KQ_DYN_STATS, KQ_DYN_EXACT and KQ_DYN_QUANT select a subset (none: all
  * three).  When all three run on bf16 rows with block = 128 and at most 8192
  * rows, phases 2 and 3 share one kernel launch (each CTA finds the exact
- * maximum before quantizing); the workspace ends with the same contents.  A tensor split over ranks (QuaRot reviews, final comments: RHT
+ * maximum before quantizing); the workspace then holds the same quantities.  A tensor split over ranks (QuaRot reviews, final comments: RHT
  * per batch of data is data parallelism) gets the tensor scale of the whole
  * tensor by running phase 1 on every rank, an all-reduce(max) of bytes 0-3
  * of every rank's workspace (as int32: a non-negative fp32 orders like its
