@@ -185,6 +185,34 @@ def test_nvfp4_block128_dynamic_tied_rows(tokens):
     P.check_nvfp4(codes, bs, ts, y)
 
 
+def test_nvfp4_block128_dynamic_after_input_write():
+    """The dynamic block-128 call right after a kernel that rewrites its input
+    on the same stream (no synchronisation between them): every call sees the
+    new input.  Its quantisation pass reads inputs before it waits for the
+    statistics pass, which itself starts only after the writer is done."""
+    w = wl.Workload("c2", 300, 4096, wl.BF16, 128, True, wl.NVFP4, 31)
+    a = wl.make_inputs(w)
+    b = wl.make_inputs(wl.Workload("c2", 300, 4096, wl.BF16, 128, True, wl.NVFP4, 32))
+    src = [torch.from_numpy(i.stored.view(np.int16)).cuda().view(torch.bfloat16) for i in (a, b)]
+    want = []
+    for i in (a, b):
+        y = oracle.rht(i.values, a.signs, 128)
+        want.append((y, oracle.nvfp4_tensor_scale(y)))
+    x = torch.empty_like(src[0])
+    s = torch.from_numpy(a.signs).cuda()
+    c, bs, t, ws = kq.empty_nvfp4(w.tokens, w.dim, 128)
+    outs = []
+    for k in (0, 1, 0, 1):
+        x.copy_(src[k])
+        kq.kq_rht_quant_nvfp4(x, 128, s, c, bs, t, ws, dynamic=True)
+        outs.append((k, c.clone(), bs.clone(), t.clone()))
+    torch.cuda.synchronize()
+    for k, cc, bb, tt in outs:
+        y, ts = want[k]
+        assert np.float32(tt.item()) == ts
+        P.check_nvfp4(cc.cpu().numpy(), bb.cpu().numpy(), ts, y)
+
+
 def test_nvfp4_block128_dynamic_many_rows():
     """Dynamic block-128 NVFP4 on more rows than the quantisation pass screens
     for the exact maximum itself (the exact step then runs as a launch of its
