@@ -55,3 +55,19 @@ def test_committed_entries_name_existing_sources():
             assert os.path.exists(os.path.join(ROOT, "hadamard_rotated_activation_b200", "csrc",
                                                name)), (key, name)
         assert set(bench.KERNEL_HEADERS) <= set(e["sources"]), key
+
+
+def test_dynamic_nvfp4_launch_counts():
+    """The per-workload launch counts follow the library's dispatch: bf16
+    block-128 rows up to 8192 run the dynamic scale in two kernels (the exact
+    maximum inside the quantisation pass), other shapes in three."""
+    import bench
+    from hadamard_rotated_activation_b200 import workloads as wl
+    counts = {}
+    for key in ("c2", "c4"):
+        w = wl.WORKLOADS[key]
+        counts[key] = bench.make_step(None, None, w, None, None, None, "dynamic")[2]
+    assert counts == {"c2": 2, "c4": 3}
+    big = wl.WORKLOADS["c2"].with_tokens(8193)
+    assert bench.make_step(None, None, big, None, None, None, "dynamic")[2] == 3
+    assert bench.make_step(None, None, wl.WORKLOADS["c2"], None, None, None, "static")[2] == 1
